@@ -1,0 +1,12 @@
+"""Exact tiled attention for B200 (sm_100a).
+
+``attn_fwd`` / ``attn_bwd`` call the C ABI of ``libattn.so`` (``include/attn.h``)
+on CUDA tensors; PyTorch only allocates device memory and provides the stream.
+Importing the package does not load the CUDA library; the first call does.
+"""
+
+from .api import (attn_bwd, attn_fwd, bwd_workspace_bytes, device_status, set_debug_flags,
+                  set_wait_limit_ns)
+
+__all__ = ["attn_fwd", "attn_bwd", "bwd_workspace_bytes", "device_status",
+           "set_debug_flags", "set_wait_limit_ns"]

@@ -1,0 +1,125 @@
+"""Python entry points over the C ABI (argument marshalling only).
+
+Every step of the computation runs in the CUDA kernels of ``libattn.so``.
+Tensors must already live on a CUDA device; nothing here computes attention,
+and there is no CPU path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import ATTN_BF16, ATTN_FP32, AttnError, AttnTensor
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float32:
+        return ATTN_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or fp32 expected")
+
+
+def _desc(t: torch.Tensor, name: str) -> AttnTensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be [B, H, N, D], got shape {tuple(t.shape)}")
+    if t.stride(3) != 1:
+        raise ValueError(f"{name} must have unit stride on D")
+    sb, sh, sn, _ = t.stride()
+    return AttnTensor(ctypes.c_void_p(t.data_ptr()), sb, sh, sn)
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise AttnError(code, what)
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None):
+    """O, lse = attention(q, k, v): q [B,Hq,N,D], k/v [B,Hkv,N,D] on one CUDA device.
+
+    Returns O (dtype of q) and lse [B,Hq,N] fp32 (natural log).
+    """
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (B, Hq, N):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, N] tensor")
+    L = _lib.lib()
+    code = L.attn_fwd(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(out, "out"),
+                      ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, N, D, _dtype_code(q),
+                      1 if causal else 0, float(scale), _stream(q.device))
+    _check(code, "attn_fwd")
+    return out, lse
+
+
+def bwd_workspace_bytes(B: int, Hq: int, N: int, D: int) -> int:
+    return int(_lib.lib().attn_bwd_workspace_bytes(B, Hq, N, D))
+
+
+def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
+             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None):
+    """dQ, dK, dV of attention from the forward's O and lse and the gradient dO."""
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if dq is None:
+        dq = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if dk is None:
+        dk = torch.empty_like(k, memory_format=torch.contiguous_format)
+    if dv is None:
+        dv = torch.empty_like(v, memory_format=torch.contiguous_format)
+    L = _lib.lib()
+    need = int(L.attn_bwd_workspace_bytes(B, Hq, N, D))
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace too small: {need} bytes needed")
+    if not lse.is_contiguous() or lse.dtype != torch.float32:
+        raise ValueError("lse must be contiguous fp32")
+    code = L.attn_bwd(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(o, "o"),
+                      ctypes.c_void_p(lse.data_ptr()), _desc(do, "do"), _desc(dq, "dq"),
+                      _desc(dk, "dk"), _desc(dv, "dv"), B, Hq, Hkv, N, D, _dtype_code(q),
+                      1 if causal else 0, float(scale), ctypes.c_void_p(workspace.data_ptr()),
+                      ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                      _stream(q.device))
+    _check(code, "attn_bwd")
+    return dq, dk, dv
+
+
+def device_status(device=None):
+    """(status code, wait-site id): syncs the current stream and reads/clears
+    the device status word (0 = no kernel wait timed out)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    where = ctypes.c_int(0)
+    code = _lib.lib().attn_device_status(_stream(dev), ctypes.byref(where))
+    return int(code), int(where.value)
+
+
+def set_wait_limit_ns(ns: int):
+    _lib.lib().attn_debug_set_wait_limit_ns(int(ns))
+
+
+def set_debug_flags(flags: int):
+    _lib.lib().attn_debug_set_flags(int(flags))

@@ -1,0 +1,261 @@
+// C ABI of the exact tiled attention library: argument validation, TMA
+// tensor-map construction, tile-configuration choice by head dimension (the
+// role the "parameter file" keyed by D plays in the FlashAttention (Metal
+// Port) README, Documentation section, here a compile-time table) and kernel
+// launches.  The library allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "bwd.cuh"
+#include "fwd.cuh"
+
+// Device status word: [0] code, [1] wait site, [2..3] block of the first failure.
+__device__ int g_attn_status[4];
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_debug_flags{0};
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+attn_status_t status_ptr(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) return ATTN_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return ATTN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks one [B, H, N, D] tensor: non-null, 16-byte aligned base, strides that
+// are positive (where the dimension has more than one entry) multiples of 16
+// bytes.
+attn_status_t check_tensor(const attn_tensor_t& t, int B, int H, int N, int es) {
+  if (!t.ptr) return ATTN_ERR_INVALID_ARG;
+  if ((B > 1 && t.sb <= 0) || (H > 1 && t.sh <= 0) || (N > 1 && t.sn <= 0))
+    return ATTN_ERR_INVALID_ARG;
+  if (t.sb < 0 || t.sh < 0 || t.sn < 0) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return ATTN_ERR_MISALIGNED;
+  if ((t.sb * es) % 16 || (t.sh * es) % 16 || (t.sn * es) % 16) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+// 4-D TMA map over [B, H, N, D] (innermost first: D, N, H, B), 128-byte
+// swizzle, boxes of (128 bytes of D) x box_rows rows.
+attn_status_t make_map(CUtensorMap* m, const attn_tensor_t& t, int B, int H, int N, int D, int es,
+                       int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  int64_t sn = N > 1 ? t.sn : D;
+  int64_t sh = H > 1 ? t.sh : sn * N;
+  int64_t sb = B > 1 ? t.sb : sh * H;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(sn * es), static_cast<cuuint64_t>(sh * es),
+                           static_cast<cuuint64_t>(sb * es)};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows), 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   4, t.ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename Kernel>
+attn_status_t set_smem(Kernel k, int bytes) {
+  // cudaFuncSetAttribute is cheap and idempotent; the result is per device.
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+attn_status_t last_launch() {
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- forward
+template <typename T, int D, int NS>
+attn_status_t launch_pingpong(const attn_tensor_t& q, const attn_tensor_t& k,
+                              const attn_tensor_t& v, const eta::FwdParams& p, int B, int Hq,
+                              int Hkv, int N, cudaStream_t st) {
+  using C = eta::PingPongCfg<T, D, NS>;
+  CUtensorMap tq, tk, tv;
+  attn_status_t s;
+  if ((s = make_map(&tq, q, B, Hq, N, D, sizeof(T), 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tk, k, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tv, v, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
+  auto kern = eta::fwd_pingpong_kernel<T, D, NS>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
+  dim3 grid((N + 255) / 256, Hq, B);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  return last_launch();
+}
+
+template <int D, int BC, int NS>
+attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, const attn_tensor_t& v,
+                            const eta::FwdParams& p, int B, int Hq, int Hkv, int N,
+                            cudaStream_t st) {
+  using C = eta::SingleCfg<D, BC, NS>;
+  CUtensorMap tq, tk, tv;
+  attn_status_t s;
+  if ((s = make_map(&tq, q, B, Hq, N, D, 2, 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tk, k, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
+  if ((s = make_map(&tv, v, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
+  auto kern = eta::fwd_single_kernel<D, BC, NS>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
+  dim3 grid((N + 127) / 128, Hq, B);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  return last_launch();
+}
+
+attn_status_t check_sizes(int B, int Hq, int Hkv, int N) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+void attn_debug_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs);
+}
+
+void attn_debug_set_flags(int flags) { g_debug_flags.store(flags); }
+
+attn_status_t attn_device_status(void* stream, int* where) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int host[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(host, g_attn_status, sizeof(host)) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero[4] = {0, 0, 0, 0};
+  if (cudaMemcpyToSymbol(g_attn_status, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (where) *where = host[1];
+  if (host[0] == 0) return ATTN_OK;
+  return host[0] == ATTN_ERR_DEVICE_TIMEOUT ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                       float* lse, int B, int Hq, int Hkv, int N, int D, attn_dtype_t dtype,
+                       int causal, float scale, void* stream) {
+  attn_status_t s;
+  if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
+  if (!lse) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
+  const bool bf16 = dtype == ATTN_BF16;
+  if (bf16 ? !(D == 64 || D == 128 || D == 256) : D != 64) return ATTN_ERR_UNSUPPORTED;
+  const int es = bf16 ? 2 : 4;
+  if ((s = check_tensor(q, B, Hq, N, es)) != ATTN_OK) return s;
+  if ((s = check_tensor(k, B, Hkv, N, es)) != ATTN_OK) return s;
+  if ((s = check_tensor(v, B, Hkv, N, es)) != ATTN_OK) return s;
+  if ((s = check_tensor(o, B, Hq, N, es)) != ATTN_OK) return s;
+  if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
+
+  eta::FwdParams p;
+  p.o = o.ptr;
+  p.lse = lse;
+  p.osb = o.sb;
+  p.osh = o.sh;
+  p.osn = o.sn;
+  p.Hq = Hq;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  p.debug_flags = g_debug_flags.load();
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!bf16) return launch_pingpong<float, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+  switch (D) {
+    case 64: return launch_pingpong<__nv_bfloat16, 64, 6>(q, k, v, p, B, Hq, Hkv, N, st);
+    case 128: return launch_pingpong<__nv_bfloat16, 128, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+    default: return launch_single<256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+  }
+}
+
+size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D) {
+  if (B < 1 || Hq < 1 || N < 1 || D < 1) return 0;
+  return eta::bwd_workspace_bytes(B, Hq, N, D);
+}
+
+attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                       const float* lse, attn_tensor_t dout, attn_tensor_t dq, attn_tensor_t dk,
+                       attn_tensor_t dv, int B, int Hq, int Hkv, int N, int D,
+                       attn_dtype_t dtype, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  attn_status_t s;
+  if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
+  if (!lse || !workspace) return !lse ? ATTN_ERR_INVALID_ARG : ATTN_ERR_WORKSPACE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_BF16) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+  if (!(D == 128 || D == 256)) return ATTN_ERR_UNSUPPORTED;
+  const int es = 2;
+  const attn_tensor_t* qs[] = {&q, &o, &dout, &dq};
+  for (auto* t : qs)
+    if ((s = check_tensor(*t, B, Hq, N, es)) != ATTN_OK) return s;
+  const attn_tensor_t* ks[] = {&k, &v, &dk, &dv};
+  for (auto* t : ks)
+    if ((s = check_tensor(*t, B, Hkv, N, es)) != ATTN_OK) return s;
+  if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < eta::bwd_workspace_bytes(B, Hq, N, D)) return ATTN_ERR_WORKSPACE;
+  int* status = nullptr;
+  if ((s = status_ptr(&status)) != ATTN_OK) return s;
+  return eta::launch_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal != 0, scale,
+                         workspace, status, g_wait_limit_ns.load(),
+                         static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,658 @@
+// Forward attention kernels for sm_100a.
+//
+// O = softmax(scale * Q K^T [+ causal mask]) V and lse = log(sum exp(...)),
+// computed tile by tile with an online softmax and deferred normalisation,
+// so the N x N score matrix never leaves the SM (the tiled online softmax of
+// FA1, the query-tile ownership and single final division of FA2, the staged
+// ping-pong pipeline of FA3 and the load / MMA / softmax roles with a
+// conditional rescale of FA4, as listed in the r/mlscaling FlashAttention-
+// PyTorch post; tensor-memory accumulators and asynchronous TMA/MMA pipelines
+// as in the "FlashAttention-4: Algorithm and Kernel Pipelining for Blackwell
+// GPUs" finding on the FlashAttention entity page).
+//
+// Two kernels:
+//  * fwd_pingpong_kernel: one CTA owns two 128-row query tiles of one
+//    (batch, head) and streams 128-row K/V tiles through a TMA ring.  While the
+//    softmax warpgroup of one query tile works, the tensor core runs the other
+//    tile's MMAs.  TMEM: S0 | S1 | O0 | O1.  Used for D*sizeof(T) <= 256 bytes
+//    (bf16 D = 64, 128; fp32/tf32 D = 64).
+//  * fwd_single_kernel: one 128-row query tile, 64-row K/V tiles and a double
+//    buffered S so that S(j+1) = Q K_{j+1}^T runs while row softmax works on
+//    S(j).  TMEM: S0 | S1 | O (D = 256 columns).  Used for bf16 D = 256.
+//
+// Roles (warp-specialised): a TMA producer warp, an MMA warp (one elected
+// thread issues every tcgen05.mma), and 128-thread softmax warpgroups in
+// which thread r owns query row r (TMEM lane r).  The softmax warpgroup also
+// does the correction (rescaling the O row in TMEM when its running maximum
+// grows by more than 2^kRescaleLog2) and the epilogue (O / l, lse).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace eta {
+
+// Rescale O and l only when the running row maximum grows by more than this
+// many powers of two; otherwise keep the stale maximum (results are
+// identical: O and l always share the same reference maximum).
+constexpr float kRescaleLog2 = 8.0f;
+
+struct FwdParams {
+  void* o;           // [B, Hq, N, D], unit stride on D
+  float* lse;        // [B, Hq, N] contiguous
+  long long osb, osh, osn;
+  int Hq, N, group;  // group = Hq / Hkv
+  int causal;
+  float scale;       // softmax scale (natural units)
+  float c;           // scale * log2(e)
+  int* status;       // device status word (4 ints)
+  unsigned long long wait_limit_ns;
+  int debug_flags;   // bit 0: producer skips the first V tile (timeout test)
+};
+
+// Online-softmax update of one row over one tile of BC scores (already masked
+// to -inf where not allowed).  m is the running maximum in raw score units,
+// l the running sum of exp2((s - m) * c).  Converts s in place into
+// p = exp2((s - m) * c).  Returns true when this warp rescaled (alpha != 1
+// for some row of the warp); alpha is this row's factor for O and l.
+template <int BC>
+__device__ __forceinline__ bool online_softmax_step(float (&s)[BC], float c, float& m, float& l,
+                                                    float& alpha) {
+  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+  for (int i = 4; i < BC; i += 4) {
+    mx0 = fmaxf(mx0, s[i]);
+    mx1 = fmaxf(mx1, s[i + 1]);
+    mx2 = fmaxf(mx2, s[i + 2]);
+    mx3 = fmaxf(mx3, s[i + 3]);
+  }
+  const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+  // +inf when m = -inf and m_new is finite; NaN (false) when both are -inf
+  const bool need = (m_new - m) * c > kRescaleLog2;
+  const bool warp_rescale = __any_sync(0xffffffffu, need);
+  alpha = 1.f;
+  if (warp_rescale) {
+    alpha = (m_new == -INFINITY) ? 1.f : ex2((m - m_new) * c);
+    m = m_new;
+    l *= alpha;
+  }
+  const float nmc = (m == -INFINITY) ? 0.f : -m * c;
+  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+  for (int i = 0; i < BC; i += 4) {
+    s[i] = ex2(fmaf(s[i], c, nmc));
+    s[i + 1] = ex2(fmaf(s[i + 1], c, nmc));
+    s[i + 2] = ex2(fmaf(s[i + 2], c, nmc));
+    s[i + 3] = ex2(fmaf(s[i + 3], c, nmc));
+    l0 += s[i];
+    l1 += s[i + 1];
+    l2 += s[i + 2];
+    l3 += s[i + 3];
+  }
+  l += (l0 + l1) + (l2 + l3);
+  return warp_rescale;
+}
+
+// Loads BC consecutive fp32 TMEM columns of this thread's lane into s.
+template <int BC>
+__device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&s)[BC]) {
+  static_assert(BC % 32 == 0, "row chunks of 32 columns");
+#pragma unroll
+  for (int c = 0; c < BC / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 32 * c, r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s[32 * c + i] = u2f(r[i]);
+  }
+  tmem_wait_ld();
+}
+
+// Writes p (BC values) back into TMEM as the A operand of the P V MMA:
+// bf16 pairs packed per 32-bit column (BC/2 columns) or fp32 (BC columns).
+template <int BC, bool TF32>
+__device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&p)[BC]) {
+  if constexpr (TF32) {
+#pragma unroll
+    for (int c = 0; c < BC / 32; ++c) {
+      uint32_t r[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(p[32 * c + i]);
+      tmem_st32(taddr + 32 * c, r);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < BC / 64; ++c) {
+      uint32_t r[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = pack_bf16x2(p[64 * c + 2 * i], p[64 * c + 2 * i + 1]);
+      tmem_st32(taddr + 32 * c, r);
+    }
+    if constexpr (BC % 64 == 32) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) r[i] = pack_bf16x2(p[BC - 32 + 2 * i], p[BC - 32 + 2 * i + 1]);
+      tmem_st16(taddr + BC / 2 - 16, r);
+    }
+  }
+}
+
+// Multiplies DC fp32 TMEM columns of this lane by alpha (the correction step).
+template <int DC>
+__device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < DC / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 32 * c, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(u2f(r[i]) * alpha);
+    tmem_st32(taddr + 32 * c, r);
+  }
+}
+
+// Epilogue of one row: O = O_acc / l written to global memory as T, lse.
+template <typename T, int D>
+__device__ __forceinline__ void store_row(uint32_t o_taddr, const FwdParams& p, int b, int h,
+                                          int qrow, float m, float l) {
+  const bool valid = qrow < p.N;
+  const float inv_l = 1.f / l;
+  char* row = static_cast<char*>(p.o) +
+              (static_cast<long long>(b) * p.osb + static_cast<long long>(h) * p.osh +
+               static_cast<long long>(qrow) * p.osn) *
+                  static_cast<long long>(sizeof(T));
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(o_taddr + 32 * c, r);
+    tmem_wait_ld();
+    if (valid) {
+      if constexpr (sizeof(T) == 2) {
+        uint4* dst = reinterpret_cast<uint4*>(row + 64 * c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 w;
+          w.x = pack_bf16x2(u2f(r[8 * v + 0]) * inv_l, u2f(r[8 * v + 1]) * inv_l);
+          w.y = pack_bf16x2(u2f(r[8 * v + 2]) * inv_l, u2f(r[8 * v + 3]) * inv_l);
+          w.z = pack_bf16x2(u2f(r[8 * v + 4]) * inv_l, u2f(r[8 * v + 5]) * inv_l);
+          w.w = pack_bf16x2(u2f(r[8 * v + 6]) * inv_l, u2f(r[8 * v + 7]) * inv_l);
+          dst[v] = w;
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(row + 128 * c);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(u2f(r[4 * v]) * inv_l, u2f(r[4 * v + 1]) * inv_l,
+                               u2f(r[4 * v + 2]) * inv_l, u2f(r[4 * v + 3]) * inv_l);
+      }
+    }
+  }
+  if (valid)
+    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = m * p.scale + logf(l);
+}
+
+// Column limit of one row in one key tile: columns >= lim are masked.
+__device__ __forceinline__ int col_limit(int kbase, int qrow, int N, int causal, int BC) {
+  int lim = N - kbase;
+  if (causal) lim = min(lim, qrow - kbase + 1);
+  return min(lim, BC);
+}
+
+template <int BC>
+__device__ __forceinline__ void apply_mask(float (&s)[BC], int lim) {
+  if (lim < BC) {
+#pragma unroll
+    for (int i = 0; i < BC; ++i)
+      if (i >= lim) s[i] = -INFINITY;
+  }
+}
+
+// =====================================================================
+// Two query tiles per CTA (ping-pong).
+// =====================================================================
+template <typename T, int D, int NS>
+struct PingPongCfg {
+  static constexpr bool TF32 = sizeof(T) == 4;
+  static constexpr int ES = sizeof(T);
+  static constexpr int ROWB = D * ES;        // bytes per row
+  static constexpr int NCHUNK = ROWB / 128;  // 128-byte swizzle chunks per row
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int CHUNK = 128 * 128;    // bytes of one chunk of a 128-row tile
+  static constexpr int TILE = 128 * ROWB;
+  static constexpr int QK_STEPS = ROWB / 32;
+  static constexpr int PV_ROWS = 32 / ES;    // V rows consumed per MMA
+  static constexpr int PV_STEPS = BN / PV_ROWS;
+  static constexpr int O_COL = 256;          // O0 at 256, O1 at 256 + D
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_KV = 2 * TILE;
+  static constexpr int SMEM_BAR = SMEM_KV + NS * TILE;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_full[2], done
+  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_KVF = 1;
+  static constexpr int BAR_KVE = 1 + NS;
+  static constexpr int BAR_S = 1 + 2 * NS;
+  static constexpr int BAR_P = 3 + 2 * NS;
+  static constexpr int BAR_O = 5 + 2 * NS;
+  static constexpr int BAR_DONE = 7 + 2 * NS;
+  static constexpr int NBAR = 8 + 2 * NS;
+  static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;  // tmem slot, abort flag
+  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int THREADS = 384;
+  static_assert(ROWB % 128 == 0, "row must be whole 128-byte chunks");
+  static_assert(256 + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <typename T, int D, int NS>
+__global__ void __launch_bounds__(384, 1)
+    fwd_pingpong_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = PingPongCfg<T, D, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::SMEM_BAR;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = gridDim.x - 1 - blockIdx.x;  // longest causal CTAs first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.group;
+  const int q0 = qb * 256;
+  int ntile[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qs = q0 + 128 * t;
+    const int kv_end = p.causal ? min(p.N, qs + 128) : p.N;
+    ntile[t] = qs < p.N ? (kv_end + 127) / 128 : 0;
+  }
+  const int nK = max(ntile[0], ntile[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::BAR_Q), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(BAR(C::BAR_KVF + s), 1);
+      mbar_init(BAR(C::BAR_KVE + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR(C::BAR_S + t), 1);
+      mbar_init(BAR(C::BAR_P + t), 4);
+      mbar_init(BAR(C::BAR_O + t), 1);
+    }
+    mbar_init(BAR(C::BAR_DONE), 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+
+  if (warp < 8) {
+    // ------------------------------------------------ softmax / correction / epilogue
+    const int t = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const int qrow = q0 + 128 * t + r;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + 128u * t;
+    const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntile[t]; ++j) {
+      if (!W.wait_warp(BAR(C::BAR_S + t), j & 1, 10 + t)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+      tmem_load_row<128>(s_addr, s);
+      apply_mask<128>(s, col_limit(128 * j, qrow, p.N, p.causal, 128));
+      float alpha;
+      const bool rescaled = online_softmax_step<128>(s, p.c, m, l, alpha);
+      tmem_store_p<128, C::TF32>(s_addr, s);
+      if (rescaled && j > 0) tmem_scale_row<D>(o_addr, alpha);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::BAR_P + t));
+    }
+    if (ok && ntile[t] > 0 && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
+      tc_fence_after();
+      store_row<T, D>(o_addr, p, b, h, qrow, m, l);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      constexpr int EPC = 128 / C::ES;  // elements per 128-byte chunk
+      mbar_expect_tx(BAR(C::BAR_Q), 2 * C::TILE);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sbase + C::SMEM_Q + t * C::TILE + c * C::CHUNK, &tm_q, BAR(C::BAR_Q), c * EPC,
+                      q0 + 128 * t, h, b);
+      int it = 0;
+      for (int j = 0; j < nK && !W.aborted(); ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int slot = it % NS;
+          const uint32_t ph = static_cast<uint32_t>(it / NS) & 1u;
+          if (!W.wait(BAR(C::BAR_KVE + slot), ph ^ 1u, 30)) break;
+          if ((p.debug_flags & 1) && kv == 1 && j == 0) continue;  // fault injection: drop V_0
+          mbar_expect_tx(BAR(C::BAR_KVF + slot), C::TILE);
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_4d(sbase + C::SMEM_KV + slot * C::TILE + c * C::CHUNK, kv ? &tm_v : &tm_k,
+                        BAR(C::BAR_KVF + slot), c * EPC, 128 * j, hk, b);
+        }
+      }
+      // Let every copy this warp started land before the CTA can exit.
+      const int issued = it;
+      W.drain(BAR(C::BAR_Q), 0, 31);
+      for (int s = 0; s < NS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NS) * NS;  // last load into slot s
+        W.drain(BAR(C::BAR_KVF + s), static_cast<uint32_t>(last / NS) & 1u, 32);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = C::TF32 ? 2u : 1u;
+      constexpr uint32_t idesc_s = idesc_make(128, 128, fmt, false, false);
+      constexpr uint32_t idesc_o = idesc_make(128, D, fmt, false, true);
+      auto kslot = [&](int j) { return (2 * j) % NS; };
+      auto kph = [&](int j) { return static_cast<uint32_t>((2 * j) / NS) & 1u; };
+      auto vslot = [&](int j) { return (2 * j + 1) % NS; };
+      auto vph = [&](int j) { return static_cast<uint32_t>((2 * j + 1) / NS) & 1u; };
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = sbase + C::SMEM_Q + t * C::TILE;
+        const uint32_t kb = sbase + C::SMEM_KV + slot * C::TILE;
+#pragma unroll
+        for (int ks = 0; ks < C::QK_STEPS; ++ks) {
+          const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+          mma_ss<C::TF32>(tmem + 128u * t, sdesc_sw128(qa + off, 16, 1024),
+                          sdesc_sw128(kb + off, 16, 1024), idesc_s, ks > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t vb = sbase + C::SMEM_KV + slot * C::TILE;
+#pragma unroll
+        for (int ks = 0; ks < C::PV_STEPS; ++ks)
+          mma_ts<C::TF32>(tmem + C::O_COL + D * t, tmem + 128u * t + 8u * ks,
+                          sdesc_sw128(vb + ks * C::PV_ROWS * 128, C::CHUNK, 1024), idesc_o,
+                          (acc || ks > 0) ? 1u : 0u);
+      };
+      const int n0 = ntile[0], n1 = ntile[1];
+      bool ok = W.wait(BAR(C::BAR_Q), 0, 40) && W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
+      if (ok) {
+        tc_fence_after();
+        if (n0 > 0) { issue_s(0, kslot(0)); mma_commit(BAR(C::BAR_S + 0)); }
+        if (n1 > 0) { issue_s(1, kslot(0)); mma_commit(BAR(C::BAR_S + 1)); }
+        mma_commit(BAR(C::BAR_KVE + kslot(0)));
+      }
+      for (int j = 0; ok && j < nK; ++j) {
+        const bool use0 = j < n0, use1 = j < n1;
+        const bool nxt0 = j + 1 < n0, nxt1 = j + 1 < n1;
+        if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 42)) { ok = false; break; }
+        if (use0) {
+          if (!W.wait(BAR(C::BAR_P + 0), j & 1, 43)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, vslot(j), j > 0);
+          if (!use1) mma_commit(BAR(C::BAR_KVE + vslot(j)));
+          if (nxt0) {
+            if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 44)) { ok = false; break; }
+            issue_s(0, kslot(j + 1));
+            mma_commit(BAR(C::BAR_S + 0));
+            if (!nxt1) mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
+          } else {
+            mma_commit(BAR(C::BAR_O + 0));
+          }
+        }
+        if (use1) {
+          if (!W.wait(BAR(C::BAR_P + 1), j & 1, 45)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, vslot(j), j > 0);
+          mma_commit(BAR(C::BAR_KVE + vslot(j)));
+          if (nxt1) {
+            if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 46)) { ok = false; break; }
+            issue_s(1, kslot(j + 1));
+            mma_commit(BAR(C::BAR_S + 1));
+            mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
+          } else {
+            mma_commit(BAR(C::BAR_O + 1));
+          }
+        }
+      }
+      // Wait until every MMA this thread issued has finished with TMEM/smem.
+      mma_commit(BAR(C::BAR_DONE));
+      W.drain(BAR(C::BAR_DONE), 0, 47);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// =====================================================================
+// One query tile per CTA, double-buffered S (large head dimension).
+// =====================================================================
+template <int D, int BC, int NS>
+struct SingleCfg {
+  static constexpr int ES = 2;
+  static constexpr int ROWB = D * ES;
+  static constexpr int NCHUNK = ROWB / 128;
+  static constexpr int QCHUNK = 128 * 128;   // chunk of the 128-row Q tile
+  static constexpr int KCHUNK = BC * 128;    // chunk of a BC-row K/V tile
+  static constexpr int QTILE = 128 * ROWB;
+  static constexpr int KTILE = BC * ROWB;
+  static constexpr int QK_STEPS = ROWB / 32;
+  static constexpr int PV_STEPS = BC / 16;
+  static constexpr int S_COL = 0;            // S buffers at 0 and BC
+  static constexpr int O_COL = 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_KV = QTILE;
+  static constexpr int SMEM_BAR = SMEM_KV + NS * KTILE;
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full, pv_done, o_full, done
+  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_KVF = 1;
+  static constexpr int BAR_KVE = 1 + NS;
+  static constexpr int BAR_S = 1 + 2 * NS;
+  static constexpr int BAR_P = 3 + 2 * NS;
+  static constexpr int BAR_PV = 4 + 2 * NS;
+  static constexpr int BAR_O = 5 + 2 * NS;
+  static constexpr int BAR_DONE = 6 + 2 * NS;
+  static constexpr int NBAR = 7 + 2 * NS;
+  static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
+  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
+  static constexpr int THREADS = 256;
+  static_assert(2 * BC <= O_COL && O_COL + D <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int D, int BC, int NS>
+__global__ void __launch_bounds__(256, 1)
+    fwd_single_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = SingleCfg<D, BC, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::SMEM_BAR;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = gridDim.x - 1 - blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.group;
+  const int q0 = qb * 128;
+  const int kv_end = p.causal ? min(p.N, q0 + 128) : p.N;
+  const int n = (kv_end + BC - 1) / BC;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::BAR_Q), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(BAR(C::BAR_KVF + s), 1);
+      mbar_init(BAR(C::BAR_KVE + s), 1);
+    }
+    mbar_init(BAR(C::BAR_S + 0), 1);
+    mbar_init(BAR(C::BAR_S + 1), 1);
+    mbar_init(BAR(C::BAR_P), 4);
+    mbar_init(BAR(C::BAR_PV), 1);
+    mbar_init(BAR(C::BAR_O), 1);
+    mbar_init(BAR(C::BAR_DONE), 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+
+  if (warp < 4) {
+    const int r = threadIdx.x & 127;
+    const int qrow = q0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t o_addr = tmem + lane_base + C::O_COL;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int buf = j & 1;
+      const uint32_t s_addr = tmem + lane_base + C::S_COL + BC * buf;
+      if (!W.wait_warp(BAR(C::BAR_S + buf), (j >> 1) & 1, 10)) { ok = false; break; }
+      tc_fence_after();
+      float s[BC];
+      tmem_load_row<BC>(s_addr, s);
+      apply_mask<BC>(s, col_limit(BC * j, qrow, p.N, p.causal, BC));
+      float alpha;
+      const bool rescaled = online_softmax_step<BC>(s, p.c, m, l, alpha);
+      tmem_store_p<BC, false>(s_addr, s);
+      if (rescaled && j > 0) {
+        // O must hold every P V product up to tile j-1 before it is rescaled.
+        if (!W.wait_warp(BAR(C::BAR_PV), (j - 1) & 1, 11)) { ok = false; break; }
+        tc_fence_after();
+        tmem_scale_row<D>(o_addr, alpha);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::BAR_P));
+    }
+    if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
+      tc_fence_after();
+      store_row<__nv_bfloat16, D>(o_addr, p, b, h, qrow, m, l);
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(BAR(C::BAR_Q), C::QTILE);
+      for (int c = 0; c < C::NCHUNK; ++c)
+        tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * 64, q0, h, b);
+      int it = 0;
+      for (int j = 0; j < n && !W.aborted(); ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int slot = it % NS;
+          const uint32_t ph = static_cast<uint32_t>(it / NS) & 1u;
+          if (!W.wait(BAR(C::BAR_KVE + slot), ph ^ 1u, 30)) break;
+          if ((p.debug_flags & 1) && kv == 1 && j == 0) continue;
+          mbar_expect_tx(BAR(C::BAR_KVF + slot), C::KTILE);
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_4d(sbase + C::SMEM_KV + slot * C::KTILE + c * C::KCHUNK, kv ? &tm_v : &tm_k,
+                        BAR(C::BAR_KVF + slot), c * 64, BC * j, hk, b);
+        }
+      }
+      const int issued = it;
+      W.drain(BAR(C::BAR_Q), 0, 31);
+      for (int s = 0; s < NS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NS) * NS;
+        W.drain(BAR(C::BAR_KVF + s), static_cast<uint32_t>(last / NS) & 1u, 32);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_make(128, BC, 1u, false, false);
+      constexpr uint32_t idesc_o = idesc_make(128, D, 1u, false, true);
+      auto kslot = [&](int j) { return (2 * j) % NS; };
+      auto kph = [&](int j) { return static_cast<uint32_t>((2 * j) / NS) & 1u; };
+      auto vslot = [&](int j) { return (2 * j + 1) % NS; };
+      auto vph = [&](int j) { return static_cast<uint32_t>((2 * j + 1) / NS) & 1u; };
+      auto issue_s = [&](int buf, int slot) {
+        const uint32_t qa = sbase + C::SMEM_Q;
+        const uint32_t kb = sbase + C::SMEM_KV + slot * C::KTILE;
+#pragma unroll
+        for (int ks = 0; ks < C::QK_STEPS; ++ks) {
+          const uint32_t qoff = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
+          const uint32_t koff = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
+          mma_ss<false>(tmem + C::S_COL + BC * buf, sdesc_sw128(qa + qoff, 16, 1024),
+                        sdesc_sw128(kb + koff, 16, 1024), idesc_s, ks > 0);
+        }
+      };
+      auto issue_pv = [&](int buf, int slot, bool acc) {
+        const uint32_t vb = sbase + C::SMEM_KV + slot * C::KTILE;
+#pragma unroll
+        for (int ks = 0; ks < C::PV_STEPS; ++ks)
+          mma_ts<false>(tmem + C::O_COL, tmem + C::S_COL + BC * buf + 8u * ks,
+                        sdesc_sw128(vb + ks * 16 * 128, C::KCHUNK, 1024), idesc_o,
+                        (acc || ks > 0) ? 1u : 0u);
+      };
+      bool ok = W.wait(BAR(C::BAR_Q), 0, 40) && W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, kslot(0));
+        mma_commit(BAR(C::BAR_S + 0));
+        mma_commit(BAR(C::BAR_KVE + kslot(0)));
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n) {
+          if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 42)) { ok = false; break; }
+          issue_s((j + 1) & 1, kslot(j + 1));
+          mma_commit(BAR(C::BAR_S + ((j + 1) & 1)));
+          mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
+        }
+        if (!W.wait(BAR(C::BAR_P), j & 1, 43)) { ok = false; break; }
+        if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 44)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(j & 1, vslot(j), j > 0);
+        mma_commit(BAR(C::BAR_PV));
+        mma_commit(BAR(C::BAR_KVE + vslot(j)));
+      }
+      if (ok) mma_commit(BAR(C::BAR_O));
+      mma_commit(BAR(C::BAR_DONE));
+      W.drain(BAR(C::BAR_DONE), 0, 47);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace eta

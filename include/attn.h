@@ -1,0 +1,141 @@
+/*
+ * Exact tiled attention for NVIDIA B200 (sm_100a) -- C ABI.
+ *
+ * The operation (r/mlscaling, FlashAttention-PyTorch post: every generation
+ * FA1..FA4 keeps "the same exact attention math"; FlashAttention entity
+ * page, finding "FlashAttention-4: Algorithm and Kernel Pipelining for
+ * Blackwell GPUs"; FlashAttention (Metal Port) README, Documentation section,
+ * for the recompute-based backward with its scratch for atomics and partial
+ * sums):
+ *
+ *   forward   S = scale * Q K^T, S[i][j] = -inf for j > i when causal,
+ *             P = row-softmax(S), O = P V, lse[i] = ln(sum_j exp(S[i][j]))
+ *   backward  dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)),
+ *             dQ = scale dS K, dK = scale dS^T Q, with P recomputed from lse
+ *
+ * Grouped-query attention: query head h reads key/value head h / (Hq / Hkv)
+ * (contiguous groups); dK and dV sum over the group.
+ *
+ * Tensors.  Every Q/K/V/O/dO/dQ/dK/dV tensor is a 4-D [B, H, N, D] array
+ * described by an attn_tensor_t: a device pointer and the element strides of
+ * the B, H and N dimensions; the D dimension has unit stride.  H is Hq for
+ * Q, O, dO, dQ and Hkv for K, V, dK, dV.  lse is a contiguous fp32
+ * [B, Hq, N] device array.  All pointers are device pointers owned by the
+ * caller; the library allocates no device memory and keeps no pointer after
+ * a call returns.
+ *
+ * Requirements (checked before anything is launched; a violation returns an
+ * error code and launches nothing):
+ *   B, Hq, Hkv, N >= 1; Hq % Hkv == 0; D in {64, 128, 256};
+ *   every pointer 16-byte aligned and every stride a multiple of 16 bytes
+ *   (the tensor-memory-accelerator rule);
+ *   ATTN_FP32 (fp32 storage, tf32 tensor-core products) only for the forward
+ *   with D = 64; the backward supports bf16 with D in {128, 256}.
+ *
+ * Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ * default stream).  The return value reports host-side validation and launch
+ * errors only.  A kernel whose internal wait times out (it never hangs: each
+ * wait is bounded) records ATTN_ERR_DEVICE_TIMEOUT in a device status word
+ * that attn_device_status() reads.
+ */
+#ifndef EXACT_TILED_ATTENTION_ATTN_H_
+#define EXACT_TILED_ATTENTION_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+typedef struct attn_tensor {
+  void* ptr;   /* device pointer to element [0, 0, 0, 0] */
+  int64_t sb;  /* element stride of the batch dimension */
+  int64_t sh;  /* element stride of the head dimension */
+  int64_t sn;  /* element stride of the sequence dimension */
+} attn_tensor_t;
+
+typedef enum attn_dtype {
+  ATTN_BF16 = 0, /* bf16 storage, fp32 accumulation */
+  ATTN_FP32 = 1  /* fp32 storage, tf32 products, fp32 accumulation */
+} attn_dtype_t;
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, Hq % Hkv != 0 */
+  ATTN_ERR_UNSUPPORTED = 2,    /* head dim / dtype / direction not built */
+  ATTN_ERR_MISALIGNED = 3,     /* pointer or stride breaks the 16-byte rule */
+  ATTN_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+  ATTN_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
+  ATTN_ERR_DEVICE_TIMEOUT = 6  /* a kernel's bounded wait gave up (device status) */
+} attn_status_t;
+
+/* ABI version of the loaded library (ATTN_ABI_VERSION). */
+ATTN_API int attn_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+ATTN_API const char* attn_status_string(attn_status_t status);
+
+/*
+ * Forward.  Reads q [B,Hq,N,D], k and v [B,Hkv,N,D]; writes o [B,Hq,N,D]
+ * (same dtype as the inputs) and lse [B,Hq,N] (fp32, natural log of the sum
+ * of exp of the scaled, masked scores).  causal != 0 applies the top-left
+ * causal mask (key j visible to query i iff j <= i).  scale multiplies
+ * q.k (1/sqrt(D) is the usual choice).  o must not alias q, k or v.
+ */
+ATTN_API attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                       float* lse, int B, int Hq, int Hkv, int N, int D, attn_dtype_t dtype,
+                       int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs for these sizes: an fp32 dQ
+ * accumulator [B,Hq,N,D] (the scratch the backward's atomic partial sums go
+ * to) plus two fp32 row statistics [B,Hq,N'] (rowsum(dO*O) and lse*log2(e),
+ * N' = N rounded up to 64).  Returns 0 for invalid sizes.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D);
+
+/*
+ * Backward.  Reads q, k, v, the forward's o and lse, and the upstream
+ * gradient dout [B,Hq,N,D]; writes dq [B,Hq,N,D], dk and dv [B,Hkv,N,D]
+ * (bf16).  workspace: device memory of at least attn_bwd_workspace_bytes()
+ * bytes, 256-byte aligned, owned by the caller; its contents on entry do not
+ * matter and are overwritten.  Outputs must not alias inputs.
+ */
+ATTN_API attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                       const float* lse, attn_tensor_t dout, attn_tensor_t dq, attn_tensor_t dk,
+                       attn_tensor_t dv, int B, int Hq, int Hkv, int N, int D,
+                       attn_dtype_t dtype, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a kernel's
+ * bounded wait gave up; *where, if not NULL, receives the wait site id) or
+ * ATTN_ERR_CUDA.
+ */
+ATTN_API attn_status_t attn_device_status(void* stream, int* where);
+
+/*
+ * Test hooks.  attn_debug_set_wait_limit_ns sets the time limit of every
+ * in-kernel wait (default 2 s; 0 restores the default).
+ * attn_debug_set_flags: bit 0 makes the next forward launches drop one tile
+ * load, so that their waits run out and report ATTN_ERR_DEVICE_TIMEOUT
+ * through attn_device_status (0 = normal operation).
+ */
+ATTN_API void attn_debug_set_wait_limit_ns(unsigned long long ns);
+ATTN_API void attn_debug_set_flags(int flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_TILED_ATTENTION_ATTN_H_ */

@@ -9,3 +9,14 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: full-size workloads (minutes)")
+
+
+def pytest_collection_modifyitems(config, items):
+    import pytest
+    import torch
+    if torch.cuda.is_available():
+        return
+    skip = pytest.mark.skip(reason="needs a CUDA device (run with -m gpu on a B200)")
+    for item in items:
+        if "gpu" in item.keywords:
+            item.add_marker(skip)

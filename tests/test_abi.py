@@ -1,0 +1,107 @@
+"""CPU checks of the C ABI: the library builds, loads and exports every
+function ``include/attn.h`` declares; host-side validation rejects bad
+arguments with the documented status codes before touching the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_tiled_attention_37_b200 import _lib, build
+
+HEADER = os.path.join(build.ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    names = set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_device_status",
+              "attn_status_string", "attn_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_functions():
+        assert hasattr(L, n), f"{n} declared in attn.h but not exported"
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.attn_abi_version() == 1
+    for code in range(7):
+        assert L.attn_status_string(code)
+
+
+def test_workspace_size(L):
+    B, H, N, D = 2, 16, 4096, 128
+    got = L.attn_bwd_workspace_bytes(B, H, N, D)
+    assert got >= B * H * N * D * 4 + 2 * B * H * N * 4
+    assert L.attn_bwd_workspace_bytes(0, H, N, D) == 0
+
+
+def _t(ptr, sb, sh, sn):
+    return _lib.AttnTensor(ctypes.c_void_p(ptr), sb, sh, sn)
+
+
+def _fwd(L, B=1, Hq=2, Hkv=1, N=256, D=128, dt=0, ptr=0x10000, lse=0x20000, scale=0.1,
+         sn=None, qptr=None):
+    sn = D if sn is None else sn
+    t = _t(ptr, Hq * N * sn, N * sn, sn)
+    q = _t(qptr if qptr is not None else ptr, Hq * N * sn, N * sn, sn)
+    kv = _t(ptr, Hkv * N * sn, N * sn, sn)
+    return L.attn_fwd(q, kv, kv, t, ctypes.c_void_p(lse), B, Hq, Hkv, N, D, dt, 0, scale, None)
+
+
+def test_fwd_validation_codes(L):
+    assert _fwd(L, Hq=3, Hkv=2) == 1           # Hq % Hkv
+    assert _fwd(L, N=0) == 1                   # empty sequence
+    assert _fwd(L, B=0) == 1
+    assert _fwd(L, ptr=0) == 1                 # null
+    assert _fwd(L, lse=0) == 1
+    assert _fwd(L, scale=0.0) == 1
+    assert _fwd(L, scale=float("nan")) == 1
+    assert _fwd(L, D=96) == 2                  # head dim not built
+    assert _fwd(L, D=128, dt=1) == 2           # fp32 only at D=64
+    assert _fwd(L, qptr=0x10008) == 3          # misaligned base
+    assert _fwd(L, sn=132) == 3                # row stride not a multiple of 16 bytes
+    assert _fwd(L, lse=0x20004) == 3
+
+
+def test_bwd_validation_codes(L):
+    B, Hq, Hkv, N, D = 1, 2, 1, 256, 128
+    q = _t(0x10000, Hq * N * D, N * D, D)
+    kv = _t(0x10000, Hkv * N * D, N * D, D)
+    ws = L.attn_bwd_workspace_bytes(B, Hq, N, D)
+    lse = ctypes.c_void_p(0x20000)
+
+    def call(D=D, ws_ptr=0x40000, ws_bytes=ws, dt=0, lse=lse):
+        return L.attn_bwd(q, kv, kv, q, lse, q, q, kv, kv, B, Hq, Hkv, N, D, dt, 1, 0.1,
+                          ctypes.c_void_p(ws_ptr), ws_bytes, None)
+
+    assert call(ws_ptr=0) == 4
+    assert call(ws_bytes=ws - 1) == 4
+    assert call(ws_ptr=0x40010) == 3           # workspace must be 256-byte aligned
+    assert call(D=64) == 2
+    assert call(dt=1) == 2
+    assert call(lse=ctypes.c_void_p(0)) == 1
+
+
+def test_python_api_refuses_cpu_tensors():
+    import torch
+    from exact_tiled_attention_37_b200 import attn_fwd
+    q = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        attn_fwd(q, q, q)

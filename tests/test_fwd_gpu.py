@@ -1,0 +1,163 @@
+"""Forward parity: the CUDA kernels (through the C ABI) against the fp64 oracle
+on the same seeded inputs.
+
+Small problems are compared element by element over every output; they span
+several 128-row tiles and a ragged tail, both mask modes, grouped-query heads
+and strided (non-contiguous) views.  The named workloads run at full size in
+the launch configuration the benchmark times; where the oracle cannot redo
+all of them in seconds, sampled heads and rows are compared one by one.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_37_b200 import attn_fwd, device_status
+from exact_tiled_attention_37_b200.inputs import make_inputs, make_random, workload
+
+from ._util import TOL_LSE, TOL_REL, abs_err, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_fwd(q, k, v, causal, scale=None):
+    o, lse = attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    code, where = device_status()
+    assert code == 0, f"device status {code} at wait site {where}"
+    return o, lse
+
+
+def check_full(q, k, v, causal, scale=None, tol=TOL_REL):
+    D = q.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o, lse = run_fwd(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention_fwd(q.float().numpy(), k.float().numpy(),
+                                          v.float().numpy(), causal, scale)
+    eo, el = rel_err(to_np(o), o_ref), abs_err(to_np(lse), lse_ref)
+    assert eo <= tol and el <= TOL_LSE, (eo, el)
+    return eo, el
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 128, 200, 256, 300, 640])
+def test_small_shapes(D, causal, N):
+    q, k, v = make_random(1, 2, 2, N, D, "bf16", seed=N * 10 + D + causal, with_do=False)
+    check_full(q, k, v, causal)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hq,hkv", [(4, 1), (4, 2), (8, 2)])
+def test_grouped_query_heads(D, causal, hq, hkv):
+    q, k, v = make_random(2, hq, hkv, 333, D, "bf16", seed=hq * 7 + hkv + D, with_do=False)
+    check_full(q, k, v, causal)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_strided_views(D):
+    # [B, N, H, D] storage viewed as [B, H, N, D]: non-contiguous head/seq strides
+    B, H, N = 2, 3, 300
+    g = torch.Generator().manual_seed(5 + D)
+    base = [torch.randn(B, N, H, D, generator=g).to(torch.bfloat16) for _ in range(3)]
+    q, k, v = (t.to(DEV).transpose(1, 2) for t in base)
+    assert not q.is_contiguous()
+    for causal in (False, True):
+        o, lse = attn_fwd(q, k, v, causal=causal)
+        o_ref, lse_ref = oracle.attention_fwd(*(to_np(t) for t in (q, k, v)), causal,
+                                              1 / math.sqrt(D))
+        assert rel_err(to_np(o), o_ref) <= TOL_REL
+        assert abs_err(to_np(lse), lse_ref) <= TOL_LSE
+
+
+def test_output_into_strided_buffer():
+    B, H, N, D = 1, 2, 256, 128
+    q, k, v = (t.to(DEV) for t in make_random(B, H, H, N, D, "bf16", seed=3, with_do=False))
+    big = torch.zeros(B, N, H, 2 * D, device=DEV, dtype=torch.bfloat16)
+    out = big[..., :D].transpose(1, 2)
+    attn_fwd(q, k, v, causal=True, out=out)
+    o_ref, _ = oracle.attention_fwd(to_np(q), to_np(k), to_np(v), True, 1 / math.sqrt(D))
+    assert rel_err(to_np(out), o_ref) <= TOL_REL
+    assert torch.all(big[..., D:] == 0), "kernel wrote outside the output view"
+
+
+def test_scale_and_sharp_softmax():
+    # large scores exercise the conditional rescale (running max grows a lot)
+    q, k, v = make_random(1, 2, 2, 1000, 128, "bf16", seed=77, k_mult=6.0, with_do=False)
+    for causal in (False, True):
+        check_full(q, k, v, causal, scale=0.3)
+
+
+def test_increasing_scores_force_rescales():
+    # scores grow along the key axis so every tile raises the row maximum
+    N, D = 1024, 64
+    q = torch.zeros(1, 1, N, D)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, 1, N, D)
+    k[..., 0] = torch.linspace(0, 60, N)
+    v = torch.randn(1, 1, N, D, generator=torch.Generator().manual_seed(1))
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    for causal in (False, True):
+        check_full(q, k, v, causal, scale=1.0)
+
+
+def test_deterministic():
+    q, k, v = (t.to(DEV) for t in make_random(2, 4, 2, 777, 128, "bf16", seed=9, with_do=False))
+    o1, l1 = attn_fwd(q, k, v, causal=True)
+    o2, l2 = attn_fwd(q, k, v, causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ------------------------------------------------------------ named workloads
+
+
+def test_workload_single_head_fp32():
+    w = workload(0)
+    q, k, v = make_inputs(w, with_do=False)
+    assert q.dtype == torch.float32
+    check_full(q, k, v, False)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_workload_mha_2048(causal):
+    w = workload(1)
+    q, k, v = make_inputs(w, with_do=False)
+    check_full(q, k, v, causal)
+
+
+def _sampled(w, causal, heads, nrows, seed):
+    q, k, v = make_inputs(w, with_do=False)
+    o, lse = run_fwd(q, k, v, causal)
+    rng = np.random.default_rng(seed)
+    worst_o, worst_l = 0.0, 0.0
+    for (b, h) in heads:
+        rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1],
+                                         rng.integers(0, w.N, nrows)]))
+        o_ref, l_ref = oracle.attention_fwd_rows(q.float().numpy(), k.float().numpy(),
+                                                 v.float().numpy(), causal, w.scale, b, h, rows)
+        og = o[b, h, torch.as_tensor(rows, device=DEV)]
+        lg = lse[b, h, torch.as_tensor(rows, device=DEV)]
+        worst_o = max(worst_o, rel_err(to_np(og), o_ref))
+        worst_l = max(worst_l, abs_err(to_np(lg), l_ref))
+    assert worst_o <= TOL_REL and worst_l <= TOL_LSE, (worst_o, worst_l)
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+def test_workload_mha_4096_causal():
+    w = workload(2)
+    _sampled(w, True, [(0, 0), (1, 15), (0, 7)], 200, 1)
+
+
+def test_workload_long_context_gqa():
+    w = workload(3)
+    _sampled(w, True, [(0, 0), (0, 3), (0, 4), (0, 31)], 96, 2)
+
+
+def test_workload_head_dim_256():
+    w = workload(4)
+    _sampled(w, False, [(0, 0), (7, 7), (3, 5)], 96, 3)
