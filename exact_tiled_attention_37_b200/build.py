@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libattn.so")
 
 SOURCES = ["attn_api.cu"]
-HEADERS = ["ptx.cuh", "fwd.cuh", "bwd.cuh"]
+HEADERS = ["ptx.cuh", "fwd.cuh", "fwd_fp32.cuh", "bwd.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

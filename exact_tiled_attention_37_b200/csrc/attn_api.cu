@@ -15,6 +15,7 @@
 #include "attn.h"
 #include "bwd.cuh"
 #include "fwd.cuh"
+#include "fwd_fp32.cuh"
 
 // Device status word: [0] code, [1] wait site, [2..3] block of the first failure.
 __device__ int g_attn_status[4];
@@ -140,6 +141,30 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
   return last_launch();
 }
 
+// ---------------------------------------------------------------- backward
+template <int D, int NQS, int NPB>
+attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const attn_tensor_t& v,
+                         const attn_tensor_t& dout, eta::BwdParams& p, cudaStream_t st) {
+  using C = eta::BwdCfg<D, NQS, NPB>;
+  CUtensorMap tq, tk, tv, tdo;
+  attn_status_t s;
+  if ((s = make_map(&tq, q, p.B, p.Hq, p.N, D, 2, C::BR)) != ATTN_OK) return s;
+  if ((s = make_map(&tdo, dout, p.B, p.Hq, p.N, D, 2, C::BR)) != ATTN_OK) return s;
+  if ((s = make_map(&tk, k, p.B, p.Hkv, p.N, D, 2, C::BC)) != ATTN_OK) return s;
+  if ((s = make_map(&tv, v, p.B, p.Hkv, p.N, D, 2, C::BC)) != ATTN_OK) return s;
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
+  eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
+  if ((s = last_launch()) != ATTN_OK) return s;
+  auto kern = eta::bwd_dkdv_kernel<D, NQS, NPB>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
+  dim3 grid((p.N + C::BC - 1) / C::BC, p.Hkv * C::DSPLIT, p.B);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+  if ((s = last_launch()) != ATTN_OK) return s;
+  const long long vec = static_cast<long long>(p.B) * p.Hq * p.N * (D / 8);
+  eta::bwd_dq_finalize_kernel<D><<<static_cast<unsigned>((vec + 255) / 256), 256, 0, st>>>(p);
+  return last_launch();
+}
+
 attn_status_t check_sizes(int B, int Hq, int Hkv, int N) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
@@ -217,7 +242,13 @@ attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
   p.debug_flags = g_debug_flags.load();
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!bf16) return launch_pingpong<float, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+  if (!bf16) {
+    dim3 grid((N + eta::kF32Rows - 1) / eta::kF32Rows, Hq, B);
+    eta::fwd_fp32_kernel<<<grid, 128, 0, st>>>(
+        static_cast<const float*>(q.ptr), static_cast<const float*>(k.ptr),
+        static_cast<const float*>(v.ptr), q.sb, q.sh, q.sn, k.sb, k.sh, k.sn, v.sb, v.sh, v.sn, p);
+    return last_launch();
+  }
   switch (D) {
     case 64: return launch_pingpong<__nv_bfloat16, 64, 6>(q, k, v, p, B, Hq, Hkv, N, st);
     case 128: return launch_pingpong<__nv_bfloat16, 128, 4>(q, k, v, p, B, Hq, Hkv, N, st);
@@ -251,11 +282,34 @@ attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
   if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
   if (workspace_bytes < eta::bwd_workspace_bytes(B, Hq, N, D)) return ATTN_ERR_WORKSPACE;
-  int* status = nullptr;
-  if ((s = status_ptr(&status)) != ATTN_OK) return s;
-  return eta::launch_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal != 0, scale,
-                         workspace, status, g_wait_limit_ns.load(),
-                         static_cast<cudaStream_t>(stream));
+  eta::BwdParams p;
+  p.o = o.ptr;
+  p.dout = dout.ptr;
+  p.lse = lse;
+  p.dq = dq.ptr;
+  p.dk = dk.ptr;
+  p.dv = dv.ptr;
+  char* ws = static_cast<char*>(workspace);
+  p.dqacc = reinterpret_cast<float*>(ws);
+  p.delta = reinterpret_cast<float*>(ws + eta::bwd_dqacc_bytes(B, Hq, N, D));
+  p.lse2 = reinterpret_cast<float*>(ws + eta::bwd_dqacc_bytes(B, Hq, N, D) +
+                                    eta::bwd_stat_bytes(B, Hq, N));
+  p.osb = o.sb; p.osh = o.sh; p.osn = o.sn;
+  p.dosb = dout.sb; p.dosh = dout.sh; p.dosn = dout.sn;
+  p.dqsb = dq.sb; p.dqsh = dq.sh; p.dqsn = dq.sn;
+  p.dksb = dk.sb; p.dksh = dk.sh; p.dksn = dk.sn;
+  p.dvsb = dv.sb; p.dvsh = dv.sh; p.dvsn = dv.sn;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.D = D;
+  p.Npad = static_cast<int>(eta::bwd_npad(N));
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) return launch_bwd<128, 2, 2>(q, k, v, dout, p, st);
+  return launch_bwd<256, 1, 1>(q, k, v, dout, p, st);
 }
 
 }  // extern "C"

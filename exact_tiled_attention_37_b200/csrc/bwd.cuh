@@ -1,5 +1,35 @@
-// Backward attention kernels for sm_100a (placeholder: filled in below the
-// forward once it is verified).
+// Backward attention kernels for sm_100a.
+//
+// Recompute-based backward from the saved per-row logsumexp: P is rebuilt
+// tile by tile as exp2(S * scale * log2(e) - lse * log2(e)) and never stored.
+// Five products per (key tile, query tile) pair as in the backward the
+// FlashAttention (Metal Port) README describes for the official
+// implementation (Documentation section: five GEMMs, scratch space for
+// atomics and partial sums), with fp32 atomics for dQ:
+//
+//   S^T  = K Q_i^T            P^T  = exp2(S^T c - lse2_i)
+//   dP^T = V dO_i^T           dS^T = P^T * (dP^T - Delta_i)
+//   dV  += P^T dO_i           dK  += dS^T Q_i            (TMEM accumulators)
+//   dQ_i^T = K^T dS^T   ->  atomically added (x scale) to an fp32 scratch dQ
+//
+// Kernels:
+//  * bwd_preprocess_kernel: Delta = rowsum(dO * O) and lse2 = lse * log2(e)
+//    per row (rows past N padded with Delta = 0, lse2 = +inf so that their P
+//    is exactly 0), and zeroes the fp32 dQ scratch.  One warp per row.
+//  * bwd_dkdv_kernel: one CTA per (batch, key/value head, 128-row key tile,
+//    128-column slice of D); loops over the query heads of the GQA group and
+//    the 64-row query tiles (causal: only tiles at or below the diagonal).
+//    Roles: TMA producer warp, MMA warp, a 128-thread softmax warpgroup
+//    (thread j owns key row j: computes P^T, dS^T rows into shared memory and
+//    finally stores dK, dV), and a 128-thread dQ warpgroup (thread d owns
+//    column d of dQ^T: drains dQ_i^T from TMEM and issues coalesced fp32
+//    reductions into the scratch).
+//  * bwd_dq_finalize_kernel: dQ (bf16, caller's strides) from the scratch.
+//
+// TMEM (512 columns): ST/dQT[2] (64 each) | dPT[2] (64 each) | dV (128) | dK (128).
+// Head dimension 256 is split into two 128-column slices (two CTAs per key
+// tile, each recomputing S^T and dP^T over the full D): the TMEM-capacity
+// analogue of the D-blocking the Metal port README describes.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -15,18 +45,456 @@ constexpr int kBwdRowPad = 128;
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-inline size_t bwd_workspace_bytes(int B, int Hq, int N, int D) {
-  const size_t rows = static_cast<size_t>(B) * Hq;
-  const size_t npad = round_up(static_cast<size_t>(N), kBwdRowPad);
-  return round_up(rows * N * D * 4, 256) + 2 * round_up(rows * npad * 4, 256);
+inline size_t bwd_npad(int N) { return round_up(static_cast<size_t>(N), kBwdRowPad); }
+
+inline size_t bwd_dqacc_bytes(int B, int Hq, int N, int D) {
+  return round_up(static_cast<size_t>(B) * Hq * N * D * 4, 256);
 }
 
-inline attn_status_t launch_bwd(const attn_tensor_t&, const attn_tensor_t&, const attn_tensor_t&,
-                                const attn_tensor_t&, const float*, const attn_tensor_t&,
-                                const attn_tensor_t&, const attn_tensor_t&, const attn_tensor_t&,
-                                int, int, int, int, int, bool, float, void*, int*,
-                                unsigned long long, cudaStream_t) {
-  return ATTN_ERR_UNSUPPORTED;
+inline size_t bwd_stat_bytes(int B, int Hq, int N) {
+  return round_up(static_cast<size_t>(B) * Hq * bwd_npad(N) * 4, 256);
+}
+
+inline size_t bwd_workspace_bytes(int B, int Hq, int N, int D) {
+  return bwd_dqacc_bytes(B, Hq, N, D) + 2 * bwd_stat_bytes(B, Hq, N);
+}
+
+struct BwdParams {
+  const void* o;        // forward output [B, Hq, N, D]
+  const void* dout;     // upstream gradient [B, Hq, N, D]
+  const float* lse;     // [B, Hq, N]
+  void* dq;             // [B, Hq, N, D] bf16
+  void* dk;             // [B, Hkv, N, D] bf16
+  void* dv;
+  float* dqacc;         // [B, Hq, N, D] fp32 scratch
+  float* delta;         // [B, Hq, Npad]
+  float* lse2;          // [B, Hq, Npad]
+  long long osb, osh, osn;
+  long long dosb, dosh, dosn;
+  long long dqsb, dqsh, dqsn;
+  long long dksb, dksh, dksn;
+  long long dvsb, dvsh, dvsn;
+  int B, Hq, Hkv, N, D, Npad, group, causal;
+  float scale, c;       // c = scale * log2(e)
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+// ---------------------------------------------------------------- preprocess
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) {
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
+  if (warp >= rows) return;
+  const int bh = static_cast<int>(warp / p.Npad);
+  const int i = static_cast<int>(warp % p.Npad);
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  if (i >= p.N) {
+    if (lane == 0) {
+      p.delta[warp] = 0.f;
+      p.lse2[warp] = INFINITY;
+    }
+    return;
+  }
+  constexpr int PER = D / 32;  // elements per lane (4 or 8)
+  const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(p.o) + b * p.osb + h * p.osh + i * p.osn;
+  const __nv_bfloat16* drow =
+      static_cast<const __nv_bfloat16*>(p.dout) + b * p.dosb + h * p.dosh + i * p.dosn;
+  float acc = 0.f;
+  if constexpr (PER == 4) {
+    const uint2 ov = *reinterpret_cast<const uint2*>(orow + lane * 4);
+    const uint2 dv = *reinterpret_cast<const uint2*>(drow + lane * 4);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float2 of = __bfloat1622float2(o2[e]);
+      const float2 df = __bfloat1622float2(d2[e]);
+      acc = fmaf(of.x, df.x, acc);
+      acc = fmaf(of.y, df.y, acc);
+    }
+  } else {
+    const uint4 ov = *reinterpret_cast<const uint4*>(orow + lane * 8);
+    const uint4 dv = *reinterpret_cast<const uint4*>(drow + lane * 8);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 of = __bfloat1622float2(o2[e]);
+      const float2 df = __bfloat1622float2(d2[e]);
+      acc = fmaf(of.x, df.x, acc);
+      acc = fmaf(of.y, df.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  // zero this row of the fp32 dQ scratch
+  float4* zrow = reinterpret_cast<float4*>(p.dqacc + (static_cast<long long>(bh) * p.N + i) * D);
+#pragma unroll
+  for (int e = lane; e < D / 4; e += 32) zrow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane == 0) {
+    p.delta[warp] = acc;
+    p.lse2[warp] = p.lse[static_cast<long long>(bh) * p.N + i] * 1.4426950408889634f;
+  }
+}
+
+// ---------------------------------------------------------------- dQ finalize
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_finalize_kernel(const BwdParams p) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  constexpr int VEC = 8;
+  const long long per_row = D / VEC;
+  const long long total = static_cast<long long>(p.B) * p.Hq * p.N * per_row;
+  if (idx >= total) return;
+  const long long row = idx / per_row;
+  const int col = static_cast<int>(idx % per_row) * VEC;
+  const int i = static_cast<int>(row % p.N);
+  const int bh = static_cast<int>(row / p.N);
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const float4* src = reinterpret_cast<const float4*>(p.dqacc + row * D + col);
+  const float4 a = src[0], c = src[1];
+  uint4 w;
+  w.x = pack_bf16x2(a.x, a.y);
+  w.y = pack_bf16x2(a.z, a.w);
+  w.z = pack_bf16x2(c.x, c.y);
+  w.w = pack_bf16x2(c.z, c.w);
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) + b * p.dqsb + h * p.dqsh + i * p.dqsn + col;
+  *reinterpret_cast<uint4*>(dst) = w;
+}
+
+// ---------------------------------------------------------------- dK / dV (+ dQ atomics)
+template <int DFULL, int NQS, int NPB>
+struct BwdCfg {
+  static constexpr int BC = 128;                 // key rows per CTA
+  static constexpr int BR = 64;                  // query rows per iteration
+  static constexpr int DH = 128;                 // D slice of dK/dV/dQ per CTA
+  static constexpr int DSPLIT = DFULL / DH;
+  static constexpr int ROWB = DFULL * 2;
+  static constexpr int NCHUNK = ROWB / 128;
+  static constexpr int KCHUNK = BC * 128;        // 16 KB
+  static constexpr int QCHUNK = BR * 128;        // 8 KB
+  static constexpr int KTILE = BC * ROWB;
+  static constexpr int QTILE = BR * ROWB;
+  static constexpr int PTILE = BC * BR * 2;      // 16 KB: one 128-byte row per key row
+  static constexpr int KSTEPS = ROWB / 32;       // S^T / dP^T MMAs over D
+  // TMEM columns
+  static constexpr int T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 384, TMEM_COLS = 512;
+  // shared memory
+  static constexpr int S_K = 0;
+  static constexpr int S_V = S_K + KTILE;
+  static constexpr int S_Q = S_V + KTILE;                  // [NQS] Q tiles
+  static constexpr int S_DO = S_Q + NQS * QTILE;           // [NQS] dO tiles
+  static constexpr int S_P = S_DO + NQS * QTILE;           // [NPB] P^T
+  static constexpr int S_DS = S_P + NPB * PTILE;           // [NPB] dS^T
+  static constexpr int S_STAT = S_DS + NPB * PTILE;        // [NQS] lse2[64], delta[64]
+  static constexpr int S_BAR = S_STAT + NQS * 512;
+  static constexpr int B_KV = 0;
+  static constexpr int B_QF = 1;
+  static constexpr int B_QE = 1 + NQS;
+  static constexpr int B_SP = 1 + 2 * NQS;                // [2]
+  static constexpr int B_DS = 3 + 2 * NQS;                // [NPB]
+  static constexpr int B_PE = 3 + 2 * NQS + NPB;          // [NPB]
+  static constexpr int B_DQF = 3 + 2 * NQS + 2 * NPB;     // [2]
+  static constexpr int B_DQE = 5 + 2 * NQS + 2 * NPB;     // [2]
+  static constexpr int B_KVD = 7 + 2 * NQS + 2 * NPB;     // dK/dV accumulated
+  static constexpr int B_DONE = 8 + 2 * NQS + 2 * NPB;
+  static constexpr int NBAR = 9 + 2 * NQS + 2 * NPB;
+  static constexpr int S_MISC = S_BAR + 8 * NBAR;
+  static constexpr int SMEM_BYTES = S_MISC + 16 + 1024;
+  static constexpr int THREADS = 384;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int DFULL, int NQS, int NPB>
+__global__ void __launch_bounds__(384, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using C = BwdCfg<DFULL, NQS, NPB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::S_BAR;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x;  // key tile (causal: tile 0 has the most work, starts first)
+  const int hk = blockIdx.y / C::DSPLIT;
+  const int half = blockIdx.y % C::DSPLIT;
+  const int b = blockIdx.z;
+  const int k0 = kt * C::BC;
+  const int nqt = (p.N + C::BR - 1) / C::BR;
+  const int i_first = p.causal ? k0 / C::BR : 0;
+  const int per_head = nqt - i_first;
+  const int n = per_head * p.group;  // iterations: query heads of the group x query tiles
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_KV), 1);
+    for (int s = 0; s < NQS; ++s) {
+      mbar_init(BAR(C::B_QF + s), 1);
+      mbar_init(BAR(C::B_QE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(C::B_SP + s), 1);
+      mbar_init(BAR(C::B_DQF + s), 1);
+      mbar_init(BAR(C::B_DQE + s), 4);
+    }
+    for (int s = 0; s < NPB; ++s) {
+      mbar_init(BAR(C::B_DS + s), 4);
+      mbar_init(BAR(C::B_PE + s), 1);
+    }
+    mbar_init(BAR(C::B_KVD), 1);
+    mbar_init(BAR(C::B_DONE), 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+
+  // iteration -> (query head, query tile)
+  auto head_of = [&](int it) { return hk * p.group + it / per_head; };
+  auto qtile_of = [&](int it) { return i_first + it % per_head; };
+
+  if (warp < 4) {
+    // ------------------------------------------------ P^T / dS^T rows, then dK / dV epilogue
+    const int j = threadIdx.x;  // key row within the tile == TMEM lane
+    const int jg = k0 + j;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < n; ++it) {
+      const int buf = it & 1, stage = it % NQS, pb = it % NPB;
+      if (!W.wait_warp(BAR(C::B_SP + buf), (it >> 1) & 1, 60)) { ok = false; break; }
+      if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 61)) { ok = false; break; }
+      tc_fence_after();
+      float s[64], dp[64];
+      tmem_load_row<64>(tmem + lane_base + C::T_ST + 64 * buf, s);
+      tmem_load_row<64>(tmem + lane_base + C::T_DPT + 64 * buf, dp);
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::S_STAT + stage * 512);
+      const float* dlt = lse2 + 64;
+      const int ig0 = qtile_of(it) * C::BR;
+      // causal: query i sees key j iff jg <= ig0 + i  ->  valid for i >= jg - ig0
+      const int ilo = p.causal ? jg - ig0 : -1;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float pv = ex2(fmaf(s[i], p.c, -lse2[i]));
+        if (i < ilo) pv = 0.f;
+        s[i] = pv;
+        dp[i] = pv * (dp[i] - dlt[i]);
+      }
+      // the MMAs that read this P/dS buffer NPB iterations ago must be done
+      if (!W.wait_warp(BAR(C::B_PE + pb), ((it / NPB) & 1) ^ 1, 62)) { ok = false; break; }
+      uint8_t* prow = smem + C::S_P + pb * C::PTILE + j * 128;
+      uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int sw = (u ^ (j & 7)) * 16;
+        uint4 a, d;
+        a.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
+        a.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
+        a.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
+        a.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
+        d.x = pack_bf16x2(dp[8 * u + 0], dp[8 * u + 1]);
+        d.y = pack_bf16x2(dp[8 * u + 2], dp[8 * u + 3]);
+        d.z = pack_bf16x2(dp[8 * u + 4], dp[8 * u + 5]);
+        d.w = pack_bf16x2(dp[8 * u + 6], dp[8 * u + 7]);
+        *reinterpret_cast<uint4*>(prow + sw) = a;
+        *reinterpret_cast<uint4*>(drow + sw) = d;
+      }
+      fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DS + pb));
+    }
+    if (ok && W.wait_warp(BAR(C::B_KVD), 0, 63)) {
+      tc_fence_after();
+      const bool valid = jg < p.N;
+      __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
+                             static_cast<long long>(jg) * p.dvsn + half * C::DH;
+      __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
+                             static_cast<long long>(jg) * p.dksn + half * C::DH;
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        __nv_bfloat16* row = t ? dkrow : dvrow;
+        const float mul = t ? p.scale : 1.f;
+        const uint32_t col = t ? C::T_DK : C::T_DV;
+#pragma unroll 1
+        for (int c = 0; c < C::DH / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + col + 32 * c, r);
+          tmem_wait_ld();
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(row + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16x2(u2f(r[8 * v + 0]) * mul, u2f(r[8 * v + 1]) * mul);
+              w.y = pack_bf16x2(u2f(r[8 * v + 2]) * mul, u2f(r[8 * v + 3]) * mul);
+              w.z = pack_bf16x2(u2f(r[8 * v + 4]) * mul, u2f(r[8 * v + 5]) * mul);
+              w.w = pack_bf16x2(u2f(r[8 * v + 6]) * mul, u2f(r[8 * v + 7]) * mul);
+              dst[v] = w;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------ dQ^T drain -> fp32 reductions
+    const int dd = threadIdx.x - 128;  // column of this CTA's D slice == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    for (int it = 0; it < n; ++it) {
+      const int buf = it & 1;
+      if (!W.wait_warp(BAR(C::B_DQF + buf), (it >> 1) & 1, 70)) break;
+      tc_fence_after();
+      float v[64];
+      tmem_load_row<64>(tmem + lane_base + C::T_ST + 64 * buf, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DQE + buf));
+      const int h = head_of(it);
+      const int ig0 = qtile_of(it) * C::BR;
+      float* dst = p.dqacc + (static_cast<long long>(b * p.Hq + h) * p.N + ig0) * DFULL +
+                   half * C::DH + dd;
+      const int imax = min(64, p.N - ig0);
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (i < imax) atomicAdd(dst + static_cast<long long>(i) * DFULL, v[i] * p.scale);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_expect_tx(BAR(C::B_KV), 2 * C::KTILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sbase + C::S_K + c * C::KCHUNK, &tm_k, BAR(C::B_KV), c * 64, k0, hk, b);
+        tma_load_4d(sbase + C::S_V + c * C::KCHUNK, &tm_v, BAR(C::B_KV), c * 64, k0, hk, b);
+      }
+      int it = 0;
+      for (; it < n; ++it) {
+        const int stage = it % NQS;
+        if (!W.wait(BAR(C::B_QE + stage), ((it / NQS) & 1) ^ 1, 80)) break;
+        const int h = head_of(it);
+        const int ig0 = qtile_of(it) * C::BR;
+        const uint32_t full = BAR(C::B_QF + stage);
+        mbar_expect_tx(full, 2 * C::QTILE + 512);
+        for (int c = 0; c < C::NCHUNK; ++c) {
+          tma_load_4d(sbase + C::S_Q + stage * C::QTILE + c * C::QCHUNK, &tm_q, full, c * 64, ig0, h, b);
+          tma_load_4d(sbase + C::S_DO + stage * C::QTILE + c * C::QCHUNK, &tm_do, full, c * 64, ig0, h, b);
+        }
+        const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
+        bulk_load(sbase + C::S_STAT + stage * 512, p.lse2 + srow, 256, full);
+        bulk_load(sbase + C::S_STAT + stage * 512 + 256, p.delta + srow, 256, full);
+      }
+      W.drain(BAR(C::B_KV), 0, 81);
+      const int issued = it;
+      for (int s = 0; s < NQS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NQS) * NQS;
+        W.drain(BAR(C::B_QF + s), static_cast<uint32_t>(last / NQS) & 1u, 82);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_make(128, 64, 1u, false, false);      // S^T, dP^T
+      constexpr uint32_t id_kv = idesc_make(128, C::DH, 1u, false, true);   // dV, dK
+      constexpr uint32_t id_q = idesc_make(128, 64, 1u, true, true);        // dQ^T
+      const uint32_t sK = sbase + C::S_K, sV = sbase + C::S_V;
+      auto issue_sdp = [&](int it) {
+        const int buf = it & 1, stage = it % NQS;
+        const uint32_t sq = sbase + C::S_Q + stage * C::QTILE;
+        const uint32_t sdo = sbase + C::S_DO + stage * C::QTILE;
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+          const uint32_t ko = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
+          const uint32_t qo = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
+          mma_ss<false>(tmem + C::T_ST + 64 * buf, sdesc_sw128(sK + ko, 16, 1024),
+                        sdesc_sw128(sq + qo, 16, 1024), id_s, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+          const uint32_t ko = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
+          const uint32_t qo = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
+          mma_ss<false>(tmem + C::T_DPT + 64 * buf, sdesc_sw128(sV + ko, 16, 1024),
+                        sdesc_sw128(sdo + qo, 16, 1024), id_s, ks > 0);
+        }
+      };
+      bool ok = W.wait(BAR(C::B_KV), 0, 90) && (n == 0 || W.wait(BAR(C::B_QF), 0, 91));
+      if (ok && n > 0) {
+        tc_fence_after();
+        issue_sdp(0);
+        mma_commit(BAR(C::B_SP + 0));
+      }
+      // S^T / dP^T of the next iteration go into the other TMEM buffer once
+      // the dQ warpgroup has drained the dQ^T that last used it.
+      auto issue_next = [&](int it) -> bool {
+        const int b1 = (it + 1) & 1, st1 = (it + 1) % NQS;
+        if (it >= 1 && !W.wait(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1, 92)) return false;
+        if (!W.wait(BAR(C::B_QF + st1), ((it + 1) / NQS) & 1, 93)) return false;
+        tc_fence_after();
+        issue_sdp(it + 1);
+        mma_commit(BAR(C::B_SP + b1));
+        return true;
+      };
+      for (int it = 0; ok && it < n; ++it) {
+        const int buf = it & 1, stage = it % NQS, pb = it % NPB;
+        // With two Q/dO stages the next tile's products overlap this tile's
+        // softmax; with one stage they must wait for this tile's products.
+        if (NQS > 1 && it + 1 < n && !issue_next(it)) { ok = false; break; }
+        if (!W.wait(BAR(C::B_DS + pb), (it / NPB) & 1, 94)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sq = sbase + C::S_Q + stage * C::QTILE + half * 2 * C::QCHUNK;
+        const uint32_t sdo = sbase + C::S_DO + stage * C::QTILE + half * 2 * C::QCHUNK;
+        const uint32_t sp = sbase + C::S_P + pb * C::PTILE;
+        const uint32_t sds = sbase + C::S_DS + pb * C::PTILE;
+        // dV += P^T dO_i (K = 64 query rows, 4 steps of 16)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss<false>(tmem + C::T_DV, sdesc_sw128(sp + ks * 32, 16, 1024),
+                        sdesc_sw128(sdo + ks * 2048, C::QCHUNK, 1024), id_kv, (it > 0 || ks > 0));
+        // dK += dS^T Q_i
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss<false>(tmem + C::T_DK, sdesc_sw128(sds + ks * 32, 16, 1024),
+                        sdesc_sw128(sq + ks * 2048, C::QCHUNK, 1024), id_kv, (it > 0 || ks > 0));
+        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed S^T buffer
+        const uint32_t kh = sK + half * 2 * C::KCHUNK;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss<false>(tmem + C::T_ST + 64 * buf, sdesc_sw128(kh + ks * 2048, C::KCHUNK, 1024),
+                        sdesc_sw128(sds + ks * 2048, C::PTILE, 1024), id_q, ks > 0);
+        mma_commit(BAR(C::B_DQF + buf));
+        mma_commit(BAR(C::B_QE + stage));
+        mma_commit(BAR(C::B_PE + pb));
+        if (NQS == 1 && it + 1 < n && !issue_next(it)) { ok = false; break; }
+      }
+      if (ok) mma_commit(BAR(C::B_KVD));
+      mma_commit(BAR(C::B_DONE));
+      W.drain(BAR(C::B_DONE), 0, 95);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
 }
 
 }  // namespace eta

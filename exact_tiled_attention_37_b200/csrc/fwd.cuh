@@ -14,8 +14,7 @@
 //  * fwd_pingpong_kernel: one CTA owns two 128-row query tiles of one
 //    (batch, head) and streams 128-row K/V tiles through a TMA ring.  While the
 //    softmax warpgroup of one query tile works, the tensor core runs the other
-//    tile's MMAs.  TMEM: S0 | S1 | O0 | O1.  Used for D*sizeof(T) <= 256 bytes
-//    (bf16 D = 64, 128; fp32/tf32 D = 64).
+//    tile's MMAs.  TMEM: S0 | S1 | O0 | O1.  Used for bf16 D = 64, 128.
 //  * fwd_single_kernel: one 128-row query tile, 64-row K/V tiles and a double
 //    buffered S so that S(j+1) = Q K_{j+1}^T runs while row softmax works on
 //    S(j).  TMEM: S0 | S1 | O (D = 256 columns).  Used for bf16 D = 256.
@@ -90,20 +89,6 @@ __device__ __forceinline__ bool online_softmax_step(float (&s)[BC], float c, flo
   }
   l += (l0 + l1) + (l2 + l3);
   return warp_rescale;
-}
-
-// Loads BC consecutive fp32 TMEM columns of this thread's lane into s.
-template <int BC>
-__device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&s)[BC]) {
-  static_assert(BC % 32 == 0, "row chunks of 32 columns");
-#pragma unroll
-  for (int c = 0; c < BC / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld32(taddr + 32 * c, r);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) s[32 * c + i] = u2f(r[i]);
-  }
-  tmem_wait_ld();
 }
 
 // Writes p (BC values) back into TMEM as the A operand of the P V MMA:
@@ -237,6 +222,9 @@ struct PingPongCfg {
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;  // tmem slot, abort flag
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
+  // bf16 only: tf32 products would keep 10 mantissa bits, which misses the
+  // logsumexp tolerance; fp32 storage goes through fwd_fp32_kernel.
+  static_assert(sizeof(T) == 2, "bf16 storage");
   static_assert(ROWB % 128 == 0, "row must be whole 128-byte chunks");
   static_assert(256 + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");

@@ -130,7 +130,20 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (no multicast); both addresses 16-byte
+// aligned, size a multiple of 16 bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
                "r"(ncols)
@@ -262,6 +275,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// Loads BC consecutive fp32 TMEM columns of this thread's lane into s.
+template <int BC>
+__device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&s)[BC]) {
+  static_assert(BC % 32 == 0, "row chunks of 32 columns");
+#pragma unroll
+  for (int c = 0; c < BC / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 32 * c, r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s[32 * c + i] = u2f(r[i]);
+  }
+  tmem_wait_ld();
+}
+
 // ----------------------------------------------------------------- math
 // Hardware base-2 exponential (MUFU); ex2(-inf) = +0.
 __device__ __forceinline__ float ex2(float x) {
@@ -275,6 +302,5 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
 }  // namespace eta

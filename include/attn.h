@@ -99,7 +99,7 @@ ATTN_API attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t 
  * Bytes of device workspace attn_bwd needs for these sizes: an fp32 dQ
  * accumulator [B,Hq,N,D] (the scratch the backward's atomic partial sums go
  * to) plus two fp32 row statistics [B,Hq,N'] (rowsum(dO*O) and lse*log2(e),
- * N' = N rounded up to 64).  Returns 0 for invalid sizes.
+ * N' = N rounded up to 128).  Returns 0 for invalid sizes.
  */
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D);
 

@@ -1,0 +1,104 @@
+"""Backward parity: dQ, dK, dV from the CUDA kernels (through the C ABI, fed
+with the CUDA forward's O and lse) against the fp64 oracle's softmax-Jacobian
+gradients on the same seeded inputs."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_37_b200 import attn_bwd, attn_fwd, device_status
+from exact_tiled_attention_37_b200.inputs import make_inputs, make_random, workload
+
+from ._util import TOL_REL, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run(q, k, v, do, causal, scale=None):
+    q, k, v, do = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = attn_fwd(q, k, v, causal=causal, scale=scale)
+    dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    code, where = device_status()
+    assert code == 0, f"device status {code} at wait site {where}"
+    return dq, dk, dv
+
+
+def check(q, k, v, do, causal, heads=None, scale=None):
+    D = q.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq, dk, dv = run(q, k, v, do, causal, scale)
+    ref = oracle.attention_bwd(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                               do.float().numpy(), causal, scale, heads=heads)
+    errs = []
+    for name, got, r in (("dq", dq, ref[0]), ("dk", dk, ref[1]), ("dv", dv, ref[2])):
+        g = to_np(got)
+        if heads is not None:
+            mask = ~np.isnan(r)
+            g, r = g[mask], r[mask]
+        e = rel_err(g, r)
+        errs.append(e)
+        assert e <= TOL_REL, (name, e)
+    return errs
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 64, 100, 128, 200, 256, 300, 640])
+def test_small_shapes(D, causal, N):
+    q, k, v, do = make_random(1, 2, 2, N, D, "bf16", seed=N * 3 + D + causal)
+    check(q, k, v, do, causal)
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hq,hkv", [(4, 1), (4, 2), (6, 3)])
+def test_grouped_query_heads(D, causal, hq, hkv):
+    q, k, v, do = make_random(2, hq, hkv, 333, D, "bf16", seed=hq * 11 + hkv + D)
+    check(q, k, v, do, causal)
+
+
+def test_strided_views():
+    B, H, N, D = 2, 3, 260, 128
+    g = torch.Generator().manual_seed(17)
+    q, k, v, do = (torch.randn(B, N, H, D, generator=g).to(torch.bfloat16).to(DEV).transpose(1, 2)
+                   for _ in range(4))
+    for causal in (False, True):
+        o, lse = attn_fwd(q, k, v, causal=causal)
+        dqb = torch.zeros(B, N, H, D, device=DEV, dtype=torch.bfloat16)
+        dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dqb.transpose(1, 2))
+        ref = oracle.attention_bwd(*(to_np(t) for t in (q, k, v, do)), causal, 1 / math.sqrt(D))
+        for got, r in zip((dq, dk, dv), ref):
+            assert rel_err(to_np(got), r) <= TOL_REL
+
+
+def test_sharp_softmax_scale():
+    q, k, v, do = make_random(1, 2, 1, 500, 128, "bf16", seed=23, k_mult=3.0)
+    for causal in (False, True):
+        check(q, k, v, do, causal, scale=0.25)
+
+
+def test_dk_dv_deterministic():
+    q, k, v, do = (t.to(DEV) for t in make_random(1, 4, 2, 700, 128, "bf16", seed=8))
+    o, lse = attn_fwd(q, k, v, causal=True)
+    a = attn_bwd(q, k, v, o, lse, do, causal=True)
+    b = attn_bwd(q, k, v, o, lse, do, causal=True)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    # dQ sums fp32 partials with atomics: equal up to summation order
+    assert rel_err(to_np(a[0]), to_np(b[0])) < 1e-2
+
+
+def test_workload_mha_4096_causal():
+    w = workload(2)
+    q, k, v, do = make_inputs(w)
+    check(q, k, v, do, True, heads=[(0, 0), (1, 15)])
+
+
+def test_workload_head_dim_256():
+    w = workload(4)
+    q, k, v, do = make_inputs(w)
+    check(q, k, v, do, False, heads=[(3, 5)])
