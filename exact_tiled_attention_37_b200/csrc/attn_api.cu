@@ -25,6 +25,8 @@ namespace {
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_debug_flags{0};
+std::atomic<void*> g_bwd_ev_start{nullptr};
+std::atomic<void*> g_bwd_ev_stop{nullptr};
 
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {};
@@ -158,8 +160,13 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
   auto kern = eta::bwd_dkdv_kernel<D, NQS, NPB>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
   dim3 grid((p.N + C::BC - 1) / C::BC, p.Hkv * C::DSPLIT, p.B);
+  cudaEvent_t ev0 = static_cast<cudaEvent_t>(g_bwd_ev_start.exchange(nullptr));
+  cudaEvent_t ev1 = static_cast<cudaEvent_t>(g_bwd_ev_stop.exchange(nullptr));
+  const bool timed = ev0 && ev1;
+  if (timed && cudaEventRecord(ev0, st) != cudaSuccess) return ATTN_ERR_CUDA;
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
   if ((s = last_launch()) != ATTN_OK) return s;
+  if (timed && cudaEventRecord(ev1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   const long long vec = static_cast<long long>(p.B) * p.Hq * p.N * (D / 8);
   eta::bwd_dq_finalize_kernel<D><<<static_cast<unsigned>((vec + 255) / 256), 256, 0, st>>>(p);
   return last_launch();
@@ -196,6 +203,11 @@ void attn_debug_set_wait_limit_ns(unsigned long long ns) {
 }
 
 void attn_debug_set_flags(int flags) { g_debug_flags.store(flags); }
+
+void attn_debug_set_bwd_events(void* start, void* stop) {
+  g_bwd_ev_start.store(start);
+  g_bwd_ev_stop.store(stop);
+}
 
 attn_status_t attn_device_status(void* stream, int* where) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;

@@ -134,6 +134,14 @@ ATTN_API attn_status_t attn_device_status(void* stream, int* where);
 ATTN_API void attn_debug_set_wait_limit_ns(unsigned long long ns);
 ATTN_API void attn_debug_set_flags(int flags);
 
+/*
+ * Timing hook.  When both are non-NULL (cudaEvent_t handles owned by the
+ * caller), the next attn_bwd call records `start` on its stream right before
+ * launching its main dK/dV kernel and `stop` right after it, then forgets
+ * them; this times that kernel alone inside a longer stream of work.
+ */
+ATTN_API void attn_debug_set_bwd_events(void* start, void* stop);
+
 #ifdef __cplusplus
 }
 #endif

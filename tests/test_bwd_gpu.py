@@ -40,7 +40,9 @@ def check(q, k, v, do, causal, heads=None, scale=None):
         if heads is not None:
             mask = ~np.isnan(r)
             g, r = g[mask], r[mask]
-        e = rel_err(g, r)
+        # With a single visible key dQ and dK are exactly zero (dS = P (dP - Delta)
+        # with P = 1 and dP = Delta); measure against a unit floor there.
+        e = rel_err(g, r) if np.max(np.abs(r)) > 1e-6 else float(np.max(np.abs(g)))
         errs.append(e)
         assert e <= TOL_REL, (name, e)
     return errs
