@@ -22,6 +22,22 @@ __device__ int g_attn_status[4];
 
 namespace {
 
+__global__ void debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n,
+                                  int mode) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float2 r;
+  if (mode == 1) {
+    r = eta::exp2_poly2(make_float2(a, b));
+  } else {
+    r.x = eta::ex2(a);
+    r.y = eta::ex2(b);
+  }
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
+
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_debug_flags{0};
@@ -207,6 +223,22 @@ void attn_debug_set_flags(int flags) { g_debug_flags.store(flags); }
 void attn_debug_set_bwd_events(void* start, void* stop) {
   g_bwd_ev_start.store(start);
   g_bwd_ev_stop.store(stop);
+}
+
+#ifdef ETA_TRACE
+ATTN_API int attn_debug_read_trace(void* dst, size_t bytes) {
+  if (bytes > sizeof(eta::g_eta_trace)) bytes = sizeof(eta::g_eta_trace);
+  return cudaMemcpyFromSymbol(dst, eta::g_eta_trace, bytes) == cudaSuccess ? 0 : 1;
+}
+#endif
+
+attn_status_t attn_debug_exp2(const float* x, float* y, int n, int mode, void* stream) {
+  if (!x || !y || n < 0 || (mode != 0 && mode != 1)) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  const int pairs = (n + 1) / 2;
+  debug_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n,
+                                                                                       mode);
+  return last_launch();
 }
 
 attn_status_t attn_device_status(void* stream, int* where) {

@@ -40,6 +40,20 @@
 
 namespace eta {
 
+#ifdef ETA_TRACE
+// Debug builds only: per-role clock64() timelines of two CTAs of the dK/dV
+// kernel ([cta][role][iteration][event]).
+__device__ unsigned long long g_eta_trace[2][4][256][4];
+#define ETA_TRACE_AT(cta, role, it, ev)                                          \
+  do {                                                                          \
+    if ((cta) >= 0 && (it) < 256) g_eta_trace[(cta)][(role)][(it)][(ev)] = clock64(); \
+  } while (0)
+#else
+#define ETA_TRACE_AT(cta, role, it, ev) \
+  do {                                  \
+  } while (0)
+#endif
+
 // Rows of the per-row statistics are padded to a multiple of this.
 constexpr int kBwdRowPad = 128;
 
@@ -263,6 +277,12 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 
+#ifdef ETA_TRACE
+  const int tcta = (blockIdx.y == 0 && blockIdx.z == 0) ? (kt == 0 ? 0 : (kt == 16 ? 1 : -1)) : -1;
+#else
+  const int tcta = -1;
+#endif
+  (void)tcta;
   // iteration -> (query head, query tile)
   auto head_of = [&](int it) { return hk * p.group + it / per_head; };
   auto qtile_of = [&](int it) { return i_first + it % per_head; };
@@ -277,6 +297,7 @@ __global__ void __launch_bounds__(384, 1)
       const int buf = it & 1, stage = it % NQS, pb = it % NPB;
       if (!W.wait_warp(BAR(C::B_SP + buf), (it >> 1) & 1, 60)) { ok = false; break; }
       if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 61)) { ok = false; break; }
+      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 0);
       tc_fence_after();
       float s[64], dp[64];
       tmem_load_row<64>(tmem + lane_base + C::T_ST + 64 * buf, s);
@@ -293,8 +314,10 @@ __global__ void __launch_bounds__(384, 1)
         s[i] = pv;
         dp[i] = pv * (dp[i] - dlt[i]);
       }
+      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 1);
       // the MMAs that read this P/dS buffer NPB iterations ago must be done
       if (!W.wait_warp(BAR(C::B_PE + pb), ((it / NPB) & 1) ^ 1, 62)) { ok = false; break; }
+      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 2);
       uint8_t* prow = smem + C::S_P + pb * C::PTILE + j * 128;
       uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
 #pragma unroll
@@ -316,6 +339,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DS + pb));
+      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 3);
     }
     if (ok && W.wait_warp(BAR(C::B_KVD), 0, 63)) {
       tc_fence_after();
@@ -356,12 +380,14 @@ __global__ void __launch_bounds__(384, 1)
     for (int it = 0; it < n; ++it) {
       const int buf = it & 1;
       if (!W.wait_warp(BAR(C::B_DQF + buf), (it >> 1) & 1, 70)) break;
+      if (threadIdx.x == 128) ETA_TRACE_AT(tcta, 1, it, 0);
       tc_fence_after();
       float v[64];
       tmem_load_row<64>(tmem + lane_base + C::T_ST + 64 * buf, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DQE + buf));
+      if (threadIdx.x == 128) ETA_TRACE_AT(tcta, 1, it, 1);
       const int h = head_of(it);
       const int ig0 = qtile_of(it) * C::BR;
       float* dst = p.dqacc + (static_cast<long long>(b * p.Hq + h) * p.N + ig0) * DFULL +
@@ -370,6 +396,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int i = 0; i < 64; ++i)
         if (i < imax) atomicAdd(dst + static_cast<long long>(i) * DFULL, v[i] * p.scale);
+      if (threadIdx.x == 128) ETA_TRACE_AT(tcta, 1, it, 2);
     }
   } else if (warp == 8) {
     // ------------------------------------------------ TMA producer
@@ -387,6 +414,7 @@ __global__ void __launch_bounds__(384, 1)
       for (; it < n; ++it) {
         const int stage = it % NQS;
         if (!W.wait(BAR(C::B_QE + stage), ((it / NQS) & 1) ^ 1, 80)) break;
+        ETA_TRACE_AT(tcta, 3, it, 0);
         const int h = head_of(it);
         const int ig0 = qtile_of(it) * C::BR;
         const uint32_t full = BAR(C::B_QF + stage);
@@ -452,10 +480,13 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int it = 0; ok && it < n; ++it) {
         const int buf = it & 1, stage = it % NQS, pb = it % NPB;
+        ETA_TRACE_AT(tcta, 2, it, 0);
         // With two Q/dO stages the next tile's products overlap this tile's
         // softmax; with one stage they must wait for this tile's products.
         if (NQS > 1 && it + 1 < n && !issue_next(it)) { ok = false; break; }
+        ETA_TRACE_AT(tcta, 2, it, 1);
         if (!W.wait(BAR(C::B_DS + pb), (it / NPB) & 1, 94)) { ok = false; break; }
+        ETA_TRACE_AT(tcta, 2, it, 2);
         tc_fence_after();
         const uint32_t sq = sbase + C::S_Q + stage * C::QTILE + half * 2 * C::QCHUNK;
         const uint32_t sdo = sbase + C::S_DO + stage * C::QTILE + half * 2 * C::QCHUNK;
@@ -480,6 +511,7 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(BAR(C::B_DQF + buf));
         mma_commit(BAR(C::B_QE + stage));
         mma_commit(BAR(C::B_PE + pb));
+        ETA_TRACE_AT(tcta, 2, it, 3);
         if (NQS == 1 && it + 1 < n && !issue_next(it)) { ok = false; break; }
       }
       if (ok) mma_commit(BAR(C::B_KVD));

@@ -35,6 +35,13 @@ namespace eta {
 // identical: O and l always share the same reference maximum).
 constexpr float kRescaleLog2 = 8.0f;
 
+// Columns (of every 8) whose exponential the ping-pong kernel computes with
+// the FMA-pipe polynomial; the rest use the MUFU ex2 unit.
+#ifndef ETA_SOFT_EXP8
+#define ETA_SOFT_EXP8 2
+#endif
+constexpr int kSoftExp8 = ETA_SOFT_EXP8;
+
 struct FwdParams {
   void* o;           // [B, Hq, N, D], unit stride on D
   float* lse;        // [B, Hq, N] contiguous
@@ -53,17 +60,23 @@ struct FwdParams {
 // l the running sum of exp2((s - m) * c).  Converts s in place into
 // p = exp2((s - m) * c).  Returns true when this warp rescaled (alpha != 1
 // for some row of the warp); alpha is this row's factor for O and l.
-template <int BC>
+// SOFT8 of every 8 columns take their exponential from the FMA-pipe
+// polynomial instead of the MUFU unit (the two run in parallel).
+template <int BC, int SOFT8>
 __device__ __forceinline__ bool online_softmax_step(float (&s)[BC], float c, float& m, float& l,
                                                     float& alpha) {
-  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+  static_assert(BC % 8 == 0 && SOFT8 % 2 == 0 && SOFT8 <= 8, "column pattern");
+  float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
+  float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
 #pragma unroll
-  for (int i = 4; i < BC; i += 4) {
-    mx0 = fmaxf(mx0, s[i]);
-    mx1 = fmaxf(mx1, s[i + 1]);
-    mx2 = fmaxf(mx2, s[i + 2]);
-    mx3 = fmaxf(mx3, s[i + 3]);
+  for (int i = 12; i + 8 <= BC; i += 8) {
+    mx0 = fmax3(mx0, s[i], s[i + 1]);
+    mx1 = fmax3(mx1, s[i + 2], s[i + 3]);
+    mx2 = fmax3(mx2, s[i + 4], s[i + 5]);
+    mx3 = fmax3(mx3, s[i + 6], s[i + 7]);
   }
+#pragma unroll
+  for (int i = BC - (BC - 12) % 8; i < BC; ++i) mx0 = fmaxf(mx0, s[i]);
   const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
   // +inf when m = -inf and m_new is finite; NaN (false) when both are -inf
   const bool need = (m_new - m) * c > kRescaleLog2;
@@ -75,19 +88,33 @@ __device__ __forceinline__ bool online_softmax_step(float (&s)[BC], float c, flo
     l *= alpha;
   }
   const float nmc = (m == -INFINITY) ? 0.f : -m * c;
-  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+  const float2 c2 = make_float2(c, c), nmc2 = make_float2(nmc, nmc);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
 #pragma unroll
-  for (int i = 0; i < BC; i += 4) {
-    s[i] = ex2(fmaf(s[i], c, nmc));
-    s[i + 1] = ex2(fmaf(s[i + 1], c, nmc));
-    s[i + 2] = ex2(fmaf(s[i + 2], c, nmc));
-    s[i + 3] = ex2(fmaf(s[i + 3], c, nmc));
-    l0 += s[i];
-    l1 += s[i + 1];
-    l2 += s[i + 2];
-    l3 += s[i + 3];
+  for (int i = 0; i < BC; i += 8) {
+    float2 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = ffma2(make_float2(s[i + 2 * u], s[i + 2 * u + 1]), c2, nmc2);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float2 e;
+      if (2 * u < SOFT8) {
+        e = exp2_poly2(x[u]);
+      } else {
+        e.x = ex2(x[u].x);
+        e.y = ex2(x[u].y);
+      }
+      s[i + 2 * u] = e.x;
+      s[i + 2 * u + 1] = e.y;
+    }
+    acc0 = fadd2(acc0, make_float2(s[i], s[i + 1]));
+    acc1 = fadd2(acc1, make_float2(s[i + 2], s[i + 3]));
+    acc2 = fadd2(acc2, make_float2(s[i + 4], s[i + 5]));
+    acc3 = fadd2(acc3, make_float2(s[i + 6], s[i + 7]));
   }
-  l += (l0 + l1) + (l2 + l3);
+  const float2 a01 = fadd2(acc0, acc1), a23 = fadd2(acc2, acc3);
+  const float2 a = fadd2(a01, a23);
+  l += a.x + a.y;
   return warp_rescale;
 }
 
@@ -302,7 +329,7 @@ __global__ void __launch_bounds__(384, 1)
       tmem_load_row<128>(s_addr, s);
       apply_mask<128>(s, col_limit(128 * j, qrow, p.N, p.causal, 128));
       float alpha;
-      const bool rescaled = online_softmax_step<128>(s, p.c, m, l, alpha);
+      const bool rescaled = online_softmax_step<128, kSoftExp8>(s, p.c, m, l, alpha);
       tmem_store_p<128, C::TF32>(s_addr, s);
       if (rescaled && j > 0) tmem_scale_row<D>(o_addr, alpha);
       tmem_wait_st();
@@ -534,7 +561,7 @@ __global__ void __launch_bounds__(256, 1)
       tmem_load_row<BC>(s_addr, s);
       apply_mask<BC>(s, col_limit(BC * j, qrow, p.N, p.causal, BC));
       float alpha;
-      const bool rescaled = online_softmax_step<BC>(s, p.c, m, l, alpha);
+      const bool rescaled = online_softmax_step<BC, 0>(s, p.c, m, l, alpha);
       tmem_store_p<BC, false>(s_addr, s);
       if (rescaled && j > 0) {
         // O must hold every P V product up to tile j-1 before it is rescaled.

@@ -297,6 +297,68 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed two-lane fp32 arithmetic (sm_100 f32x2 instructions).
+__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long r) {
+  float2 o;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+  return o;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)), "l"(f2_pack(c.x, c.y)));
+  return f2_unpack(r);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)));
+  return f2_unpack(r);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)));
+  return f2_unpack(r);
+}
+
+// 2^x on the FMA pipes for two lanes, x <= 2^22 (x is clamped below at -126):
+// Cody-Waite style split x = n + f with n = round-to-nearest(x) (obtained by
+// adding 1.5 * 2^23, which leaves n in the low mantissa bits) and
+// f in [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted by this project for
+// minimum relative error on [-0.5, 0.5] (csrc/fit_exp2_poly.py; max relative
+// error 7.5e-5 in fp32 Horner arithmetic); 2^n is added to the exponent field.
+constexpr float kExp2P0 = 0.9999280571937561f;
+constexpr float kExp2P1 = 0.6932609677314758f;
+constexpr float kExp2P2 = 0.2426111400127411f;
+constexpr float kExp2P3 = 0.0551716685295105f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fsub2(t, make_float2(kRound, kRound));
+  const float2 f = fsub2(x, n);
+  float2 q = ffma2(f, make_float2(kExp2P3, kExp2P3), make_float2(kExp2P2, kExp2P2));
+  q = ffma2(q, f, make_float2(kExp2P1, kExp2P1));
+  q = ffma2(q, f, make_float2(kExp2P0, kExp2P0));
+  float2 r;
+  r.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+  r.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

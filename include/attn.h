@@ -142,6 +142,13 @@ ATTN_API void attn_debug_set_flags(int flags);
  */
 ATTN_API void attn_debug_set_bwd_events(void* start, void* stop);
 
+/*
+ * Test hook for the exponential the softmax kernels use: y[i] = 2^x[i] for
+ * n device floats, computed by the MUFU unit (mode 0) or by the FMA-pipe
+ * polynomial (mode 1), asynchronously on `stream`.
+ */
+ATTN_API attn_status_t attn_debug_exp2(const float* x, float* y, int n, int mode, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
