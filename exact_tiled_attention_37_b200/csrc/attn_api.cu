@@ -137,7 +137,7 @@ attn_status_t launch_pingpong(const attn_tensor_t& q, const attn_tensor_t& k,
   if ((s = make_map(&tv, v, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
   auto kern = eta::fwd_pingpong_kernel<T, D, NS>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
-  dim3 grid((N + 255) / 256, Hq, B);
+  dim3 grid(Hq, B, (N + 255) / 256);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
   return last_launch();
 }
@@ -154,7 +154,7 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
   if ((s = make_map(&tv, v, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
   auto kern = eta::fwd_single_kernel<D, BC, NS>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
-  dim3 grid((N + 127) / 128, Hq, B);
+  dim3 grid(Hq, B, (N + 127) / 128);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
   return last_launch();
 }
@@ -170,17 +170,33 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
   if ((s = make_map(&tdo, dout, p.B, p.Hq, p.N, D, 2, C::BR)) != ATTN_OK) return s;
   if ((s = make_map(&tk, k, p.B, p.Hkv, p.N, D, 2, C::BC)) != ATTN_OK) return s;
   if ((s = make_map(&tv, v, p.B, p.Hkv, p.N, D, 2, C::BC)) != ATTN_OK) return s;
+  // fp32 dQ scratch as a (D, N, B*Hq) tensor; boxes of 32 columns x 64 rows
+  CUtensorMap tdq;
+  {
+    auto enc = encode_fn();
+    if (!enc) return ATTN_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(p.N),
+                          static_cast<cuuint64_t>(p.B) * p.Hq};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4,
+                             static_cast<cuuint64_t>(D) * 4 * p.N};
+    cuuint32_t box[3] = {32u, static_cast<cuuint32_t>(C::BR), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (enc(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.dqacc, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ATTN_ERR_CUDA;
+  }
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
   eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
   auto kern = eta::bwd_dkdv_kernel<D, NQS, NPB>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
-  dim3 grid((p.N + C::BC - 1) / C::BC, p.Hkv * C::DSPLIT, p.B);
+  dim3 grid(p.Hkv * C::DSPLIT, p.B, (p.N + C::BC - 1) / C::BC);
   cudaEvent_t ev0 = static_cast<cudaEvent_t>(g_bwd_ev_start.exchange(nullptr));
   cudaEvent_t ev1 = static_cast<cudaEvent_t>(g_bwd_ev_stop.exchange(nullptr));
   const bool timed = ev0 && ev1;
   if (timed && cudaEventRecord(ev0, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
   if ((s = last_launch()) != ATTN_OK) return s;
   if (timed && cudaEventRecord(ev1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   const long long vec = static_cast<long long>(p.B) * p.Hq * p.N * (D / 8);
@@ -191,7 +207,7 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
 attn_status_t check_sizes(int B, int Hq, int Hkv, int N) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535 || (N + 63) / 64 > 65535) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 

@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(256) bwd_dq_finalize_kernel(const BwdParams p)
   *reinterpret_cast<uint4*>(dst) = w;
 }
 
-// ---------------------------------------------------------------- dK / dV (+ dQ atomics)
+// ---------------------------------------------------------------- dK / dV (+ dQ reductions)
 template <int DFULL, int NQS, int NPB>
 struct BwdCfg {
   static constexpr int BC = 128;                 // key rows per CTA
@@ -192,6 +192,13 @@ struct BwdCfg {
   static constexpr int QTILE = BR * ROWB;
   static constexpr int PTILE = BC * BR * 2;      // 16 KB: one 128-byte row per key row
   static constexpr int KSTEPS = ROWB / 32;       // S^T / dP^T MMAs over D
+  // dQ_i partials: each drain warp stages its 32 columns x 64 rows (8 KB) in
+  // shared memory and hands them to the TMA engine as one tiled bulk
+  // reduction (when shared memory allows: D = 128), otherwise fp32
+  // reductions from registers.
+  static constexpr bool DQ_BULK = DFULL == DH;
+  static constexpr int DQWARP = BR * 32 * 4;                 // 8 KB per drain warp
+  static constexpr int DQTILE = DQ_BULK ? 4 * DQWARP : 0;    // 32 KB
   // TMEM columns
   static constexpr int T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 384, TMEM_COLS = 512;
   // shared memory
@@ -201,7 +208,8 @@ struct BwdCfg {
   static constexpr int S_DO = S_Q + NQS * QTILE;           // [NQS] dO tiles
   static constexpr int S_P = S_DO + NQS * QTILE;           // [NPB] P^T
   static constexpr int S_DS = S_P + NPB * PTILE;           // [NPB] dS^T
-  static constexpr int S_STAT = S_DS + NPB * PTILE;        // [NQS] lse2[64], delta[64]
+  static constexpr int S_DQ = S_DS + NPB * PTILE;          // dQ staging
+  static constexpr int S_STAT = S_DQ + DQTILE;             // [NQS] lse2[64], delta[64]
   static constexpr int S_BAR = S_STAT + NQS * 512;
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;
@@ -216,15 +224,52 @@ struct BwdCfg {
   static constexpr int NBAR = 9 + 2 * NQS + 2 * NPB;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = S_MISC + 16 + 1024;
-  static constexpr int THREADS = 384;
+  // warps: 0-3 softmax (even iterations), 4-7 dQ drain, 8-11 softmax (odd
+  // iterations), 12 TMA producer, 13 MMA issuer / TMEM owner, 14-15 idle
+  static constexpr int THREADS = 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+// P^T and dS^T for 32 query columns [c0, c0 + 32) of this thread's key row:
+// loads S^T and dP^T from TMEM, applies exp2 / causal mask / softmax
+// Jacobian, writes both bf16 rows (4 swizzled 16-byte chunks each).
+__device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr, int c0,
+                                             const float* lse2, const float* dlt, float c,
+                                             int ilo, uint8_t* prow, uint8_t* drow, int swz) {
+  uint32_t rs[32], rd[32];
+  tmem_ld32(st_addr + c0, rs);
+  tmem_ld32(dpt_addr + c0, rd);
+  tmem_wait_ld();
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t pw[4], dw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = 8 * u + 2 * e;  // column within this half
+      const float2 l2 = *reinterpret_cast<const float2*>(lse2 + c0 + i);
+      const float2 dd = *reinterpret_cast<const float2*>(dlt + c0 + i);
+      const float2 x = ffma2(make_float2(u2f(rs[i]), u2f(rs[i + 1])), c2,
+                             make_float2(-l2.x, -l2.y));
+      float2 pv = make_float2(ex2(x.x), ex2(x.y));
+      if (c0 + i < ilo) pv.x = 0.f;
+      if (c0 + i + 1 < ilo) pv.y = 0.f;
+      const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
+      pw[e] = pack_bf16x2(pv.x, pv.y);
+      dw[e] = pack_bf16x2(pv.x * g.x, pv.y * g.y);
+    }
+    const int chunk = (c0 >> 3) + u;  // 16-byte chunk index within the 128-byte row
+    const int off = (chunk ^ swz) * 16;
+    *reinterpret_cast<uint4*>(prow + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+    *reinterpret_cast<uint4*>(drow + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+  }
+}
+
 template <int DFULL, int NQS, int NPB>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<DFULL, NQS, NPB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -236,10 +281,12 @@ __global__ void __launch_bounds__(384, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;  // key tile (causal: tile 0 has the most work, starts first)
-  const int hk = blockIdx.y / C::DSPLIT;
-  const int half = blockIdx.y % C::DSPLIT;
-  const int b = blockIdx.z;
+  // grid (Hkv * D-slices, B, key tiles): the key tile varies slowest, and
+  // causal tile 0 (the most work) of every head is dispatched first
+  const int kt = blockIdx.z;
+  const int hk = blockIdx.x / C::DSPLIT;
+  const int half = blockIdx.x % C::DSPLIT;
+  const int b = blockIdx.y;
   const int k0 = kt * C::BC;
   const int nqt = (p.N + C::BR - 1) / C::BR;
   const int i_first = p.causal ? k0 / C::BR : 0;
@@ -267,7 +314,7 @@ __global__ void __launch_bounds__(384, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -278,7 +325,7 @@ __global__ void __launch_bounds__(384, 1)
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 
 #ifdef ETA_TRACE
-  const int tcta = (blockIdx.y == 0 && blockIdx.z == 0) ? (kt == 0 ? 0 : (kt == 16 ? 1 : -1)) : -1;
+  const int tcta = (blockIdx.x == 0 && blockIdx.y == 0) ? (kt == 0 ? 0 : (kt == 16 ? 1 : -1)) : -1;
 #else
   const int tcta = -1;
 #endif
@@ -287,88 +334,66 @@ __global__ void __launch_bounds__(384, 1)
   auto head_of = [&](int it) { return hk * p.group + it / per_head; };
   auto qtile_of = [&](int it) { return i_first + it % per_head; };
 
-  if (warp < 4) {
+  if (warp < 4 || (warp >= 8 && warp < 12)) {
     // ------------------------------------------------ P^T / dS^T rows, then dK / dV epilogue
-    const int j = threadIdx.x;  // key row within the tile == TMEM lane
+    const int par = warp < 4 ? 0 : 1;   // this warpgroup takes iterations of this parity
+    const int j = threadIdx.x & 127;    // key row within the tile == TMEM lane
     const int jg = k0 + j;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
+    for (int it = par; it < n; it += 2) {
       const int buf = it & 1, stage = it % NQS, pb = it % NPB;
       if (!W.wait_warp(BAR(C::B_SP + buf), (it >> 1) & 1, 60)) { ok = false; break; }
       if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 61)) { ok = false; break; }
-      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 0);
+      if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 0);
+      // the MMAs that read this P/dS buffer NPB iterations ago must be done
+      if (!W.wait_warp(BAR(C::B_PE + pb), ((it / NPB) & 1) ^ 1, 62)) { ok = false; break; }
+      if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 1);
       tc_fence_after();
-      float s[64], dp[64];
-      tmem_load_row<64>(tmem + lane_base + C::T_ST + 64 * buf, s);
-      tmem_load_row<64>(tmem + lane_base + C::T_DPT + 64 * buf, dp);
       const float* lse2 = reinterpret_cast<const float*>(smem + C::S_STAT + stage * 512);
       const float* dlt = lse2 + 64;
       const int ig0 = qtile_of(it) * C::BR;
       // causal: query i sees key j iff jg <= ig0 + i  ->  valid for i >= jg - ig0
       const int ilo = p.causal ? jg - ig0 : -1;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        float pv = ex2(fmaf(s[i], p.c, -lse2[i]));
-        if (i < ilo) pv = 0.f;
-        s[i] = pv;
-        dp[i] = pv * (dp[i] - dlt[i]);
-      }
-      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 1);
-      // the MMAs that read this P/dS buffer NPB iterations ago must be done
-      if (!W.wait_warp(BAR(C::B_PE + pb), ((it / NPB) & 1) ^ 1, 62)) { ok = false; break; }
-      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 2);
       uint8_t* prow = smem + C::S_P + pb * C::PTILE + j * 128;
       uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int sw = (u ^ (j & 7)) * 16;
-        uint4 a, d;
-        a.x = pack_bf16x2(s[8 * u + 0], s[8 * u + 1]);
-        a.y = pack_bf16x2(s[8 * u + 2], s[8 * u + 3]);
-        a.z = pack_bf16x2(s[8 * u + 4], s[8 * u + 5]);
-        a.w = pack_bf16x2(s[8 * u + 6], s[8 * u + 7]);
-        d.x = pack_bf16x2(dp[8 * u + 0], dp[8 * u + 1]);
-        d.y = pack_bf16x2(dp[8 * u + 2], dp[8 * u + 3]);
-        d.z = pack_bf16x2(dp[8 * u + 4], dp[8 * u + 5]);
-        d.w = pack_bf16x2(dp[8 * u + 6], dp[8 * u + 7]);
-        *reinterpret_cast<uint4*>(prow + sw) = a;
-        *reinterpret_cast<uint4*>(drow + sw) = d;
-      }
+      const uint32_t st_addr = tmem + lane_base + C::T_ST + 64 * buf;
+      const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + 64 * buf;
+      bwd_row_half(st_addr, dpt_addr, 0, lse2, dlt, p.c, ilo, prow, drow, j & 7);
+      bwd_row_half(st_addr, dpt_addr, 32, lse2, dlt, p.c, ilo, prow, drow, j & 7);
+      if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 2);
       fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DS + pb));
-      if (threadIdx.x == 0) ETA_TRACE_AT(tcta, 0, it, 3);
+      if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 3);
     }
     if (ok && W.wait_warp(BAR(C::B_KVD), 0, 63)) {
       tc_fence_after();
+      // even warpgroup stores dV, odd warpgroup stores dK (x scale)
       const bool valid = jg < p.N;
-      __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
-                             static_cast<long long>(jg) * p.dvsn + half * C::DH;
-      __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
-                             static_cast<long long>(jg) * p.dksn + half * C::DH;
+      __nv_bfloat16* row =
+          par == 0 ? static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
+                         static_cast<long long>(jg) * p.dvsn + half * C::DH
+                   : static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
+                         static_cast<long long>(jg) * p.dksn + half * C::DH;
+      const float mul = par ? p.scale : 1.f;
+      const uint32_t col = par ? C::T_DK : C::T_DV;
 #pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        __nv_bfloat16* row = t ? dkrow : dvrow;
-        const float mul = t ? p.scale : 1.f;
-        const uint32_t col = t ? C::T_DK : C::T_DV;
-#pragma unroll 1
-        for (int c = 0; c < C::DH / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + col + 32 * c, r);
-          tmem_wait_ld();
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(row + 32 * c);
+      for (int c = 0; c < C::DH / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + col + 32 * c, r);
+        tmem_wait_ld();
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(row + 32 * c);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16x2(u2f(r[8 * v + 0]) * mul, u2f(r[8 * v + 1]) * mul);
-              w.y = pack_bf16x2(u2f(r[8 * v + 2]) * mul, u2f(r[8 * v + 3]) * mul);
-              w.z = pack_bf16x2(u2f(r[8 * v + 4]) * mul, u2f(r[8 * v + 5]) * mul);
-              w.w = pack_bf16x2(u2f(r[8 * v + 6]) * mul, u2f(r[8 * v + 7]) * mul);
-              dst[v] = w;
-            }
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(u2f(r[8 * v + 0]) * mul, u2f(r[8 * v + 1]) * mul);
+            w.y = pack_bf16x2(u2f(r[8 * v + 2]) * mul, u2f(r[8 * v + 3]) * mul);
+            w.z = pack_bf16x2(u2f(r[8 * v + 4]) * mul, u2f(r[8 * v + 5]) * mul);
+            w.w = pack_bf16x2(u2f(r[8 * v + 6]) * mul, u2f(r[8 * v + 7]) * mul);
+            dst[v] = w;
           }
         }
       }
@@ -377,6 +402,8 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------ dQ^T drain -> fp32 reductions
     const int dd = threadIdx.x - 128;  // column of this CTA's D slice == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int dw = warp & 3;  // drain warp: columns [32 dw, 32 dw + 32) of the D slice
+    float* stage_dq = reinterpret_cast<float*>(smem + C::S_DQ + dw * C::DQWARP);
     for (int it = 0; it < n; ++it) {
       const int buf = it & 1;
       if (!W.wait_warp(BAR(C::B_DQF + buf), (it >> 1) & 1, 70)) break;
@@ -390,15 +417,36 @@ __global__ void __launch_bounds__(384, 1)
       if (threadIdx.x == 128) ETA_TRACE_AT(tcta, 1, it, 1);
       const int h = head_of(it);
       const int ig0 = qtile_of(it) * C::BR;
-      float* dst = p.dqacc + (static_cast<long long>(b * p.Hq + h) * p.N + ig0) * DFULL +
-                   half * C::DH + dd;
       const int imax = min(64, p.N - ig0);
+      float* dst = p.dqacc + (static_cast<long long>(b * p.Hq + h) * p.N + ig0) * DFULL;
+      if constexpr (C::DQ_BULK) {
+        // this warp's previous reduction must have finished reading its staging box
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if (i < imax) atomicAdd(dst + static_cast<long long>(i) * DFULL, v[i] * p.scale);
+        for (int i = 0; i < 64; ++i) stage_dq[i * 32 + lane] = v[i] * p.scale;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // box of 32 columns x 64 rows of the (D, N, B*Hq) scratch; rows past N are skipped
+          tma_reduce_add_3d(&tm_dq, smem_u32(stage_dq), half * C::DH + 32 * dw, ig0, b * p.Hq + h);
+          bulk_commit();
+        }
+        (void)imax;
+        (void)dst;
+      } else {
+        float* col = dst + half * C::DH + dd;
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i < imax) atomicAdd(col + static_cast<long long>(i) * DFULL, v[i] * p.scale);
+      }
       if (threadIdx.x == 128) ETA_TRACE_AT(tcta, 1, it, 2);
     }
-  } else if (warp == 8) {
+    if constexpr (C::DQ_BULK) {
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
+    }
+  } else if (warp == 12) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -435,7 +483,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_make(128, 64, 1u, false, false);      // S^T, dP^T
@@ -523,7 +571,7 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -273,8 +273,10 @@ __global__ void __launch_bounds__(384, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest causal CTAs first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (Hq, B, query blocks): the block index varies slowest so that every
+  // head's longest causal CTAs are dispatched first
+  const int qb = gridDim.z - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / p.group;
   const int q0 = qb * 256;
   int ntile[2];
@@ -512,8 +514,10 @@ __global__ void __launch_bounds__(256, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = gridDim.x - 1 - blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (Hq, B, query blocks): the block index varies slowest so that every
+  // head's longest causal CTAs are dispatched first
+  const int qb = gridDim.z - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / p.group;
   const int q0 = qb * 128;
   const int kv_end = p.causal ? min(p.N, q0 + 128) : p.N;

@@ -141,6 +141,30 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Bulk-group bookkeeping is per issuing thread.
+// Wait until no committed bulk group is still reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk group has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Tiled bulk reduction (fp32 add) of a shared-memory box into the 3-D tensor
+// described by `m` at coordinates (c0, c1, c2); elements outside the tensor
+// are skipped.  Coordinates must be non-negative.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, uint32_t ssrc, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(ssrc), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
