@@ -373,3 +373,46 @@ attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- backward without allocation
+// Fixed scratch used by attn_bwd_noalloc in place of a caller-provided
+// workspace.  In host code the name below is only a host-side stand-in for
+// the array; its device address comes from cudaGetSymbolAddress, once per
+// device, with that device current.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+attn_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                          attn_tensor_t o, const float* lse, attn_tensor_t dout,
+                                          attn_tensor_t dq, attn_tensor_t dk, attn_tensor_t dv,
+                                          int B, int Hq, int Hkv, int N, int D,
+                                          attn_dtype_t dtype, int causal, float scale,
+                                          void* stream) {
+  const size_t need = attn_bwd_workspace_bytes(B, Hq, N, D);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* ws = nullptr;
+  attn_status_t s = noalloc_scratch(&ws);
+  if (s != ATTN_OK) return s;
+  return attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, dtype, causal, scale, ws,
+                  kNoAllocScratchBytes, stream);
+}

@@ -117,6 +117,36 @@ ATTN_API attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t 
                        size_t workspace_bytes, void* stream);
 
 /*
+ * attn_bwd for callers that cannot allocate device memory.
+ *
+ * Some callers must not allocate GPU memory once they are running: a service
+ * that reserves all of its device memory up front and forbids any later
+ * cudaMalloc, or a host framework whose own allocator this library cannot
+ * reach.  They cannot provide attn_bwd's workspace, so this entry point uses
+ * a fixed scratch array that is part of the library itself (a static device
+ * array of 64 MiB = 67108864 bytes; every GPU on which the library is loaded
+ * holds it until the process exits).  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.  (This entry point has no counterpart in the
+ * method's description; it only changes where the backward's scratch lives.)
+ *
+ * Arguments and results are those of attn_bwd without the workspace.  Sizes
+ * whose workspace (attn_bwd_workspace_bytes) exceeds 64 MiB are rejected with
+ * ATTN_ERR_WORKSPACE before anything is launched.  The first call on each
+ * device looks up the scratch array's device address with that device
+ * current; make that first call before any stream capture.  Every call
+ * shares the one array: the kernels re-initialise everything they read from
+ * it (the dQ accumulator is zeroed and the row statistics rewritten on every
+ * call), but two calls whose work overlaps on the GPU (different streams, or
+ * different host threads) race on it and must be serialised by the caller.
+ */
+ATTN_API attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                        attn_tensor_t o, const float* lse, attn_tensor_t dout,
+                                        attn_tensor_t dq, attn_tensor_t dk, attn_tensor_t dv,
+                                        int B, int Hq, int Hkv, int N, int D,
+                                        attn_dtype_t dtype, int causal, float scale,
+                                        void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a kernel's
  * bounded wait gave up; *where, if not NULL, receives the wait site id) or
