@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD_INDEX = 2  # MHA fwd+bwd B=2 H=16 N=4096 D=128 causal
 
-# DRAM traffic of one launch of the dominant kernel (bwd_dkdv_kernel<128,2,2>)
+# DRAM traffic of one launch of the dominant kernel (bwd_dkdv_kernel<128,3,2>)
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the kernel source it was taken on; it is reported as null once the
 # source changes.  See profiles/ for the capture summary and command.
@@ -41,7 +41,7 @@ DOMINANT_TRAFFIC = {"bytes": None, "src_sha": None}
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -273,29 +273,64 @@ def run_native(args):
     bwd_ms = timed(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dq, dk=dk, dv=dv,
                                     workspace=ws), min(K, 50))
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, fwd + bwd, D2H of the gradients
-    out_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
-    h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    # end to end through the public API with host buffers: every step uploads
+    # its inputs (pinned Q, K, V, dO), runs forward + backward and downloads its
+    # gradients (dQ, dK, dV).  Uploads run on one stream, compute on another,
+    # downloads on a third, double-buffered, so step i+1's upload and step
+    # i-1's download overlap step i's compute (as a user pipeline would).
     n_e2e = max(3, min(K, 20))
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    dbuf = [[torch.empty_like(t, device=dev) for t in host] for _ in range(2)]
+    gbuf = [[torch.empty_like(t) for t in (dq, dk, dv)] for _ in range(2)]
+    hout = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
+            for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = sum(t.numel() * t.element_size() for t in hout[0])
 
-    def e2e_step():
-        qq, kk, vv, dd = (t.to(dev, non_blocking=True) for t in host)
-        oo, ll = attn_fwd(qq, kk, vv, causal=causal)
-        g = attn_bwd(qq, kk, vv, oo, ll, dd, causal=causal, workspace=ws)
-        for hst, dvc in zip(out_host, g):
-            hst.copy_(dvc, non_blocking=True)
+    def e2e_run(n):
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        for e in ev_comp + ev_out:
+            e.record(stream)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_in.wait_stream(stream)
+        s_comp.wait_stream(stream)
+        s_out.wait_stream(stream)
+        start.record(s_in)
+        for i in range(n + 2):
+            if i < n:
+                with torch.cuda.stream(s_in):
+                    s_in.wait_event(ev_comp[i % 2])
+                    for d_, h_ in zip(dbuf[i % 2], host):
+                        d_.copy_(h_, non_blocking=True)
+                    ev_in[i % 2].record(s_in)
+            if 1 <= i <= n:
+                j = i - 1
+                with torch.cuda.stream(s_comp):
+                    s_comp.wait_event(ev_in[j % 2])
+                    s_comp.wait_event(ev_out[j % 2])
+                    qq, kk, vv, dd = dbuf[j % 2]
+                    oo, ll = attn_fwd(qq, kk, vv, causal=causal)
+                    g0, g1, g2 = gbuf[j % 2]
+                    attn_bwd(qq, kk, vv, oo, ll, dd, causal=causal, dq=g0, dk=g1, dv=g2,
+                             workspace=ws)
+                    ev_comp[j % 2].record(s_comp)
+            if i >= 2:
+                j = i - 2
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_comp[j % 2])
+                    for h_, d_ in zip(hout[j % 2], gbuf[j % 2]):
+                        h_.copy_(d_, non_blocking=True)
+                    ev_out[j % 2].record(s_out)
+        stop.record(s_out)
+        stop.synchronize()
+        return start.elapsed_time(stop) / n
 
-    e2e_step()
+    e2e_run(2)
     barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    b.record(stream)
+    e2e_ms = e2e_run(n_e2e)
     barrier()
-    e2e_ms = a.elapsed_time(b) / n_e2e
 
     flops_step = w.fwd_flops(causal) + w.bwd_flops(causal)
     ms_per_step, e2e_ms = max_over_ranks([total_ms / K, e2e_ms], dev)
@@ -332,13 +367,14 @@ def run_native(args):
                 "frac_of_peak": round(w.fwd_flops(causal) / fwd_ms / 1e9 / peaks["bf16_tflops"], 4)},
         "bwd": {"ms": round(bwd_ms, 4), "tflops": round(w.bwd_flops(causal) / bwd_ms / 1e9, 1),
                 "frac_of_peak": round(w.bwd_flops(causal) / bwd_ms / 1e9 / peaks["bf16_tflops"], 4)},
-        "roofline": {"kernel": "bwd_dkdv_kernel<128,2,2>", "bound": "tensor",
+        "roofline": {"kernel": "bwd_dkdv_kernel<128,3,2>", "bound": "tensor",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16 sustained",
                      "launch_ms": round(dom_ms, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "pipeline": "upload / compute / download on three streams, double-buffered"},
         "clocks": clk,
         "gpu_launches": 4 * K,
     }

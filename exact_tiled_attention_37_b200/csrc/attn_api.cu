@@ -242,6 +242,10 @@ void attn_debug_set_bwd_events(void* start, void* stop) {
 }
 
 #ifdef ETA_TRACE
+ATTN_API int attn_debug_read_ftrace(void* dst, size_t bytes) {
+  if (bytes > sizeof(eta::g_eta_ftrace)) bytes = sizeof(eta::g_eta_ftrace);
+  return cudaMemcpyFromSymbol(dst, eta::g_eta_ftrace, bytes) == cudaSuccess ? 0 : 1;
+}
 ATTN_API int attn_debug_read_trace(void* dst, size_t bytes) {
   if (bytes > sizeof(eta::g_eta_trace)) bytes = sizeof(eta::g_eta_trace);
   return cudaMemcpyFromSymbol(dst, eta::g_eta_trace, bytes) == cudaSuccess ? 0 : 1;
@@ -368,7 +372,7 @@ attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
   p.wait_limit_ns = g_wait_limit_ns.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_bwd<128, 2, 2>(q, k, v, dout, p, st);
+  if (D == 128) return launch_bwd<128, 3, 2>(q, k, v, dout, p, st);
   return launch_bwd<256, 1, 1>(q, k, v, dout, p, st);
 }
 

@@ -190,7 +190,7 @@ struct BwdCfg {
   static constexpr int QCHUNK = BR * 128;        // 8 KB
   static constexpr int KTILE = BC * ROWB;
   static constexpr int QTILE = BR * ROWB;
-  static constexpr int PTILE = BC * BR * 2;      // 16 KB: one 128-byte row per key row
+  static constexpr int PTILE = BC * BR * 2;      // 16 KB dS^T: one 128-byte row per key row
   static constexpr int KSTEPS = ROWB / 32;       // S^T / dP^T MMAs over D
   // dQ_i partials: each drain warp stages its 32 columns x 64 rows (8 KB) in
   // shared memory and hands them to the TMA engine as one tiled bulk
@@ -206,8 +206,7 @@ struct BwdCfg {
   static constexpr int S_V = S_K + KTILE;
   static constexpr int S_Q = S_V + KTILE;                  // [NQS] Q tiles
   static constexpr int S_DO = S_Q + NQS * QTILE;           // [NQS] dO tiles
-  static constexpr int S_P = S_DO + NQS * QTILE;           // [NPB] P^T
-  static constexpr int S_DS = S_P + NPB * PTILE;           // [NPB] dS^T
+  static constexpr int S_DS = S_DO + NQS * QTILE;          // [NPB] dS^T
   static constexpr int S_DQ = S_DS + NPB * PTILE;          // dQ staging
   static constexpr int S_STAT = S_DQ + DQTILE;             // [NQS] lse2[64], delta[64]
   static constexpr int S_BAR = S_STAT + NQS * 512;
@@ -232,18 +231,21 @@ struct BwdCfg {
 
 // P^T and dS^T for 32 query columns [c0, c0 + 32) of this thread's key row:
 // loads S^T and dP^T from TMEM, applies exp2 / causal mask / softmax
-// Jacobian, writes both bf16 rows (4 swizzled 16-byte chunks each).
+// Jacobian, writes P^T as bf16 pairs back into the S^T columns it has read
+// (TMEM columns c0/2 .. c0/2 + 15, the A operand of dV += P^T dO) and dS^T
+// as a bf16 shared-memory row (4 swizzled 16-byte chunks).
 __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr, int c0,
                                              const float* lse2, const float* dlt, float c,
-                                             int ilo, uint8_t* prow, uint8_t* drow, int swz) {
+                                             int ilo, uint8_t* drow, int swz) {
   uint32_t rs[32], rd[32];
   tmem_ld32(st_addr + c0, rs);
   tmem_ld32(dpt_addr + c0, rd);
   tmem_wait_ld();
   const float2 c2 = make_float2(c, c);
+  uint32_t pk[16];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    uint32_t pw[4], dw[4];
+    uint32_t dw[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int i = 8 * u + 2 * e;  // column within this half
@@ -255,14 +257,14 @@ __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr
       if (c0 + i < ilo) pv.x = 0.f;
       if (c0 + i + 1 < ilo) pv.y = 0.f;
       const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
-      pw[e] = pack_bf16x2(pv.x, pv.y);
+      pk[4 * u + e] = pack_bf16x2(pv.x, pv.y);
       dw[e] = pack_bf16x2(pv.x * g.x, pv.y * g.y);
     }
     const int chunk = (c0 >> 3) + u;  // 16-byte chunk index within the 128-byte row
     const int off = (chunk ^ swz) * 16;
-    *reinterpret_cast<uint4*>(prow + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
     *reinterpret_cast<uint4*>(drow + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
   }
+  tmem_st16(st_addr + c0 / 2, pk);
 }
 
 template <int DFULL, int NQS, int NPB>
@@ -355,13 +357,13 @@ __global__ void __launch_bounds__(512, 1)
       const int ig0 = qtile_of(it) * C::BR;
       // causal: query i sees key j iff jg <= ig0 + i  ->  valid for i >= jg - ig0
       const int ilo = p.causal ? jg - ig0 : -1;
-      uint8_t* prow = smem + C::S_P + pb * C::PTILE + j * 128;
       uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
       const uint32_t st_addr = tmem + lane_base + C::T_ST + 64 * buf;
       const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + 64 * buf;
-      bwd_row_half(st_addr, dpt_addr, 0, lse2, dlt, p.c, ilo, prow, drow, j & 7);
-      bwd_row_half(st_addr, dpt_addr, 32, lse2, dlt, p.c, ilo, prow, drow, j & 7);
+      bwd_row_half(st_addr, dpt_addr, 0, lse2, dlt, p.c, ilo, drow, j & 7);
+      bwd_row_half(st_addr, dpt_addr, 32, lse2, dlt, p.c, ilo, drow, j & 7);
       if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 2);
+      tmem_wait_st();
       fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
       tc_fence_before();
       __syncwarp();
@@ -538,19 +540,19 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         const uint32_t sq = sbase + C::S_Q + stage * C::QTILE + half * 2 * C::QCHUNK;
         const uint32_t sdo = sbase + C::S_DO + stage * C::QTILE + half * 2 * C::QCHUNK;
-        const uint32_t sp = sbase + C::S_P + pb * C::PTILE;
         const uint32_t sds = sbase + C::S_DS + pb * C::PTILE;
-        // dV += P^T dO_i (K = 64 query rows, 4 steps of 16)
+        // dV += P^T dO_i with P^T read from TMEM (K = 64 query rows, 4 steps of 16)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ss<false>(tmem + C::T_DV, sdesc_sw128(sp + ks * 32, 16, 1024),
+          mma_ts<false>(tmem + C::T_DV, tmem + C::T_ST + 64 * buf + 8 * ks,
                         sdesc_sw128(sdo + ks * 2048, C::QCHUNK, 1024), id_kv, (it > 0 || ks > 0));
         // dK += dS^T Q_i
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_ss<false>(tmem + C::T_DK, sdesc_sw128(sds + ks * 32, 16, 1024),
                         sdesc_sw128(sq + ks * 2048, C::QCHUNK, 1024), id_kv, (it > 0 || ks > 0));
-        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed S^T buffer
+        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed S^T
+        // buffer; issued after dV, whose P^T operand lives in those columns
         const uint32_t kh = sK + half * 2 * C::KCHUNK;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)

@@ -38,9 +38,23 @@ constexpr float kRescaleLog2 = 8.0f;
 // Columns (of every 8) whose exponential the ping-pong kernel computes with
 // the FMA-pipe polynomial; the rest use the MUFU ex2 unit.
 #ifndef ETA_SOFT_EXP8
-#define ETA_SOFT_EXP8 2
+#define ETA_SOFT_EXP8 0
 #endif
 constexpr int kSoftExp8 = ETA_SOFT_EXP8;
+
+#ifdef ETA_TRACE
+// Debug builds only: clock64() timelines of two CTAs of the ping-pong kernel
+// ([cta][role: softmax 0, softmax 1, MMA][key tile][event]).
+__device__ unsigned long long g_eta_ftrace[2][3][256][4];
+#define ETA_FTRACE_AT(cta, role, it, ev)                                          \
+  do {                                                                           \
+    if ((cta) >= 0 && (it) < 256) g_eta_ftrace[(cta)][(role)][(it)][(ev)] = clock64(); \
+  } while (0)
+#else
+#define ETA_FTRACE_AT(cta, role, it, ev) \
+  do {                                   \
+  } while (0)
+#endif
 
 struct FwdParams {
   void* o;           // [B, Hq, N, D], unit stride on D
@@ -313,6 +327,12 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+#ifdef ETA_TRACE
+  const int tcta = (h == 0 && b == 0) ? (qb == (int)gridDim.z - 1 ? 0 : (qb == (int)gridDim.z / 2 ? 1 : -1)) : -1;
+#else
+  const int tcta = -1;
+#endif
+  (void)tcta;
 
   if (warp < 8) {
     // ------------------------------------------------ softmax / correction / epilogue
@@ -326,18 +346,22 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int j = 0; j < ntile[t]; ++j) {
       if (!W.wait_warp(BAR(C::BAR_S + t), j & 1, 10 + t)) { ok = false; break; }
+      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 0);
       tc_fence_after();
       float s[128];
       tmem_load_row<128>(s_addr, s);
+      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 1);
       apply_mask<128>(s, col_limit(128 * j, qrow, p.N, p.causal, 128));
       float alpha;
       const bool rescaled = online_softmax_step<128, kSoftExp8>(s, p.c, m, l, alpha);
+      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 2);
       tmem_store_p<128, C::TF32>(s_addr, s);
       if (rescaled && j > 0) tmem_scale_row<D>(o_addr, alpha);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::BAR_P + t));
+      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 3);
     }
     if (ok && ntile[t] > 0 && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
       tc_fence_after();
@@ -419,6 +443,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 42)) { ok = false; break; }
         if (use0) {
           if (!W.wait(BAR(C::BAR_P + 0), j & 1, 43)) { ok = false; break; }
+          ETA_FTRACE_AT(tcta, 2, j, 0);
           tc_fence_after();
           issue_pv(0, vslot(j), j > 0);
           if (!use1) mma_commit(BAR(C::BAR_KVE + vslot(j)));
@@ -426,6 +451,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 44)) { ok = false; break; }
             issue_s(0, kslot(j + 1));
             mma_commit(BAR(C::BAR_S + 0));
+            ETA_FTRACE_AT(tcta, 2, j, 1);
             if (!nxt1) mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
           } else {
             mma_commit(BAR(C::BAR_O + 0));
@@ -433,6 +459,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (use1) {
           if (!W.wait(BAR(C::BAR_P + 1), j & 1, 45)) { ok = false; break; }
+          ETA_FTRACE_AT(tcta, 2, j, 2);
           tc_fence_after();
           issue_pv(1, vslot(j), j > 0);
           mma_commit(BAR(C::BAR_KVE + vslot(j)));
@@ -440,6 +467,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 46)) { ok = false; break; }
             issue_s(1, kslot(j + 1));
             mma_commit(BAR(C::BAR_S + 1));
+            ETA_FTRACE_AT(tcta, 2, j, 3);
             mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
           } else {
             mma_commit(BAR(C::BAR_O + 1));
