@@ -231,9 +231,10 @@ struct BwdCfg {
 
 // P^T and dS^T for 32 query columns [c0, c0 + 32) of this thread's key row:
 // loads S^T and dP^T from TMEM, applies exp2 / causal mask / softmax
-// Jacobian, writes P^T as bf16 pairs back into the S^T columns it has read
-// (TMEM columns c0/2 .. c0/2 + 15, the A operand of dV += P^T dO) and dS^T
-// as a bf16 shared-memory row (4 swizzled 16-byte chunks).
+// Jacobian, writes P^T and dS^T as bf16 pairs back into the S^T and dP^T
+// columns it has read (TMEM columns c0/2 .. c0/2 + 15: the A operands of
+// dV += P^T dO and dK += dS^T Q) and dS^T also as a bf16 shared-memory row
+// (4 swizzled 16-byte chunks: the B operand of dQ^T = K^T dS^T).
 __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr, int c0,
                                              const float* lse2, const float* dlt, float c,
                                              int ilo, uint8_t* drow, int swz) {
@@ -242,7 +243,7 @@ __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr
   tmem_ld32(dpt_addr + c0, rd);
   tmem_wait_ld();
   const float2 c2 = make_float2(c, c);
-  uint32_t pk[16];
+  uint32_t pk[16], dk[16];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     uint32_t dw[4];
@@ -259,12 +260,14 @@ __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr
       const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
       pk[4 * u + e] = pack_bf16x2(pv.x, pv.y);
       dw[e] = pack_bf16x2(pv.x * g.x, pv.y * g.y);
+      dk[4 * u + e] = dw[e];
     }
     const int chunk = (c0 >> 3) + u;  // 16-byte chunk index within the 128-byte row
     const int off = (chunk ^ swz) * 16;
     *reinterpret_cast<uint4*>(drow + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
   }
   tmem_st16(st_addr + c0 / 2, pk);
+  tmem_st16(dpt_addr + c0 / 2, dk);
 }
 
 template <int DFULL, int NQS, int NPB>
@@ -491,24 +494,26 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t id_s = idesc_make(128, 64, 1u, false, false);      // S^T, dP^T
       constexpr uint32_t id_kv = idesc_make(128, C::DH, 1u, false, true);   // dV, dK
       constexpr uint32_t id_q = idesc_make(128, 64, 1u, true, true);        // dQ^T
-      const uint32_t sK = sbase + C::S_K, sV = sbase + C::S_V;
+      const SDesc dK = sdesc_base(sbase + C::S_K, 16, 1024);
+      const SDesc dV = sdesc_base(sbase + C::S_V, 16, 1024);
+      // K^T for dQ^T: MN-major view of this CTA's D slice of the K tile
+      const SDesc dKt = sdesc_base(sbase + C::S_K + half * 2 * C::KCHUNK, C::KCHUNK, 1024);
       auto issue_sdp = [&](int it) {
         const int buf = it & 1, stage = it % NQS;
-        const uint32_t sq = sbase + C::S_Q + stage * C::QTILE;
-        const uint32_t sdo = sbase + C::S_DO + stage * C::QTILE;
+        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::QTILE, 16, 1024);
+        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::QTILE, 16, 1024);
+        const uint32_t ds = tmem + C::T_ST + 64 * buf, ddp = tmem + C::T_DPT + 64 * buf;
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks) {
           const uint32_t ko = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
           const uint32_t qo = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
-          mma_ss<false>(tmem + C::T_ST + 64 * buf, sdesc_sw128(sK + ko, 16, 1024),
-                        sdesc_sw128(sq + qo, 16, 1024), id_s, ks > 0);
+          mma_ss<false>(ds, sdesc_at(dK, ko), sdesc_at(dq, qo), id_s, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks) {
           const uint32_t ko = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
           const uint32_t qo = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
-          mma_ss<false>(tmem + C::T_DPT + 64 * buf, sdesc_sw128(sV + ko, 16, 1024),
-                        sdesc_sw128(sdo + qo, 16, 1024), id_s, ks > 0);
+          mma_ss<false>(ddp, sdesc_at(dV, ko), sdesc_at(ddo, qo), id_s, ks > 0);
         }
       };
       bool ok = W.wait(BAR(C::B_KV), 0, 90) && (n == 0 || W.wait(BAR(C::B_QF), 0, 91));
@@ -538,26 +543,28 @@ __global__ void __launch_bounds__(512, 1)
         if (!W.wait(BAR(C::B_DS + pb), (it / NPB) & 1, 94)) { ok = false; break; }
         ETA_TRACE_AT(tcta, 2, it, 2);
         tc_fence_after();
-        const uint32_t sq = sbase + C::S_Q + stage * C::QTILE + half * 2 * C::QCHUNK;
-        const uint32_t sdo = sbase + C::S_DO + stage * C::QTILE + half * 2 * C::QCHUNK;
-        const uint32_t sds = sbase + C::S_DS + pb * C::PTILE;
+        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::QTILE + half * 2 * C::QCHUNK,
+                                    C::QCHUNK, 1024);
+        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::QTILE + half * 2 * C::QCHUNK,
+                                     C::QCHUNK, 1024);
+        const SDesc dds = sdesc_base(sbase + C::S_DS + pb * C::PTILE, C::PTILE, 1024);
+        const uint32_t tst = tmem + C::T_ST + 64 * buf, tdp = tmem + C::T_DPT + 64 * buf;
+        const uint32_t acc0 = it > 0 ? 1u : 0u;
         // dV += P^T dO_i with P^T read from TMEM (K = 64 query rows, 4 steps of 16)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts<false>(tmem + C::T_DV, tmem + C::T_ST + 64 * buf + 8 * ks,
-                        sdesc_sw128(sdo + ks * 2048, C::QCHUNK, 1024), id_kv, (it > 0 || ks > 0));
-        // dK += dS^T Q_i
+          mma_ts<false>(tmem + C::T_DV, tst + 8 * ks, sdesc_at(ddo, ks * 2048), id_kv,
+                        ks > 0 ? 1u : acc0);
+        // dK += dS^T Q_i with dS^T read from TMEM
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ss<false>(tmem + C::T_DK, sdesc_sw128(sds + ks * 32, 16, 1024),
-                        sdesc_sw128(sq + ks * 2048, C::QCHUNK, 1024), id_kv, (it > 0 || ks > 0));
+          mma_ts<false>(tmem + C::T_DK, tdp + 8 * ks, sdesc_at(dq, ks * 2048), id_kv,
+                        ks > 0 ? 1u : acc0);
         // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed S^T
         // buffer; issued after dV, whose P^T operand lives in those columns
-        const uint32_t kh = sK + half * 2 * C::KCHUNK;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ss<false>(tmem + C::T_ST + 64 * buf, sdesc_sw128(kh + ks * 2048, C::KCHUNK, 1024),
-                        sdesc_sw128(sds + ks * 2048, C::PTILE, 1024), id_q, ks > 0);
+          mma_ss<false>(tst, sdesc_at(dKt, ks * 2048), sdesc_at(dds, ks * 2048), id_q, ks > 0);
         mma_commit(BAR(C::B_DQF + buf));
         mma_commit(BAR(C::B_QE + stage));
         mma_commit(BAR(C::B_PE + pb));

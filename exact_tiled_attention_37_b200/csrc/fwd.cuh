@@ -412,22 +412,23 @@ __global__ void __launch_bounds__(384, 1)
       auto vslot = [&](int j) { return (2 * j + 1) % NS; };
       auto vph = [&](int j) { return static_cast<uint32_t>((2 * j + 1) / NS) & 1u; };
       auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = sbase + C::SMEM_Q + t * C::TILE;
-        const uint32_t kb = sbase + C::SMEM_KV + slot * C::TILE;
+        const SDesc qa = sdesc_base(sbase + C::SMEM_Q + t * C::TILE, 16, 1024);
+        const SDesc kb = sdesc_base(sbase + C::SMEM_KV + slot * C::TILE, 16, 1024);
+        const uint32_t d = tmem + 128u * t;
 #pragma unroll
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
           const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          mma_ss<C::TF32>(tmem + 128u * t, sdesc_sw128(qa + off, 16, 1024),
-                          sdesc_sw128(kb + off, 16, 1024), idesc_s, ks > 0);
+          mma_ss<C::TF32>(d, sdesc_at(qa, off), sdesc_at(kb, off), idesc_s, ks > 0);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t vb = sbase + C::SMEM_KV + slot * C::TILE;
+        const SDesc vb = sdesc_base(sbase + C::SMEM_KV + slot * C::TILE, C::CHUNK, 1024);
+        const uint32_t d = tmem + C::O_COL + D * t, a = tmem + 128u * t;
+        const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
         for (int ks = 0; ks < C::PV_STEPS; ++ks)
-          mma_ts<C::TF32>(tmem + C::O_COL + D * t, tmem + 128u * t + 8u * ks,
-                          sdesc_sw128(vb + ks * C::PV_ROWS * 128, C::CHUNK, 1024), idesc_o,
-                          (acc || ks > 0) ? 1u : 0u);
+          mma_ts<C::TF32>(d, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128), idesc_o,
+                          ks > 0 ? 1u : acc0);
       };
       const int n0 = ntile[0], n1 = ntile[1];
       bool ok = W.wait(BAR(C::BAR_Q), 0, 40) && W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
@@ -647,24 +648,25 @@ __global__ void __launch_bounds__(256, 1)
       auto kph = [&](int j) { return static_cast<uint32_t>((2 * j) / NS) & 1u; };
       auto vslot = [&](int j) { return (2 * j + 1) % NS; };
       auto vph = [&](int j) { return static_cast<uint32_t>((2 * j + 1) / NS) & 1u; };
+      const SDesc qa = sdesc_base(sbase + C::SMEM_Q, 16, 1024);
       auto issue_s = [&](int buf, int slot) {
-        const uint32_t qa = sbase + C::SMEM_Q;
-        const uint32_t kb = sbase + C::SMEM_KV + slot * C::KTILE;
+        const SDesc kb = sdesc_base(sbase + C::SMEM_KV + slot * C::KTILE, 16, 1024);
+        const uint32_t d = tmem + C::S_COL + BC * buf;
 #pragma unroll
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
           const uint32_t qoff = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
           const uint32_t koff = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
-          mma_ss<false>(tmem + C::S_COL + BC * buf, sdesc_sw128(qa + qoff, 16, 1024),
-                        sdesc_sw128(kb + koff, 16, 1024), idesc_s, ks > 0);
+          mma_ss<false>(d, sdesc_at(qa, qoff), sdesc_at(kb, koff), idesc_s, ks > 0);
         }
       };
       auto issue_pv = [&](int buf, int slot, bool acc) {
-        const uint32_t vb = sbase + C::SMEM_KV + slot * C::KTILE;
+        const SDesc vb = sdesc_base(sbase + C::SMEM_KV + slot * C::KTILE, C::KCHUNK, 1024);
+        const uint32_t a = tmem + C::S_COL + BC * buf;
+        const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
         for (int ks = 0; ks < C::PV_STEPS; ++ks)
-          mma_ts<false>(tmem + C::O_COL, tmem + C::S_COL + BC * buf + 8u * ks,
-                        sdesc_sw128(vb + ks * 16 * 128, C::KCHUNK, 1024), idesc_o,
-                        (acc || ks > 0) ? 1u : 0u);
+          mma_ts<false>(tmem + C::O_COL, a + 8u * ks, sdesc_at(vb, ks * 16 * 128), idesc_o,
+                        ks > 0 ? 1u : acc0);
       };
       bool ok = W.wait(BAR(C::BAR_Q), 0, 40) && W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
       if (ok) {

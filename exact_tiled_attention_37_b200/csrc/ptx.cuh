@@ -200,6 +200,23 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The same descriptor split into its 32-bit halves, so that the issue loop
+// only adds a (compile-time) byte offset to the start-address field of the
+// low half for each MMA: one integer add per operand instead of rebuilding
+// the descriptor.  Offsets must keep the address inside the 14-bit field.
+struct SDesc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc_base(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  SDesc d;
+  d.lo = ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+  d.hi = ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+  return d;
+}
+__device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t byte_off) {
+  return (static_cast<uint64_t>(d.hi) << 32) | static_cast<uint64_t>(d.lo + (byte_off >> 4));
+}
+
 // Instruction descriptor for kind::f16 / kind::tf32 with an f32 accumulator.
 // fmt: 1 = bf16, 2 = tf32.  a_mn / b_mn: operand is MN-major (else K-major).
 __host__ __device__ constexpr uint32_t idesc_make(int M, int N, uint32_t fmt, bool a_mn, bool b_mn) {
