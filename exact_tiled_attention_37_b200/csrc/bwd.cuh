@@ -223,8 +223,9 @@ struct BwdCfg {
   static constexpr int NBAR = 9 + 2 * NQS + 2 * NPB;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = S_MISC + 16 + 1024;
-  // warps: 0-3 softmax (even iterations), 4-7 dQ drain, 8-11 softmax (odd
-  // iterations), 12 TMA producer, 13 MMA issuer / TMEM owner, 14-15 idle
+  // warps: 0-3 softmax (query columns 0-31 of every tile), 4-7 dQ drain,
+  // 8-11 softmax (columns 32-63), 12 TMA producer, 13 MMA issuer / TMEM
+  // owner, 14-15 idle
   static constexpr int THREADS = 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(BAR(C::B_DQE + s), 4);
     }
     for (int s = 0; s < NPB; ++s) {
-      mbar_init(BAR(C::B_DS + s), 4);
+      mbar_init(BAR(C::B_DS + s), 8);
       mbar_init(BAR(C::B_PE + s), 1);
     }
     mbar_init(BAR(C::B_KVD), 1);
@@ -341,12 +342,12 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp < 4 || (warp >= 8 && warp < 12)) {
     // ------------------------------------------------ P^T / dS^T rows, then dK / dV epilogue
-    const int par = warp < 4 ? 0 : 1;   // this warpgroup takes iterations of this parity
+    const int par = warp < 4 ? 0 : 1;   // this warpgroup's half of the 64 query columns
     const int j = threadIdx.x & 127;    // key row within the tile == TMEM lane
     const int jg = k0 + j;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int it = par; it < n; it += 2) {
+    for (int it = 0; it < n; ++it) {
       const int buf = it & 1, stage = it % NQS, pb = it % NPB;
       if (!W.wait_warp(BAR(C::B_SP + buf), (it >> 1) & 1, 60)) { ok = false; break; }
       if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 61)) { ok = false; break; }
@@ -363,8 +364,7 @@ __global__ void __launch_bounds__(512, 1)
       uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
       const uint32_t st_addr = tmem + lane_base + C::T_ST + 64 * buf;
       const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + 64 * buf;
-      bwd_row_half(st_addr, dpt_addr, 0, lse2, dlt, p.c, ilo, drow, j & 7);
-      bwd_row_half(st_addr, dpt_addr, 32, lse2, dlt, p.c, ilo, drow, j & 7);
+      bwd_row_half(st_addr, dpt_addr, 32 * par, lse2, dlt, p.c, ilo, drow, j & 7);
       if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 2);
       tmem_wait_st();
       fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
