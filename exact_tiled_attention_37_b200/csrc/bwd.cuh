@@ -26,7 +26,8 @@
 //    reductions into the scratch).
 //  * bwd_dq_finalize_kernel: dQ (bf16, caller's strides) from the scratch.
 //
-// TMEM (512 columns): ST/dQT[2] (64 each) | dPT[2] (64 each) | dV (128) | dK (128).
+// TMEM (512 columns): ST[2] (64 each: S^T, then P^T and dS^T packed) |
+// dPT[2] (64 each: dP^T, then dQ^T) | dV (128) | dK (128).
 // Head dimension 256 is split into two 128-column slices (two CTAs per key
 // tile, each recomputing S^T and dP^T over the full D): the TMEM-capacity
 // analogue of the D-blocking the Metal port README describes.
@@ -232,10 +233,11 @@ struct BwdCfg {
 
 // P^T and dS^T for 32 query columns [c0, c0 + 32) of this thread's key row:
 // loads S^T and dP^T from TMEM, applies exp2 / causal mask / softmax
-// Jacobian, writes P^T and dS^T as bf16 pairs back into the S^T and dP^T
-// columns it has read (TMEM columns c0/2 .. c0/2 + 15: the A operands of
-// dV += P^T dO and dK += dS^T Q) and dS^T also as a bf16 shared-memory row
-// (4 swizzled 16-byte chunks: the B operand of dQ^T = K^T dS^T).
+// Jacobian, and writes P^T and dS^T as bf16 pairs into the 32 S^T columns it
+// has just read (P^T at columns c0 .. c0 + 15, dS^T at c0 + 16 .. c0 + 31:
+// the A operands of dV += P^T dO and dK += dS^T Q), and dS^T also as a bf16
+// shared-memory row (4 swizzled 16-byte chunks: the B operand of
+// dQ^T = K^T dS^T).  The dP^T columns are left free for dQ^T.
 __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr, int c0,
                                              const float* lse2, const float* dlt, float c,
                                              int ilo, uint8_t* drow, int swz) {
@@ -267,8 +269,8 @@ __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr
     const int off = (chunk ^ swz) * 16;
     *reinterpret_cast<uint4*>(drow + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
   }
-  tmem_st16(st_addr + c0 / 2, pk);
-  tmem_st16(dpt_addr + c0 / 2, dk);
+  tmem_st16(st_addr + c0, pk);
+  tmem_st16(st_addr + c0 + 16, dk);
 }
 
 template <int DFULL, int NQS, int NPB>
@@ -415,7 +417,7 @@ __global__ void __launch_bounds__(512, 1)
       if (threadIdx.x == 128) ETA_TRACE_AT(tcta, 1, it, 0);
       tc_fence_after();
       float v[64];
-      tmem_load_row<64>(tmem + lane_base + C::T_ST + 64 * buf, v);
+      tmem_load_row<64>(tmem + lane_base + C::T_DPT + 64 * buf, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DQE + buf));
@@ -522,8 +524,8 @@ __global__ void __launch_bounds__(512, 1)
         issue_sdp(0);
         mma_commit(BAR(C::B_SP + 0));
       }
-      // S^T / dP^T of the next iteration go into the other TMEM buffer once
-      // the dQ warpgroup has drained the dQ^T that last used it.
+      // S^T / dP^T of the next iteration go into the other TMEM buffers once
+      // the dQ warpgroup has drained the dQ^T that last used that dP^T buffer.
       auto issue_next = [&](int it) -> bool {
         const int b1 = (it + 1) & 1, st1 = (it + 1) % NQS;
         if (it >= 1 && !W.wait(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1, 92)) return false;
@@ -550,22 +552,24 @@ __global__ void __launch_bounds__(512, 1)
         const SDesc dds = sdesc_base(sbase + C::S_DS + pb * C::PTILE, C::PTILE, 1024);
         const uint32_t tst = tmem + C::T_ST + 64 * buf, tdp = tmem + C::T_DPT + 64 * buf;
         const uint32_t acc0 = it > 0 ? 1u : 0u;
+        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed dP^T
+        // buffer, first, so that the dQ warpgroup drains it while dV and dK run
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss<false>(tdp, sdesc_at(dKt, ks * 2048), sdesc_at(dds, ks * 2048), id_q, ks > 0);
+        mma_commit(BAR(C::B_DQF + buf));
+        // P^T / dS^T of query rows [16 ks, 16 ks + 16) sit at S^T column
+        // 32 (ks / 2) + 8 (ks % 2) (+ 16 for dS^T)
         // dV += P^T dO_i with P^T read from TMEM (K = 64 query rows, 4 steps of 16)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts<false>(tmem + C::T_DV, tst + 8 * ks, sdesc_at(ddo, ks * 2048), id_kv,
-                        ks > 0 ? 1u : acc0);
+          mma_ts<false>(tmem + C::T_DV, tst + 32 * (ks >> 1) + 8 * (ks & 1), sdesc_at(ddo, ks * 2048),
+                        id_kv, ks > 0 ? 1u : acc0);
         // dK += dS^T Q_i with dS^T read from TMEM
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts<false>(tmem + C::T_DK, tdp + 8 * ks, sdesc_at(dq, ks * 2048), id_kv,
-                        ks > 0 ? 1u : acc0);
-        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed S^T
-        // buffer; issued after dV, whose P^T operand lives in those columns
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss<false>(tst, sdesc_at(dKt, ks * 2048), sdesc_at(dds, ks * 2048), id_q, ks > 0);
-        mma_commit(BAR(C::B_DQF + buf));
+          mma_ts<false>(tmem + C::T_DK, tst + 32 * (ks >> 1) + 16 + 8 * (ks & 1),
+                        sdesc_at(dq, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
         mma_commit(BAR(C::B_QE + stage));
         mma_commit(BAR(C::B_PE + pb));
         ETA_TRACE_AT(tcta, 2, it, 3);
