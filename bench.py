@@ -34,8 +34,8 @@ WORKLOAD_INDEX = 2  # MHA fwd+bwd B=2 H=16 N=4096 D=128 causal
 # DRAM traffic of one launch of the dominant kernel (bwd_dkdv_kernel<128,3,2>)
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the kernel source it was taken on; it is reported as null once the
-# source changes.  See profiles/ for the capture summary and command.
-DOMINANT_TRAFFIC = {"bytes": None, "src_sha": None}
+# source changes (profiles/ncu_full_fwd_bwd_mha_4096_causal.md has the capture).
+DOMINANT_TRAFFIC = {"bytes": 678316800, "src_sha": "7905a6d0eb2a1f45"}
 
 
 def parse_args():
