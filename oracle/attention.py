@@ -31,6 +31,13 @@ Readings where the pages are silent (each listed in the design doc): top-left
 causal alignment with equal query and key lengths; contiguous GQA groups
 (query head h reads key/value head ``h // G``); lse in natural log.
 
+Local (sliding-window) attention, the mask variant the pages mention
+(FlashAttention entity page and heapsort-ai.news attention tag: global plus
+sliding-window attention; twiscan MHA search: a 112-token local window):
+``window=(wl, wr)`` lets query i see key j only when ``i - wl <= j <= i + wr``;
+a negative bound is unbounded on that side.  ``causal`` is the same as
+``window=(-1, 0)`` and both may be combined.
+
 Precision: every input is upcast to float64 first; numpy/OpenBLAS does the
 matrix products (a library primitive used as one step, no fusion).
 """
@@ -68,12 +75,19 @@ def _check_shapes(q, k, v):
 
 
 def _scores(q_rows: np.ndarray, k_all: np.ndarray, row_ids: np.ndarray,
-            causal: bool, scale: float) -> np.ndarray:
+            causal: bool, scale: float, window=None) -> np.ndarray:
     """Scaled, masked scores for the given query rows against every key."""
     s = scale * (q_rows @ k_all.T)
+    cols = np.arange(k_all.shape[0])[None, :]
+    rows = row_ids[:, None]
     if causal:
-        cols = np.arange(k_all.shape[0])
-        s = np.where(cols[None, :] > row_ids[:, None], -np.inf, s)
+        s = np.where(cols > rows, -np.inf, s)
+    if window is not None:
+        wl, wr = window
+        if wl >= 0:
+            s = np.where(cols < rows - wl, -np.inf, s)
+        if wr >= 0:
+            s = np.where(cols > rows + wr, -np.inf, s)
     return s
 
 
@@ -87,7 +101,7 @@ def softmax_probs(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     return p, lse
 
 
-def attention_fwd(q, k, v, causal: bool, scale: float):
+def attention_fwd(q, k, v, causal: bool, scale: float, window=None):
     """O [B,Hq,N,D] and lse [B,Hq,N] in float64 for the whole problem."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     b_, hq, hkv, n, d = _check_shapes(q, k, v)
@@ -99,14 +113,14 @@ def attention_fwd(q, k, v, causal: bool, scale: float):
             hk = h // g
             for r0 in range(0, n, _ROW_BLOCK):
                 rows = np.arange(r0, min(n, r0 + _ROW_BLOCK))
-                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale)
+                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale, window)
                 p, l = softmax_probs(s)
                 o[b, h, rows] = p @ v[b, hk]
                 lse[b, h, rows] = l
     return o, lse
 
 
-def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
+def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows, window=None):
     """O and lse of selected query rows of one (batch, query head) only.
 
     Rows of attention are independent, so this is the same definition
@@ -119,12 +133,12 @@ def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows
     qr = _f64(q[b, h][rows])
     kk = _f64(k[b, hk])
     vv = _f64(v[b, hk])
-    s = _scores(qr, kk, rows, causal, scale)
+    s = _scores(qr, kk, rows, causal, scale, window)
     p, l = softmax_probs(s)
     return p @ vv, l
 
 
-def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None):
+def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None, window=None):
     """(dQ, dK, dV) in float64 from the plain softmax Jacobian.
 
     ``heads``: optional iterable of (b, h_kv) pairs to restrict the work to
@@ -147,7 +161,7 @@ def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None):
             dq_h = np.empty((n, d))
             for r0 in range(0, n, _ROW_BLOCK):
                 rows = np.arange(r0, min(n, r0 + _ROW_BLOCK))
-                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale)
+                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale, window)
                 p, _ = softmax_probs(s)
                 dO = do[b, h, rows]
                 dv_acc += p.T @ dO

@@ -262,7 +262,7 @@ def _run_pins():
 def test_mutants_are_caught(monkeypatch):
     assert _run_pins() == []
 
-    def off_by_one_mask(q_rows, k_all, row_ids, causal, scale):
+    def off_by_one_mask(q_rows, k_all, row_ids, causal, scale, window=None):
         s = scale * (q_rows @ k_all.T)
         if causal:
             cols = np.arange(k_all.shape[0])
@@ -270,8 +270,8 @@ def test_mutants_are_caught(monkeypatch):
             s[:, 0] = np.where(np.isinf(s[:, 0]), 0.0, s[:, 0])
         return s
 
-    def dropped_scale(q_rows, k_all, row_ids, causal, scale):
-        return oa.__dict__["_orig_scores"](q_rows, k_all, row_ids, causal, 1.0)
+    def dropped_scale(q_rows, k_all, row_ids, causal, scale, window=None):
+        return oa.__dict__["_orig_scores"](q_rows, k_all, row_ids, causal, 1.0, window)
 
     def lse_without_max(s):
         m = np.max(s, axis=1, keepdims=True)
@@ -315,3 +315,85 @@ def test_mutant_backward_without_row_term(monkeypatch):
     failed = _run_pins()
     assert "fd" in failed or "colsum" in failed
     monkeypatch.setattr(oracle, "attention_bwd", src_bwd)
+
+
+# ---------------------------------------------------------------- local windows
+
+
+def _brute_window(q, k, v, wl, wr, scale):
+    """Explicit loops over (i, j) for one head: the window definition written out."""
+    n = q.shape[0]
+    o = np.zeros_like(v)
+    lse = np.zeros(n)
+    for i in range(n):
+        js = [j for j in range(n) if (wl < 0 or j >= i - wl) and (wr < 0 or j <= i + wr)]
+        sc = np.array([scale * float(q[i] @ k[j]) for j in js])
+        w = np.exp(sc - sc.max())
+        o[i] = sum(wj * v[j] for wj, j in zip(w, js)) / w.sum()
+        lse[i] = sc.max() + math.log(w.sum())
+    return o, lse
+
+
+@pytest.mark.parametrize("wl,wr", [(0, 0), (2, 0), (3, 1), (-1, 2), (1, -1), (100, 100)])
+def test_window_matches_explicit_loops(wl, wr):
+    q, k, v = rnd((9, 4), 60), rnd((9, 4), 61), rnd((9, 4), 62)
+    o, lse = oracle.attention_fwd(q[None, None], k[None, None], v[None, None], False, 0.7,
+                                  window=(wl, wr))
+    o_b, lse_b = _brute_window(q, k, v, wl, wr, 0.7)
+    np.testing.assert_allclose(o[0, 0], o_b, atol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], lse_b, atol=1e-13)
+
+
+def test_window_special_cases():
+    q, k, v = rnd((1, 2, 12, 5), 63), rnd((1, 2, 12, 5), 64), rnd((1, 2, 12, 5), 65)
+    full, lf = fwd(q, k, v, False, 0.4)
+    caus, lc = fwd(q, k, v, True, 0.4)
+    for win, (o_ref, l_ref) in (((-1, -1), (full, lf)), ((12, 12), (full, lf)),
+                                ((-1, 0), (caus, lc)), ((11, 0), (caus, lc))):
+        o, l = oracle.attention_fwd(q, k, v, False, 0.4, window=win)
+        np.testing.assert_allclose(o, o_ref, atol=1e-13)
+        np.testing.assert_allclose(l, l_ref, atol=1e-13)
+    # a zero-width window: every query sees only its own key
+    o, l = oracle.attention_fwd(q, k, v, False, 0.4, window=(0, 0))
+    np.testing.assert_allclose(o, v, atol=1e-14)
+    np.testing.assert_allclose(l, 0.4 * np.sum(q * k, axis=-1), atol=1e-13)
+
+
+def test_zero_query_window_mean():
+    # Q = 0: O_i is the mean of V over the window [max(0, i - w), i]; lse = log(count)
+    n, d, w = 10, 3, 3
+    v = rnd((1, 1, n, d), 66)
+    o, l = oracle.attention_fwd(np.zeros((1, 1, n, d)), rnd((1, 1, n, d), 67), v, True, 0.5,
+                                window=(w, 0))
+    for i in range(n):
+        lo = max(0, i - w)
+        np.testing.assert_allclose(o[0, 0, i], v[0, 0, lo:i + 1].mean(axis=0), atol=1e-13)
+        assert abs(l[0, 0, i] - math.log(i + 1 - lo)) < 1e-13
+
+
+@pytest.mark.parametrize("window", [(2, 0), (1, 2)])
+def test_window_backward_finite_differences(window):
+    n, d, scale, h = 6, 3, 0.8, 1e-6
+    q, k, v, do = (rnd((1, 2, n, d), s) for s in (70, 71, 72, 73))
+    k, v = k[:, :1], v[:, :1]
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, False, scale, window=window)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.attention_fwd(qq, kk, vv, False, scale, window=window)
+        return float(np.sum(o * do))
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = {"q": q, "k": k, "v": v}
+            args_p[name], args_m[name] = xp, xm
+            fd[idx] = (loss(args_p["q"], args_p["k"], args_p["v"])
+                       - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
+        err = np.max(np.abs(fd - g)) / max(np.max(np.abs(g)), 1e-30)
+        assert err < 1e-6, (name, err)
