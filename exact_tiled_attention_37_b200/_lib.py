@@ -56,6 +56,11 @@ def lib(path: str | None = None) -> ctypes.CDLL:
     L.attn_status_string.argtypes = [i]
     L.attn_fwd.restype = i
     L.attn_fwd.argtypes = [T, T, T, T, vp, i, i, i, i, i, i, i, f, vp]
+    L.attn_fwd_window.restype = i
+    L.attn_fwd_window.argtypes = [T, T, T, T, vp, i, i, i, i, i, i, i, i, f, vp]
+    L.attn_bwd_window.restype = i
+    L.attn_bwd_window.argtypes = [T, T, T, T, vp, T, T, T, T, i, i, i, i, i, i, i, i, f, vp,
+                                  ctypes.c_size_t, vp]
     L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
     L.attn_bwd.restype = i

@@ -44,11 +44,20 @@ def _check(code: int, what: str):
         raise AttnError(code, what)
 
 
+def _window(causal: bool, window) -> tuple[int, int]:
+    """(window_left, window_right) of the C ABI: -1 = unbounded; causal caps the right side at 0."""
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    if causal:
+        wr = 0
+    return wl, wr
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              scale: float | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None):
+             lse: torch.Tensor | None = None, window=None):
     """O, lse = attention(q, k, v): q [B,Hq,N,D], k/v [B,Hkv,N,D] on one CUDA device.
 
+    window=(wl, wr): query i sees keys i - wl .. i + wr (-1 = unbounded side).
     Returns O (dtype of q) and lse [B,Hq,N] fp32 (natural log).
     """
     B, Hq, N, D = q.shape
@@ -66,9 +75,10 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (B, Hq, N):
         raise ValueError("lse must be a contiguous fp32 [B, Hq, N] tensor")
     L = _lib.lib()
-    code = L.attn_fwd(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(out, "out"),
-                      ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, N, D, _dtype_code(q),
-                      1 if causal else 0, float(scale), _stream(q.device))
+    wl, wr = _window(causal, window)
+    code = L.attn_fwd_window(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(out, "out"),
+                             ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, N, D, _dtype_code(q),
+                             wl, wr, float(scale), _stream(q.device))
     _check(code, "attn_fwd")
     return out, lse
 
@@ -78,7 +88,7 @@ def bwd_workspace_bytes(B: int, Hq: int, N: int, D: int) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
-             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None):
+             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, window=None):
     """dQ, dK, dV of attention from the forward's O and lse and the gradient dO."""
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
@@ -98,12 +108,14 @@ def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
         raise ValueError(f"workspace too small: {need} bytes needed")
     if not lse.is_contiguous() or lse.dtype != torch.float32:
         raise ValueError("lse must be contiguous fp32")
-    code = L.attn_bwd(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(o, "o"),
-                      ctypes.c_void_p(lse.data_ptr()), _desc(do, "do"), _desc(dq, "dq"),
-                      _desc(dk, "dk"), _desc(dv, "dv"), B, Hq, Hkv, N, D, _dtype_code(q),
-                      1 if causal else 0, float(scale), ctypes.c_void_p(workspace.data_ptr()),
-                      ctypes.c_size_t(workspace.numel() * workspace.element_size()),
-                      _stream(q.device))
+    wl, wr = _window(causal, window)
+    code = L.attn_bwd_window(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(o, "o"),
+                             ctypes.c_void_p(lse.data_ptr()), _desc(do, "do"), _desc(dq, "dq"),
+                             _desc(dk, "dk"), _desc(dv, "dv"), B, Hq, Hkv, N, D,
+                             _dtype_code(q), wl, wr, float(scale),
+                             ctypes.c_void_p(workspace.data_ptr()),
+                             ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                             _stream(q.device))
     _check(code, "attn_bwd")
     return dq, dk, dv
 

@@ -275,7 +275,16 @@ attn_status_t attn_device_status(void* stream, int* where) {
 attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
                        float* lse, int B, int Hq, int Hkv, int N, int D, attn_dtype_t dtype,
                        int causal, float scale, void* stream) {
+  return attn_fwd_window(q, k, v, o, lse, B, Hq, Hkv, N, D, dtype, -1, causal ? 0 : -1, scale,
+                         stream);
+}
+
+attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                              float* lse, int B, int Hq, int Hkv, int N, int D,
+                              attn_dtype_t dtype, int window_left, int window_right, float scale,
+                              void* stream) {
   attn_status_t s;
+  if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
   if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
   if (!lse) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
@@ -298,7 +307,8 @@ attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
   p.Hq = Hq;
   p.N = N;
   p.group = Hq / Hkv;
-  p.causal = causal ? 1 : 0;
+  p.wl = window_left >= N ? -1 : window_left;
+  p.wr = window_right >= N ? -1 : window_right;
   p.scale = scale;
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
@@ -330,7 +340,18 @@ attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
                        attn_tensor_t dv, int B, int Hq, int Hkv, int N, int D,
                        attn_dtype_t dtype, int causal, float scale, void* workspace,
                        size_t workspace_bytes, void* stream) {
+  return attn_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, dtype, -1,
+                         causal ? 0 : -1, scale, workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                              const float* lse, attn_tensor_t dout, attn_tensor_t dq,
+                              attn_tensor_t dk, attn_tensor_t dv, int B, int Hq, int Hkv, int N,
+                              int D, attn_dtype_t dtype, int window_left, int window_right,
+                              float scale, void* workspace, size_t workspace_bytes,
+                              void* stream) {
   attn_status_t s;
+  if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
   if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
   if (!lse || !workspace) return !lse ? ATTN_ERR_INVALID_ARG : ATTN_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
@@ -366,7 +387,8 @@ attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_t
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.D = D;
   p.Npad = static_cast<int>(eta::bwd_npad(N));
   p.group = Hq / Hkv;
-  p.causal = causal ? 1 : 0;
+  p.wl = window_left >= N ? -1 : window_left;
+  p.wr = window_right >= N ? -1 : window_right;
   p.scale = scale;
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;

@@ -89,7 +89,8 @@ struct BwdParams {
   long long dqsb, dqsh, dqsn;
   long long dksb, dksh, dksn;
   long long dvsb, dvsh, dvsn;
-  int B, Hq, Hkv, N, D, Npad, group, causal;
+  int B, Hq, Hkv, N, D, Npad, group;
+  int wl, wr;           // local window (query i sees keys [i - wl, i + wr]); -1 = unbounded
   float scale, c;       // c = scale * log2(e)
   int* status;
   unsigned long long wait_limit_ns;
@@ -240,7 +241,7 @@ struct BwdCfg {
 // dQ^T = K^T dS^T).  The dP^T columns are left free for dQ^T.
 __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr, int c0,
                                              const float* lse2, const float* dlt, float c,
-                                             int ilo, uint8_t* drow, int swz) {
+                                             int ilo, int ihi, uint8_t* drow, int swz) {
   uint32_t rs[32], rd[32];
   tmem_ld32(st_addr + c0, rs);
   tmem_ld32(dpt_addr + c0, rd);
@@ -258,8 +259,8 @@ __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr
       const float2 x = ffma2(make_float2(u2f(rs[i]), u2f(rs[i + 1])), c2,
                              make_float2(-l2.x, -l2.y));
       float2 pv = make_float2(ex2(x.x), ex2(x.y));
-      if (c0 + i < ilo) pv.x = 0.f;
-      if (c0 + i + 1 < ilo) pv.y = 0.f;
+      if (c0 + i < ilo || c0 + i > ihi) pv.x = 0.f;
+      if (c0 + i + 1 < ilo || c0 + i + 1 > ihi) pv.y = 0.f;
       const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
       pk[4 * u + e] = pack_bf16x2(pv.x, pv.y);
       dw[e] = pack_bf16x2(pv.x * g.x, pv.y * g.y);
@@ -296,9 +297,12 @@ __global__ void __launch_bounds__(512, 1)
   const int half = blockIdx.x % C::DSPLIT;
   const int b = blockIdx.y;
   const int k0 = kt * C::BC;
-  const int nqt = (p.N + C::BR - 1) / C::BR;
-  const int i_first = p.causal ? k0 / C::BR : 0;
-  const int per_head = nqt - i_first;
+  // queries that see any key of [k0, k0 + BC): key j is visible to query i iff
+  // j - wr <= i <= j + wl
+  const int q_lo = p.wr < 0 ? 0 : max(0, k0 - p.wr);
+  const int q_hi = p.wl < 0 ? p.N : min(p.N, min(p.N, k0 + C::BC) + p.wl);
+  const int i_first = q_lo / C::BR;
+  const int per_head = (q_hi + C::BR - 1) / C::BR - i_first;
   const int n = per_head * p.group;  // iterations: query heads of the group x query tiles
 
   if (threadIdx.x == 0) {
@@ -361,12 +365,13 @@ __global__ void __launch_bounds__(512, 1)
       const float* lse2 = reinterpret_cast<const float*>(smem + C::S_STAT + stage * 512);
       const float* dlt = lse2 + 64;
       const int ig0 = qtile_of(it) * C::BR;
-      // causal: query i sees key j iff jg <= ig0 + i  ->  valid for i >= jg - ig0
-      const int ilo = p.causal ? jg - ig0 : -1;
+      // window: query ig0 + i sees key jg iff jg - wr <= ig0 + i <= jg + wl
+      const int ilo = p.wr < 0 ? -(1 << 30) : jg - p.wr - ig0;
+      const int ihi = p.wl < 0 ? (1 << 30) : jg + p.wl - ig0;
       uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
       const uint32_t st_addr = tmem + lane_base + C::T_ST + 64 * buf;
       const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + 64 * buf;
-      bwd_row_half(st_addr, dpt_addr, 32 * par, lse2, dlt, p.c, ilo, drow, j & 7);
+      bwd_row_half(st_addr, dpt_addr, 32 * par, lse2, dlt, p.c, ilo, ihi, drow, j & 7);
       if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 2);
       tmem_wait_st();
       fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads

@@ -61,7 +61,7 @@ struct FwdParams {
   float* lse;        // [B, Hq, N] contiguous
   long long osb, osh, osn;
   int Hq, N, group;  // group = Hq / Hkv
-  int causal;
+  int wl, wr;        // local window: query i sees keys [i - wl, i + wr]; -1 = unbounded
   float scale;       // softmax scale (natural units)
   float c;           // scale * log2(e)
   int* status;       // device status word (4 ints)
@@ -215,20 +215,36 @@ __device__ __forceinline__ void store_row(uint32_t o_taddr, const FwdParams& p, 
     p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = m * p.scale + logf(l);
 }
 
-// Column limit of one row in one key tile: columns >= lim are masked.
-__device__ __forceinline__ int col_limit(int kbase, int qrow, int N, int causal, int BC) {
-  int lim = N - kbase;
-  if (causal) lim = min(lim, qrow - kbase + 1);
-  return min(lim, BC);
+// Keys [lo, hi) that query rows [qs, qe) may see under the window (wl, wr)
+// (-1 = unbounded; the causal mask is (-1, 0)), clipped to [0, N).
+__device__ __forceinline__ int2 window_keys(int qs, int qe, int N, int wl, int wr) {
+  const int lo = wl < 0 ? 0 : max(0, qs - wl);
+  const int hi = wr < 0 ? N : min(N, qe + wr);
+  return make_int2(lo, hi);
+}
+
+// Visible columns [lo, hi) of one query row in the key tile starting at kbase.
+__device__ __forceinline__ int2 col_window(int kbase, int qrow, int N, int wl, int wr) {
+  const int lo = wl < 0 ? 0 : qrow - wl - kbase;
+  const int hi = min(N, wr < 0 ? N : qrow + wr + 1) - kbase;
+  return make_int2(lo, hi);
 }
 
 template <int BC>
-__device__ __forceinline__ void apply_mask(float (&s)[BC], int lim) {
-  if (lim < BC) {
+__device__ __forceinline__ void apply_mask(float (&s)[BC], int2 cw) {
+  if (cw.x > 0 || cw.y < BC) {
 #pragma unroll
     for (int i = 0; i < BC; ++i)
-      if (i >= lim) s[i] = -INFINITY;
+      if (i < cw.x || i >= cw.y) s[i] = -INFINITY;
   }
+}
+
+// Key-tile range [j_lo, j_hi) of a 128-row query tile starting at qs (empty
+// when the tile lies past N).
+__device__ __forceinline__ int2 key_tiles(int qs, int N, int wl, int wr, int BN) {
+  if (qs >= N) return make_int2(0, 0);
+  const int2 kr = window_keys(qs, min(N, qs + 128), N, wl, wr);
+  return make_int2(kr.x / BN, (kr.y + BN - 1) / BN);
 }
 
 // =====================================================================
@@ -293,14 +309,18 @@ __global__ void __launch_bounds__(384, 1)
   const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / p.group;
   const int q0 = qb * 256;
-  int ntile[2];
+  // key tiles [jlo[t], jhi[t]) of each query tile; tile 0's range never starts
+  // or ends after tile 1's, so tile 1 (when it has work) is the last reader of
+  // every K/V tile it uses
+  int jlo[2], jhi[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int qs = q0 + 128 * t;
-    const int kv_end = p.causal ? min(p.N, qs + 128) : p.N;
-    ntile[t] = qs < p.N ? (kv_end + 127) / 128 : 0;
+    const int2 r = key_tiles(q0 + 128 * t, p.N, p.wl, p.wr, 128);
+    jlo[t] = r.x;
+    jhi[t] = r.y;
   }
-  const int nK = max(ntile[0], ntile[1]);
+  const bool has1 = jhi[1] > jlo[1];
+  const int jmin = jlo[0], jmax = has1 ? jhi[1] : jhi[0];
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::BAR_Q), 1);
@@ -344,8 +364,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntile[t]; ++j) {
-      if (!W.wait_warp(BAR(C::BAR_S + t), j & 1, 10 + t)) { ok = false; break; }
+    for (int j = jlo[t]; j < jhi[t]; ++j) {
+      if (!W.wait_warp(BAR(C::BAR_S + t), (j - jlo[t]) & 1, 10 + t)) { ok = false; break; }
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 0);
       tc_fence_after();
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 1);
@@ -355,18 +375,18 @@ __global__ void __launch_bounds__(384, 1)
       float alpha;
       float s[128];
       tmem_load_row<128>(s_addr, s);
-      apply_mask<128>(s, col_limit(128 * j, qrow, p.N, p.causal, 128));
+      apply_mask<128>(s, col_window(128 * j, qrow, p.N, p.wl, p.wr));
       const bool rescaled = online_softmax_step<128, kSoftExp8>(s, p.c, m, l, alpha);
       tmem_store_p<128, C::TF32>(s_addr, s);
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 2);
-      if (rescaled && j > 0) tmem_scale_row<D>(o_addr, alpha);
+      if (rescaled && j > jlo[t]) tmem_scale_row<D>(o_addr, alpha);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::BAR_P + t));
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 3);
     }
-    if (ok && ntile[t] > 0 && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
+    if (ok && jhi[t] > jlo[t] && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
       tc_fence_after();
       store_row<T, D>(o_addr, p, b, h, qrow, m, l);
     }
@@ -383,12 +403,12 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sbase + C::SMEM_Q + t * C::TILE + c * C::CHUNK, &tm_q, BAR(C::BAR_Q), c * EPC,
                       q0 + 128 * t, h, b);
       int it = 0;
-      for (int j = 0; j < nK && !W.aborted(); ++j) {
+      for (int j = jmin; j < jmax && !W.aborted(); ++j) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = it % NS;
           const uint32_t ph = static_cast<uint32_t>(it / NS) & 1u;
           if (!W.wait(BAR(C::BAR_KVE + slot), ph ^ 1u, 30)) break;
-          if ((p.debug_flags & 1) && kv == 1 && j == 0) continue;  // fault injection: drop V_0
+          if ((p.debug_flags & 1) && kv == 1 && j == jmin) continue;  // fault injection: drop V
           mbar_expect_tx(BAR(C::BAR_KVF + slot), C::TILE);
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_4d(sbase + C::SMEM_KV + slot * C::TILE + c * C::CHUNK, kv ? &tm_v : &tm_k,
@@ -410,10 +430,12 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t fmt = C::TF32 ? 2u : 1u;
       constexpr uint32_t idesc_s = idesc_make(128, 128, fmt, false, false);
       constexpr uint32_t idesc_o = idesc_make(128, D, fmt, false, true);
-      auto kslot = [&](int j) { return (2 * j) % NS; };
-      auto kph = [&](int j) { return static_cast<uint32_t>((2 * j) / NS) & 1u; };
-      auto vslot = [&](int j) { return (2 * j + 1) % NS; };
-      auto vph = [&](int j) { return static_cast<uint32_t>((2 * j + 1) / NS) & 1u; };
+      // ring position of K_j / V_j (loads start at key tile jmin)
+      auto kslot = [&](int j) { return (2 * (j - jmin)) % NS; };
+      auto kph = [&](int j) { return static_cast<uint32_t>((2 * (j - jmin)) / NS) & 1u; };
+      auto vslot = [&](int j) { return (2 * (j - jmin) + 1) % NS; };
+      auto vph = [&](int j) { return static_cast<uint32_t>((2 * (j - jmin) + 1) / NS) & 1u; };
+      auto uses = [&](int t, int j) { return j >= jlo[t] && j < jhi[t]; };
       auto issue_s = [&](int t, int slot) {
         const SDesc qa = sdesc_base(sbase + C::SMEM_Q + t * C::TILE, 16, 1024);
         const SDesc kb = sdesc_base(sbase + C::SMEM_KV + slot * C::TILE, 16, 1024);
@@ -433,48 +455,43 @@ __global__ void __launch_bounds__(384, 1)
           mma_ts<C::TF32>(d, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128), idesc_o,
                           ks > 0 ? 1u : acc0);
       };
-      const int n0 = ntile[0], n1 = ntile[1];
-      bool ok = W.wait(BAR(C::BAR_Q), 0, 40) && W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
-      if (ok) {
+      // S_t(j) = Q_t K_j^T; K_j's last reader (tile 1 when it uses K_j) frees its slot
+      auto start_s = [&](int t, int j) -> bool {
+        if (!W.wait(BAR(C::BAR_KVF + kslot(j)), kph(j), 44 + t)) return false;
         tc_fence_after();
-        if (n0 > 0) { issue_s(0, kslot(0)); mma_commit(BAR(C::BAR_S + 0)); }
-        if (n1 > 0) { issue_s(1, kslot(0)); mma_commit(BAR(C::BAR_S + 1)); }
-        mma_commit(BAR(C::BAR_KVE + kslot(0)));
-      }
-      for (int j = 0; ok && j < nK; ++j) {
-        const bool use0 = j < n0, use1 = j < n1;
-        const bool nxt0 = j + 1 < n0, nxt1 = j + 1 < n1;
+        issue_s(t, kslot(j));
+        mma_commit(BAR(C::BAR_S + t));
+        if (t == 1 || !uses(1, j)) mma_commit(BAR(C::BAR_KVE + kslot(j)));
+        return true;
+      };
+      bool ok = W.wait(BAR(C::BAR_Q), 0, 40);
+      for (int j = jmin; ok && j < jmax; ++j) {
+        for (int t = 0; ok && t < 2; ++t)
+          if (j == jlo[t] && uses(t, j)) ok = start_s(t, j);
+        if (!ok) break;
         if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 42)) { ok = false; break; }
-        if (use0) {
-          if (!W.wait(BAR(C::BAR_P + 0), j & 1, 43)) { ok = false; break; }
-          ETA_FTRACE_AT(tcta, 2, j, 0);
-          tc_fence_after();
-          issue_pv(0, vslot(j), j > 0);
-          if (!use1) mma_commit(BAR(C::BAR_KVE + vslot(j)));
-          if (nxt0) {
-            if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 44)) { ok = false; break; }
-            issue_s(0, kslot(j + 1));
-            mma_commit(BAR(C::BAR_S + 0));
-            ETA_FTRACE_AT(tcta, 2, j, 1);
-            if (!nxt1) mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
-          } else {
-            mma_commit(BAR(C::BAR_O + 0));
-          }
+        if (!uses(0, j) && !uses(1, j)) {
+          // no query tile reads this key tile (cannot happen with windows >= 0:
+          // the two tiles' ranges overlap); hand both slots back
+          if (!W.wait(BAR(C::BAR_KVF + kslot(j)), kph(j), 41)) { ok = false; break; }
+          mbar_arrive(BAR(C::BAR_KVE + kslot(j)));
+          mbar_arrive(BAR(C::BAR_KVE + vslot(j)));
+          continue;
         }
-        if (use1) {
-          if (!W.wait(BAR(C::BAR_P + 1), j & 1, 45)) { ok = false; break; }
-          ETA_FTRACE_AT(tcta, 2, j, 2);
+        for (int t = 0; ok && t < 2; ++t) {
+          if (!uses(t, j)) continue;
+          if (!W.wait(BAR(C::BAR_P + t), (j - jlo[t]) & 1, 43 + 2 * t)) { ok = false; break; }
+          if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 0);
+          if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 2);
           tc_fence_after();
-          issue_pv(1, vslot(j), j > 0);
-          mma_commit(BAR(C::BAR_KVE + vslot(j)));
-          if (nxt1) {
-            if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 46)) { ok = false; break; }
-            issue_s(1, kslot(j + 1));
-            mma_commit(BAR(C::BAR_S + 1));
-            ETA_FTRACE_AT(tcta, 2, j, 3);
-            mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
+          issue_pv(t, vslot(j), j > jlo[t]);
+          if (t == 1 || !uses(1, j)) mma_commit(BAR(C::BAR_KVE + vslot(j)));
+          if (j + 1 < jhi[t]) {
+            ok = start_s(t, j + 1);
+            if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 1);
+            if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 3);
           } else {
-            mma_commit(BAR(C::BAR_O + 1));
+            mma_commit(BAR(C::BAR_O + t));
           }
         }
       }
@@ -552,8 +569,11 @@ __global__ void __launch_bounds__(256, 1)
   const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / p.group;
   const int q0 = qb * 128;
-  const int kv_end = p.causal ? min(p.N, q0 + 128) : p.N;
-  const int n = (kv_end + BC - 1) / BC;
+  // key tiles j0 .. j0 + n - 1 are visible to this query tile; loop counters
+  // below run over 0 .. n - 1
+  const int2 ktr = key_tiles(q0, p.N, p.wl, p.wr, BC);
+  const int j0 = ktr.x;
+  const int n = ktr.y - ktr.x;
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::BAR_Q), 1);
@@ -595,7 +615,7 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       float s[BC];
       tmem_load_row<BC>(s_addr, s);
-      apply_mask<BC>(s, col_limit(BC * j, qrow, p.N, p.causal, BC));
+      apply_mask<BC>(s, col_window(BC * (j0 + j), qrow, p.N, p.wl, p.wr));
       float alpha;
       const bool rescaled = online_softmax_step<BC, 0>(s, p.c, m, l, alpha);
       tmem_store_p<BC, false>(s_addr, s);
@@ -632,7 +652,7 @@ __global__ void __launch_bounds__(256, 1)
           mbar_expect_tx(BAR(C::BAR_KVF + slot), C::KTILE);
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_4d(sbase + C::SMEM_KV + slot * C::KTILE + c * C::KCHUNK, kv ? &tm_v : &tm_k,
-                        BAR(C::BAR_KVF + slot), c * 64, BC * j, hk, b);
+                        BAR(C::BAR_KVF + slot), c * 64, BC * (j0 + j), hk, b);
         }
       }
       const int issued = it;

@@ -53,8 +53,8 @@ __global__ void __launch_bounds__(128) fwd_fp32_kernel(const float* __restrict__
     o1[r] = 0.f;
   }
   const int row0 = warp * 8;
-  const int kv_end = p.causal ? min(p.N, q0 + kF32Rows) : p.N;
-  for (int kt = 0; kt < kv_end; kt += kF32Keys) {
+  const int2 kr = window_keys(q0, min(p.N, q0 + kF32Rows), p.N, p.wl, p.wr);
+  for (int kt = (kr.x / kF32Keys) * kF32Keys; kt < kr.y; kt += kF32Keys) {
     __syncthreads();
     for (int e = threadIdx.x; e < kF32Keys * kF32D; e += blockDim.x) {
       const int r = e / kF32D, d = e % kF32D;
@@ -81,8 +81,9 @@ __global__ void __launch_bounds__(128) fwd_fp32_kernel(const float* __restrict__
     for (int r = 0; r < 8; ++r) {
       const int qrow = q0 + row0 + r;
       float a = s0[r] * p.scale, c = s1[r] * p.scale;
-      if (key0 >= p.N || (p.causal && key0 > qrow)) a = -INFINITY;
-      if (key1 >= p.N || (p.causal && key1 > qrow)) c = -INFINITY;
+      const int2 cw = col_window(0, qrow, p.N, p.wl, p.wr);  // visible keys [cw.x, cw.y)
+      if (key0 < cw.x || key0 >= cw.y) a = -INFINITY;
+      if (key1 < cw.x || key1 >= cw.y) c = -INFINITY;
       float mx = fmaxf(a, c);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));

@@ -96,6 +96,21 @@ ATTN_API attn_status_t attn_fwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t 
                        int causal, float scale, void* stream);
 
 /*
+ * Forward with a local (sliding) window: query i sees key j only when
+ * i - window_left <= j <= i + window_right; -1 leaves that side unbounded
+ * (attn_fwd's causal mask is window (-1, 0), no mask is (-1, -1)).  Windows
+ * wider than N behave as unbounded.  The pages name this mask variant: global
+ * plus sliding-window attention (heapsort-ai.news attention tag) and a
+ * 112-token local window (twiscan MHA search), i.e. window (111, 0).  Other
+ * arguments as attn_fwd; window_left or window_right < -1 is
+ * ATTN_ERR_INVALID_ARG.
+ */
+ATTN_API attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                       attn_tensor_t o, float* lse, int B, int Hq, int Hkv, int N,
+                                       int D, attn_dtype_t dtype, int window_left,
+                                       int window_right, float scale, void* stream);
+
+/*
  * Bytes of device workspace attn_bwd needs for these sizes: an fp32 dQ
  * accumulator [B,Hq,N,D] (the scratch the backward's atomic partial sums go
  * to) plus two fp32 row statistics [B,Hq,N'] (rowsum(dO*O) and lse*log2(e),
@@ -115,6 +130,18 @@ ATTN_API attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t 
                        attn_tensor_t dv, int B, int Hq, int Hkv, int N, int D,
                        attn_dtype_t dtype, int causal, float scale, void* workspace,
                        size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of attn_fwd_window (same window convention; other arguments as
+ * attn_bwd).
+ */
+ATTN_API attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                       attn_tensor_t o, const float* lse, attn_tensor_t dout,
+                                       attn_tensor_t dq, attn_tensor_t dk, attn_tensor_t dv,
+                                       int B, int Hq, int Hkv, int N, int D,
+                                       attn_dtype_t dtype, int window_left, int window_right,
+                                       float scale, void* workspace, size_t workspace_bytes,
+                                       void* stream);
 
 /*
  * attn_bwd for callers that cannot allocate device memory.

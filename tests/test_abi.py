@@ -80,6 +80,17 @@ def test_fwd_validation_codes(L):
     assert _fwd(L, lse=0x20004) == 3
 
 
+def test_window_validation_codes(L):
+    B, Hq, N, D = 1, 2, 256, 128
+    t = _t(0x10000, Hq * N * D, N * D, D)
+    lse = ctypes.c_void_p(0x20000)
+    assert L.attn_fwd_window(t, t, t, t, lse, B, Hq, Hq, N, D, 0, -2, 0, 0.1, None) == 1
+    assert L.attn_fwd_window(t, t, t, t, lse, B, Hq, Hq, N, D, 0, 3, -5, 0.1, None) == 1
+    ws = L.attn_bwd_workspace_bytes(B, Hq, N, D)
+    assert L.attn_bwd_window(t, t, t, t, lse, t, t, t, t, B, Hq, Hq, N, D, 0, -3, 0, 0.1,
+                             ctypes.c_void_p(0x40000), ws, None) == 1
+
+
 def test_bwd_validation_codes(L):
     B, Hq, Hkv, N, D = 1, 2, 1, 256, 128
     q = _t(0x10000, Hq * N * D, N * D, D)
