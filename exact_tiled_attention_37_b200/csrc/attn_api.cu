@@ -14,6 +14,7 @@
 
 #include "attn.h"
 #include "bwd.cuh"
+#include "bwd_split.cuh"
 #include "fwd.cuh"
 #include "fwd_fp32.cuh"
 
@@ -204,6 +205,39 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
   return last_launch();
 }
 
+// Head dimensions 64 and 128: preprocess, then the column-parallel dK/dV
+// kernel and the row-parallel dQ kernel (no scratch, no atomics).
+template <int D, int NQS, int NS>
+attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
+                               const attn_tensor_t& v, const attn_tensor_t& dout,
+                               eta::BwdParams& p, cudaStream_t st) {
+  using CKV = eta::BwdKVCfg<D, NQS>;
+  using CQ = eta::BwdQCfg<D, NS>;
+  CUtensorMap tq, tk, tv, tdo;
+  attn_status_t s;
+  if ((s = make_map(&tq, q, p.B, p.Hq, p.N, D, 2, 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tdo, dout, p.B, p.Hq, p.N, D, 2, 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tk, k, p.B, p.Hkv, p.N, D, 2, 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tv, v, p.B, p.Hkv, p.N, D, 2, 128)) != ATTN_OK) return s;
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
+  eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
+  if ((s = last_launch()) != ATTN_OK) return s;
+  auto kkv = eta::bwd_kv_kernel<D, NQS>;
+  auto kq = eta::bwd_q_kernel<D, NS>;
+  if ((s = set_smem(kkv, CKV::SMEM_BYTES)) != ATTN_OK) return s;
+  if ((s = set_smem(kq, CQ::SMEM_BYTES)) != ATTN_OK) return s;
+  const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128);
+  cudaEvent_t ev0 = static_cast<cudaEvent_t>(g_bwd_ev_start.exchange(nullptr));
+  cudaEvent_t ev1 = static_cast<cudaEvent_t>(g_bwd_ev_stop.exchange(nullptr));
+  const bool timed = ev0 && ev1;
+  if (timed && cudaEventRecord(ev0, st) != cudaSuccess) return ATTN_ERR_CUDA;
+  kkv<<<dim3(p.Hkv, p.B, tiles), CKV::THREADS, CKV::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+  if ((s = last_launch()) != ATTN_OK) return s;
+  if (timed && cudaEventRecord(ev1, st) != cudaSuccess) return ATTN_ERR_CUDA;
+  kq<<<dim3(p.Hq, p.B, tiles), CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+  return last_launch();
+}
+
 attn_status_t check_sizes(int B, int Hq, int Hkv, int N) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
@@ -356,7 +390,7 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if (!lse || !workspace) return !lse ? ATTN_ERR_INVALID_ARG : ATTN_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
-  if (!(D == 128 || D == 256)) return ATTN_ERR_UNSUPPORTED;
+  if (!(D == 64 || D == 128 || D == 256)) return ATTN_ERR_UNSUPPORTED;
   const int es = 2;
   const attn_tensor_t* qs[] = {&q, &o, &dout, &dq};
   for (auto* t : qs)
@@ -375,7 +409,7 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.dk = dk.ptr;
   p.dv = dv.ptr;
   char* ws = static_cast<char*>(workspace);
-  p.dqacc = reinterpret_cast<float*>(ws);
+  p.dqacc = eta::bwd_dqacc_bytes(B, Hq, N, D) ? reinterpret_cast<float*>(ws) : nullptr;
   p.delta = reinterpret_cast<float*>(ws + eta::bwd_dqacc_bytes(B, Hq, N, D));
   p.lse2 = reinterpret_cast<float*>(ws + eta::bwd_dqacc_bytes(B, Hq, N, D) +
                                     eta::bwd_stat_bytes(B, Hq, N));
@@ -394,7 +428,8 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
   p.wait_limit_ns = g_wait_limit_ns.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128) return launch_bwd<128, 3, 2>(q, k, v, dout, p, st);
+  if (D == 64) return launch_bwd_split<64, 4, 8>(q, k, v, dout, p, st);
+  if (D == 128) return launch_bwd_split<128, 2, 4>(q, k, v, dout, p, st);
   return launch_bwd<256, 1, 1>(q, k, v, dout, p, st);
 }
 

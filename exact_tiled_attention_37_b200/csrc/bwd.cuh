@@ -62,7 +62,10 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline size_t bwd_npad(int N) { return round_up(static_cast<size_t>(N), kBwdRowPad); }
 
+// fp32 dQ scratch: only the fused kernel (head dimension 256) accumulates dQ
+// there; for D <= 128 the row-parallel dQ kernel writes dQ directly.
 inline size_t bwd_dqacc_bytes(int B, int Hq, int N, int D) {
+  if (D <= 128) return 0;
   return round_up(static_cast<size_t>(B) * Hq * N * D * 4, 256);
 }
 
@@ -113,12 +116,17 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) 
     }
     return;
   }
-  constexpr int PER = D / 32;  // elements per lane (4 or 8)
+  constexpr int PER = D / 32;  // elements per lane (2, 4 or 8)
   const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(p.o) + b * p.osb + h * p.osh + i * p.osn;
   const __nv_bfloat16* drow =
       static_cast<const __nv_bfloat16*>(p.dout) + b * p.dosb + h * p.dosh + i * p.dosn;
   float acc = 0.f;
-  if constexpr (PER == 4) {
+  if constexpr (PER == 2) {
+    const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(orow + lane * 2));
+    const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(drow + lane * 2));
+    acc = fmaf(of.x, df.x, acc);
+    acc = fmaf(of.y, df.y, acc);
+  } else if constexpr (PER == 4) {
     const uint2 ov = *reinterpret_cast<const uint2*>(orow + lane * 4);
     const uint2 dv = *reinterpret_cast<const uint2*>(drow + lane * 4);
     const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
@@ -145,10 +153,12 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) 
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  // zero this row of the fp32 dQ scratch
-  float4* zrow = reinterpret_cast<float4*>(p.dqacc + (static_cast<long long>(bh) * p.N + i) * D);
+  // zero this row of the fp32 dQ scratch (when dQ is accumulated there)
+  if (p.dqacc) {
+    float4* zrow = reinterpret_cast<float4*>(p.dqacc + (static_cast<long long>(bh) * p.N + i) * D);
 #pragma unroll
-  for (int e = lane; e < D / 4; e += 32) zrow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = lane; e < D / 4; e += 32) zrow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (lane == 0) {
     p.delta[warp] = acc;
     p.lse2[warp] = p.lse[static_cast<long long>(bh) * p.N + i] * 1.4426950408889634f;

@@ -30,7 +30,7 @@
  *   every pointer 16-byte aligned and every stride a multiple of 16 bytes
  *   (the tensor-memory-accelerator rule);
  *   ATTN_FP32 (fp32 storage, tf32 tensor-core products) only for the forward
- *   with D = 64; the backward supports bf16 with D in {128, 256}.
+ *   with D = 64; the backward supports bf16 with D in {64, 128, 256}.
  *
  * Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
  * default stream).  The return value reports host-side validation and launch
@@ -111,10 +111,10 @@ ATTN_API attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_te
                                        int window_right, float scale, void* stream);
 
 /*
- * Bytes of device workspace attn_bwd needs for these sizes: an fp32 dQ
- * accumulator [B,Hq,N,D] (the scratch the backward's atomic partial sums go
- * to) plus two fp32 row statistics [B,Hq,N'] (rowsum(dO*O) and lse*log2(e),
- * N' = N rounded up to 128).  Returns 0 for invalid sizes.
+ * Bytes of device workspace attn_bwd needs for these sizes: two fp32 row
+ * statistics [B,Hq,N'] (rowsum(dO*O) and lse*log2(e), N' = N rounded up to
+ * 128), and for D = 256 also an fp32 dQ accumulator [B,Hq,N,D] (the scratch
+ * that backward's partial sums are added into).  Returns 0 for invalid sizes.
  */
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D);
 
@@ -124,6 +124,13 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D);
  * (bf16).  workspace: device memory of at least attn_bwd_workspace_bytes()
  * bytes, 256-byte aligned, owned by the caller; its contents on entry do not
  * matter and are overwritten.  Outputs must not alias inputs.
+ *
+ * D = 64 and 128 use the atomic-free form with seven products per tile pair
+ * (FlashAttention (Metal Port) README, Documentation section): a
+ * column-parallel kernel computes dK and dV, a row-parallel kernel computes
+ * dQ, every gradient element is summed in one fixed order and the results
+ * are bitwise reproducible.  D = 256 uses the five-product form with dQ
+ * partial sums added into the fp32 workspace.
  */
 ATTN_API attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
                        const float* lse, attn_tensor_t dout, attn_tensor_t dq, attn_tensor_t dk,
@@ -162,8 +169,8 @@ ATTN_API attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_te
  * device looks up the scratch array's device address with that device
  * current; make that first call before any stream capture.  Every call
  * shares the one array: the kernels re-initialise everything they read from
- * it (the dQ accumulator is zeroed and the row statistics rewritten on every
- * call), but two calls whose work overlaps on the GPU (different streams, or
+ * it (the row statistics are rewritten and, for D = 256, the dQ accumulator
+ * is zeroed on every call), but two calls whose work overlaps on the GPU (different streams, or
  * different host threads) race on it and must be serialised by the caller.
  */
 ATTN_API attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
@@ -194,8 +201,8 @@ ATTN_API void attn_debug_set_flags(int flags);
 /*
  * Timing hook.  When both are non-NULL (cudaEvent_t handles owned by the
  * caller), the next attn_bwd call records `start` on its stream right before
- * launching its main dK/dV kernel and `stop` right after it, then forgets
- * them; this times that kernel alone inside a longer stream of work.
+ * launching its dK/dV kernel and `stop` right after it, then forgets them;
+ * this times that kernel alone inside a longer stream of work.
  */
 ATTN_API void attn_debug_set_bwd_events(void* start, void* stop);
 

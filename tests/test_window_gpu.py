@@ -44,7 +44,7 @@ def test_forward_window_fp32(window):
     assert abs_err(to_np(lse), l_ref) <= 1e-4
 
 
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("window", [(111, 0), (0, 0), (200, 200), (64, 300), (-1, 50)])
 def test_backward_window(D, window):
     N = 700

@@ -58,7 +58,8 @@ def test_noalloc_backward_matches_workspace_backward(D, causal, hq, hkv):
 
 def test_noalloc_rejects_sizes_beyond_the_scratch():
     f = _noalloc()
-    B, H, N, D = 4, 32, 4096, 128  # needs ~268 MB of scratch, more than 64 MiB
+    # head dimension 256 accumulates dQ in an fp32 scratch: ~537 MB here, more than 64 MiB
+    B, H, N, D = 4, 32, 4096, 256
     x = torch.zeros(16, device="cuda", dtype=torch.bfloat16)
     t = AttnTensor(ctypes.c_void_p(x.data_ptr()), H * N * D, N * D, D)
     code = f(t, t, t, t, ctypes.c_void_p(x.data_ptr()), t, t, t, t, B, H, H, N, D, 0, 1,
