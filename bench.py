@@ -31,11 +31,12 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD_INDEX = 2  # MHA fwd+bwd B=2 H=16 N=4096 D=128 causal
 
-# DRAM traffic of one launch of the dominant kernel (bwd_dkdv_kernel<128,3,2>)
-# from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
-# hash of the kernel source it was taken on; it is reported as null once the
-# source changes (profiles/ncu_full_fwd_bwd_mha_4096_causal.md has the capture).
-DOMINANT_TRAFFIC = {"bytes": 678316800, "src_sha": "7905a6d0eb2a1f45"}
+# The dominant kernel of the step: the backward's dK/dV kernel.
+DOMINANT_KERNEL = "bwd_kv_kernel<128,2,2>"
+# DRAM traffic of one launch of it from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), with the hash of the kernel sources it was taken on;
+# it is reported as null once the sources change (profiles/ holds the capture).
+DOMINANT_TRAFFIC = {"bytes": None, "src_sha": ""}
 
 
 def parse_args():
@@ -59,7 +60,7 @@ def dist_info():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "bwd.cuh"):
+    for f in ("ptx.cuh", "bwd.cuh", "bwd_split.cuh"):
         with open(os.path.join(ROOT, "exact_tiled_attention_37_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -339,9 +340,10 @@ def run_native(args):
 
     peaks = load_peaks()
     dom_ms = statistics.mean(main_ms)
-    # algorithmic FLOPs of one dK/dV-kernel launch: all five products of the
-    # backward (the preprocess and dQ-finalize kernels do no tensor work)
-    dom_flops = w.bwd_flops(causal)
+    # algorithmic FLOPs of one dK/dV-kernel launch: four products (S^T, dP^T,
+    # dV, dK) over the visible tile pairs, each as costly as one of the
+    # forward's two products
+    dom_flops = 4 * w.fwd_flops(causal) / 2
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     traffic = DOMINANT_TRAFFIC["bytes"] if DOMINANT_TRAFFIC["src_sha"] == kernel_source_sha() else None
     peak = peaks["bf16_tflops_sustained"]
@@ -367,7 +369,7 @@ def run_native(args):
                 "frac_of_peak": round(w.fwd_flops(causal) / fwd_ms / 1e9 / peaks["bf16_tflops"], 4)},
         "bwd": {"ms": round(bwd_ms, 4), "tflops": round(w.bwd_flops(causal) / bwd_ms / 1e9, 1),
                 "frac_of_peak": round(w.bwd_flops(causal) / bwd_ms / 1e9 / peaks["bf16_tflops"], 4)},
-        "roofline": {"kernel": "bwd_dkdv_kernel<128,3,2>", "bound": "tensor",
+        "roofline": {"kernel": DOMINANT_KERNEL, "bound": "tensor",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16 sustained",

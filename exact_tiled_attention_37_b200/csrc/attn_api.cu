@@ -207,12 +207,12 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
 
 // Head dimensions 64 and 128: preprocess, then the column-parallel dK/dV
 // kernel and the row-parallel dQ kernel (no scratch, no atomics).
-template <int D, int NQS, int NS>
+template <int D, int NQS, int NS, int NWG>
 attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
                                const attn_tensor_t& v, const attn_tensor_t& dout,
                                eta::BwdParams& p, cudaStream_t st) {
-  using CKV = eta::BwdKVCfg<D, NQS>;
-  using CQ = eta::BwdQCfg<D, NS>;
+  using CKV = eta::BwdKVCfg<D, NQS, NWG>;
+  using CQ = eta::BwdQCfg<D, NS, NWG>;
   CUtensorMap tq, tk, tv, tdo;
   attn_status_t s;
   if ((s = make_map(&tq, q, p.B, p.Hq, p.N, D, 2, 128)) != ATTN_OK) return s;
@@ -222,8 +222,8 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
   eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
-  auto kkv = eta::bwd_kv_kernel<D, NQS>;
-  auto kq = eta::bwd_q_kernel<D, NS>;
+  auto kkv = eta::bwd_kv_kernel<D, NQS, NWG>;
+  auto kq = eta::bwd_q_kernel<D, NS, NWG>;
   if ((s = set_smem(kkv, CKV::SMEM_BYTES)) != ATTN_OK) return s;
   if ((s = set_smem(kq, CQ::SMEM_BYTES)) != ATTN_OK) return s;
   const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128);
@@ -428,8 +428,10 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
   p.wait_limit_ns = g_wait_limit_ns.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 64) return launch_bwd_split<64, 4, 8>(q, k, v, dout, p, st);
-  if (D == 128) return launch_bwd_split<128, 2, 4>(q, k, v, dout, p, st);
+  // per head dimension: Q/dO stages of the dK/dV kernel, K/V ring slots of
+  // the dQ kernel, elementwise warpgroups (measured best on B200)
+  if (D == 64) return launch_bwd_split<64, 4, 8, 4>(q, k, v, dout, p, st);
+  if (D == 128) return launch_bwd_split<128, 2, 5, 2>(q, k, v, dout, p, st);
   return launch_bwd<256, 1, 1>(q, k, v, dout, p, st);
 }
 

@@ -11,7 +11,12 @@
 //    dP^T = V dO_i^T, P^T, dS^T, dV += P^T dO_i, dK += dS^T Q_i.
 //
 // Both read lse2 = lse log2(e) and Delta = rowsum(dO O) from the
-// preprocess kernel.  All MMAs are M = 128, N = 128 (or D) shapes.
+// preprocess kernel.  All MMAs are M = 128, N = 128 (or D) shapes, issued
+// by one whole warp (one elected lane issues each instruction).  NWG
+// elementwise warpgroups split the 128 columns of every tile: warpgroup g
+// owns columns [CW g, CW g + CW), CW = 128 / NWG, and thread t of it owns
+// row t (its TMEM lane).  A bf16 tile written back into TMEM keeps column c
+// of warpgroup g at packed column CW g + (c - CW g) / 2.
 #pragma once
 
 #include "bwd.cuh"
@@ -19,36 +24,83 @@
 
 namespace eta {
 
+// Packed TMEM column of the first element of MMA K-step ks (16 elements)
+// when the 128 columns were split into groups of CW and each group packed
+// two bf16 per column at its own start.
+template <int CW>
+__device__ __forceinline__ constexpr uint32_t packed_col(int ks) {
+  return static_cast<uint32_t>((16 * ks / CW) * CW + ((16 * ks) % CW) / 2);
+}
+
+// NC fp32 TMEM columns of this thread's lane, times mul, as bf16 to row[0..NC).
+template <int NC>
+__device__ __forceinline__ void tmem_row_to_bf16(uint32_t taddr, __nv_bfloat16* row, float mul,
+                                                 bool valid) {
+  static_assert(NC % 16 == 0, "16-column chunks");
+#pragma unroll 1
+  for (int c = 0; c < NC / 16; ++c) {
+    uint32_t r[16];
+    tmem_ld16(taddr + 16 * c, r);
+    tmem_wait_ld();
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(row + 16 * c);
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(u2f(r[8 * v + 0]) * mul, u2f(r[8 * v + 1]) * mul);
+        w.y = pack_bf16x2(u2f(r[8 * v + 2]) * mul, u2f(r[8 * v + 3]) * mul);
+        w.z = pack_bf16x2(u2f(r[8 * v + 4]) * mul, u2f(r[8 * v + 5]) * mul);
+        w.w = pack_bf16x2(u2f(r[8 * v + 6]) * mul, u2f(r[8 * v + 7]) * mul);
+        dst[v] = w;
+      }
+    }
+  }
+}
+
+// Stores CW/2 packed columns (CW = 32 or 64).
+template <int CW>
+__device__ __forceinline__ void tmem_store_packed(uint32_t taddr, const uint32_t (&pk)[CW / 2]) {
+  if constexpr (CW == 64) {
+    tmem_st32(taddr, pk);
+  } else {
+    tmem_st16(taddr, pk);
+  }
+}
+
 // ============================================================ dQ kernel
-template <int D, int NS_>
+template <int D, int NS_, int NWG_>
 struct BwdQCfg {
   static constexpr int BM = 128, BN = 128;
+  static constexpr int NWG = NWG_, CW = 128 / NWG;
   static constexpr int ROWB = D * 2;
   static constexpr int NCHUNK = ROWB / 128;
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * ROWB;
   static constexpr int KSTEPS = ROWB / 32;      // S, dP over D
   static constexpr int NS = NS_;                // K/V ring slots (K_j, V_j alternate)
-  // TMEM: S[2] (128 each; dS bf16 written back into its first 64 columns) | dP | dQ
+  // TMEM: S[2] (128 each; dS bf16 written back) | dP | dQ
   static constexpr int T_S = 0, T_DP = 256, T_DQ = 384, TMEM_COLS = 512;
   static constexpr int SMEM_Q = 0, SMEM_DO = TILE, SMEM_KV = 2 * TILE;
   static constexpr int SMEM_BAR = SMEM_KV + NS * TILE;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], dp_full, ds_full, dq_done, done
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], dp_full, ds_full, dq_done, done, dp_consumed
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS, B_DP = 3 + 2 * NS,
                        B_DS = 4 + 2 * NS, B_DQ = 5 + 2 * NS, B_DONE = 6 + 2 * NS,
-                       NBAR = 7 + 2 * NS;
+                       B_DPC = 7 + 2 * NS, NBAR = 8 + 2 * NS;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
-  static constexpr int THREADS = 320;           // 2 warpgroups (64 key columns each) + producer + MMA
+  static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;  // warp indices
+  static constexpr int THREADS = 128 * NWG + 64;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(D % (16 * NWG) == 0, "dQ columns per warpgroup");
 };
 
-template <int D, int NS>
-__global__ void __launch_bounds__(320, 1)
+template <int D, int NS, int NWG>
+__global__ void __launch_bounds__(128 * NWG + 64, 1)
     bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                  const BwdParams p) {
-  using C = BwdQCfg<D, NS>;
+  using C = BwdQCfg<D, NS, NWG>;
+  constexpr int CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -81,14 +133,15 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(BAR(C::B_S + 0), 1);
     mbar_init(BAR(C::B_S + 1), 1);
     mbar_init(BAR(C::B_DP), 1);
-    mbar_init(BAR(C::B_DS), 8);
+    mbar_init(BAR(C::B_DS), 4 * NWG);
+    mbar_init(BAR(C::B_DPC), 4 * NWG);
     mbar_init(BAR(C::B_DQ), 1);
     mbar_init(BAR(C::B_DONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == C::MMA) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -98,9 +151,9 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 
-  if (warp < 8) {
+  if (warp < 4 * NWG) {
     // ---------------------------------------- dS rows (thread r = query row r), then dQ
-    const int par = warp >> 2;             // key columns [64 par, 64 par + 64) of each tile
+    const int par = warp >> 2;             // key columns [CW par, CW par + CW) of each tile
     const int r = threadIdx.x & 127;
     const int qrow = q0 + r;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -110,67 +163,62 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int u = 0; u < n; ++u) {
       const int buf = u & 1;
-      const uint32_t s_addr = tmem + lane_base + C::T_S + 128 * buf + 64 * par;
+      const uint32_t s_addr = tmem + lane_base + C::T_S + 128 * buf + CW * par;
       if (!W.wait_warp(BAR(C::B_S + buf), (u >> 1) & 1, 100)) { ok = false; break; }
-      if (r == 0) ETA_FTRACE_AT(tcta, par, u, 0);
+      if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 0);
       tc_fence_after();
-      float s[64];
-      tmem_load_row<64>(s_addr, s);
-      const int2 cw = col_window(C::BN * (j0 + u) + 64 * par, qrow, p.N, p.wl, p.wr);
+      float s[CW];
+      tmem_load_row<CW>(s_addr, s);
+      const int2 cw = col_window(C::BN * (j0 + u) + CW * par, qrow, p.N, p.wl, p.wr);
       const float2 c2 = make_float2(p.c, p.c), nl2 = make_float2(-lse2, -lse2);
+      if (cw.x <= 0 && cw.y >= CW) {
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const float2 x = ffma2(make_float2(s[i], s[i + 1]), c2, nl2);
-        s[i] = (i < cw.x || i >= cw.y) ? 0.f : ex2(x.x);
-        s[i + 1] = (i + 1 < cw.x || i + 1 >= cw.y) ? 0.f : ex2(x.y);
+        for (int i = 0; i < CW; i += 2) {
+          const float2 x = ffma2(make_float2(s[i], s[i + 1]), c2, nl2);
+          s[i] = ex2(x.x);
+          s[i + 1] = ex2(x.y);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < CW; i += 2) {
+          const float2 x = ffma2(make_float2(s[i], s[i + 1]), c2, nl2);
+          s[i] = (i < cw.x || i >= cw.y) ? 0.f : ex2(x.x);
+          s[i + 1] = (i + 1 < cw.x || i + 1 >= cw.y) ? 0.f : ex2(x.y);
+        }
       }
-      if (r == 0) ETA_FTRACE_AT(tcta, par, u, 1);
+      if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 1);
       if (!W.wait_warp(BAR(C::B_DP), u & 1, 101)) { ok = false; break; }
-      if (r == 0) ETA_FTRACE_AT(tcta, par, u, 2);
+      if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 2);
       tc_fence_after();
-      float dp[64];
-      tmem_load_row<64>(tmem + lane_base + C::T_DP + 64 * par, dp);
-      uint32_t pk[32];
+      float dp[CW];
+      tmem_load_row<CW>(tmem + lane_base + C::T_DP + CW * par, dp);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DPC));  // dP may be overwritten
+      uint32_t pk[CW / 2];
       const float2 d2 = make_float2(dlt, dlt);
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
+      for (int i = 0; i < CW; i += 2) {
         const float2 g = fsub2(make_float2(dp[i], dp[i + 1]), d2);
         pk[i / 2] = pack_bf16x2(s[i] * g.x, s[i + 1] * g.y);
       }
-      // dS (bf16 pairs) into the first 32 of this half's 64 S columns
-      tmem_st32(s_addr, pk);
+      // dS (bf16 pairs) into the first CW/2 of this group's S columns
+      tmem_store_packed<CW>(s_addr, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DS));
-      if (r == 0) ETA_FTRACE_AT(tcta, par, u, 3);
+      if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 3);
     }
-    if (ok && W.wait_warp(BAR(C::B_DQ), 0, 102)) {
+    if (ok && n > 0 && W.wait_warp(BAR(C::B_DQ), 0, 102)) {
       tc_fence_after();
-      // dQ * scale in bf16: warpgroup par stores columns [D/2 par, D/2 par + D/2)
-      const bool valid = qrow < p.N;
+      // dQ * scale in bf16: warpgroup par stores columns [D/NWG par, D/NWG (par + 1))
+      constexpr int DC = D / NWG;
       __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.dq) + b * p.dqsb + h * p.dqsh +
-                           static_cast<long long>(qrow) * p.dqsn + (D / 2) * par;
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + C::T_DQ + (D / 2) * par + 32 * c, rr);
-        tmem_wait_ld();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(row + 32 * c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(u2f(rr[8 * v + 0]) * p.scale, u2f(rr[8 * v + 1]) * p.scale);
-            w.y = pack_bf16x2(u2f(rr[8 * v + 2]) * p.scale, u2f(rr[8 * v + 3]) * p.scale);
-            w.z = pack_bf16x2(u2f(rr[8 * v + 4]) * p.scale, u2f(rr[8 * v + 5]) * p.scale);
-            w.w = pack_bf16x2(u2f(rr[8 * v + 6]) * p.scale, u2f(rr[8 * v + 7]) * p.scale);
-            dst[v] = w;
-          }
-        }
-      }
+                           static_cast<long long>(qrow) * p.dqsn + DC * par;
+      tmem_row_to_bf16<DC>(tmem + lane_base + C::T_DQ + DC * par, row, p.scale, qrow < p.N);
     }
-  } else if (warp == 8) {
+  } else if (warp == C::PRODUCER) {
     // ---------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -201,124 +249,131 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ---------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_make(128, 128, 1u, false, false);  // S, dP
-      constexpr uint32_t id_q = idesc_make(128, D, 1u, false, true);     // dQ += dS K
-      const SDesc dq_ = sdesc_base(sbase + C::SMEM_Q, 16, 1024);
-      const SDesc ddo = sdesc_base(sbase + C::SMEM_DO, 16, 1024);
-      auto kslot = [&](int u) { return (2 * u) % C::NS; };
-      auto kph = [&](int u) { return static_cast<uint32_t>((2 * u) / C::NS) & 1u; };
-      auto vslot = [&](int u) { return (2 * u + 1) % C::NS; };
-      auto vph = [&](int u) { return static_cast<uint32_t>((2 * u + 1) / C::NS) & 1u; };
-      // S(u) = Q K^T into S[u % 2]
-      auto issue_s = [&](int u) -> bool {
-        if (!W.wait(BAR(C::B_KVF + kslot(u)), kph(u), 120)) return false;
-        tc_fence_after();
-        const SDesc kb = sdesc_base(sbase + C::SMEM_KV + kslot(u) * C::TILE, 16, 1024);
-        const uint32_t d = tmem + C::T_S + 128 * (u & 1);
+  } else if (warp == C::MMA) {
+    // ---------------------------------------- MMA issuer (whole warp, one elected lane issues)
+    constexpr uint32_t id_s = idesc_make(128, 128, 1u, false, false);  // S, dP
+    constexpr uint32_t id_q = idesc_make(128, D, 1u, false, true);     // dQ += dS K
+    const SDesc dq_ = sdesc_base(sbase + C::SMEM_Q, 16, 1024);
+    const SDesc ddo = sdesc_base(sbase + C::SMEM_DO, 16, 1024);
+    auto kslot = [&](int u) { return (2 * u) % C::NS; };
+    auto kph = [&](int u) { return static_cast<uint32_t>((2 * u) / C::NS) & 1u; };
+    auto vslot = [&](int u) { return (2 * u + 1) % C::NS; };
+    auto vph = [&](int u) { return static_cast<uint32_t>((2 * u + 1) / C::NS) & 1u; };
+    // S(u) = Q K^T into S[u % 2]
+    auto issue_s = [&](int u) -> bool {
+      if (!W.wait_warp(BAR(C::B_KVF + kslot(u)), kph(u), 120)) return false;
+      tc_fence_after();
+      const SDesc kb = sdesc_base(sbase + C::SMEM_KV + kslot(u) * C::TILE, 16, 1024);
+      const uint32_t d = tmem + C::T_S + 128 * (u & 1);
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          mma_ss<false>(d, sdesc_at(dq_, off), sdesc_at(kb, off), id_s, ks > 0);
-        }
-        mma_commit(BAR(C::B_S + (u & 1)));
-        return true;
-      };
-      // dP(u) = dO V^T
-      auto issue_dp = [&](int u) -> bool {
-        if (!W.wait(BAR(C::B_KVF + vslot(u)), vph(u), 121)) return false;
-        tc_fence_after();
-        const SDesc vb = sdesc_base(sbase + C::SMEM_KV + vslot(u) * C::TILE, 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          mma_ss<false>(tmem + C::T_DP, sdesc_at(ddo, off), sdesc_at(vb, off), id_s, ks > 0);
-        }
-        mma_commit(BAR(C::B_DP));
-        mma_commit(BAR(C::B_KVE + vslot(u)));  // V_u is not read again
-        return true;
-      };
-      bool ok = W.wait(BAR(C::B_Q), 0, 122);
-      if (ok && n > 0) ok = issue_s(0) && issue_dp(0);
-      if (ok && n > 1) ok = issue_s(1);
-      for (int u = 0; ok && u < n; ++u) {
-        // dS(u) is in S[u % 2] and dP has been read
-        if (!W.wait(BAR(C::B_DS), u & 1, 123)) { ok = false; break; }
-        ETA_FTRACE_AT(tcta, 2, u, 0);
-        tc_fence_after();
-        // dQ += dS K_u: A = dS from TMEM (key k at column (k / 64) * 64 + (k % 64) / 2),
-        // B = K_u as an MN-major operand (N = D, K = 128 keys)
-        const SDesc kb = sdesc_base(sbase + C::SMEM_KV + kslot(u) * C::TILE, C::CHUNK, 1024);
-        const uint32_t a = tmem + C::T_S + 128 * (u & 1);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ts<false>(tmem + C::T_DQ, a + 64 * (ks >> 2) + 8 * (ks & 3), sdesc_at(kb, ks * 2048),
-                        id_q, (u > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(BAR(C::B_KVE + kslot(u)));  // K_u is not read again
-        ETA_FTRACE_AT(tcta, 2, u, 1);
-        if (u + 1 < n && !issue_dp(u + 1)) { ok = false; break; }
-        ETA_FTRACE_AT(tcta, 2, u, 2);
-        if (u + 2 < n && !issue_s(u + 2)) { ok = false; break; }
-        ETA_FTRACE_AT(tcta, 2, u, 3);
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+        mma_ss_w(d, sdesc_at(dq_, off), sdesc_at(kb, off), id_s, ks > 0);
       }
-      if (ok) mma_commit(BAR(C::B_DQ));
-      mma_commit(BAR(C::B_DONE));
-      W.drain(BAR(C::B_DONE), 0, 124);
+      mma_commit_w(BAR(C::B_S + (u & 1)));
+      return true;
+    };
+    // dP(u) = dO V^T
+    auto issue_dp = [&](int u) -> bool {
+      if (!W.wait_warp(BAR(C::B_KVF + vslot(u)), vph(u), 121)) return false;
+      tc_fence_after();
+      const SDesc vb = sdesc_base(sbase + C::SMEM_KV + vslot(u) * C::TILE, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+        mma_ss_w(tmem + C::T_DP, sdesc_at(ddo, off), sdesc_at(vb, off), id_s, ks > 0);
+      }
+      mma_commit_w(BAR(C::B_DP));
+      mma_commit_w(BAR(C::B_KVE + vslot(u)));  // V_u is not read again
+      return true;
+    };
+    bool ok = W.wait_warp(BAR(C::B_Q), 0, 122);
+    if (ok && n > 0) ok = issue_s(0) && issue_dp(0);
+    if (ok && n > 1) ok = issue_s(1);
+    for (int u = 0; ok && u < n; ++u) {
+      // dP(u + 1) as soon as the elementwise warps have loaded dP(u)
+      if (u + 1 < n) {
+        if (!W.wait_warp(BAR(C::B_DPC), u & 1, 125)) { ok = false; break; }
+        if (!issue_dp(u + 1)) { ok = false; break; }
+      }
+      ETA_FTRACE_AT(tcta, 2, u, 2);
+      // dS(u) is in S[u % 2]
+      if (!W.wait_warp(BAR(C::B_DS), u & 1, 123)) { ok = false; break; }
+      ETA_FTRACE_AT(tcta, 2, u, 0);
+      tc_fence_after();
+      // dQ += dS K_u: A = dS from TMEM, B = K_u as an MN-major operand (N = D, K = 128 keys)
+      const SDesc kb = sdesc_base(sbase + C::SMEM_KV + kslot(u) * C::TILE, C::CHUNK, 1024);
+      const uint32_t a = tmem + C::T_S + 128 * (u & 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts_w(tmem + C::T_DQ, a + packed_col<CW>(ks), sdesc_at(kb, ks * 2048), id_q,
+                 (u > 0 || ks > 0) ? 1u : 0u);
+      mma_commit_w(BAR(C::B_KVE + kslot(u)));  // K_u is not read again
+      ETA_FTRACE_AT(tcta, 2, u, 1);
+      // S(u + 2) into S[u % 2] after dQ(u) has read dS(u) (issue order)
+      if (u + 2 < n && !issue_s(u + 2)) { ok = false; break; }
+      ETA_FTRACE_AT(tcta, 2, u, 3);
     }
+    if (ok) mma_commit_w(BAR(C::B_DQ));
+    mma_commit_w(BAR(C::B_DONE));
+    W.drain(BAR(C::B_DONE), 0, 124);
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-
 // ============================================================ dK / dV kernel
 // P^T goes through shared memory (the A operand of dV += P^T dO_i) so that
-// S^T of the next query tile can be computed as soon as the softmax
-// warpgroups have loaded S^T of this one; dS^T stays in TMEM (in the dP^T
+// S^T of the next query tile can be computed as soon as the elementwise
+// warps have loaded S^T of this one; dS^T stays in TMEM (in the dP^T
 // columns it was computed from).
-template <int D, int NQS>
+template <int D, int NQS, int NWG_>
 struct BwdKVCfg {
   static constexpr int BC = 128, BR = 128;
+  static constexpr int NWG = NWG_, CW = 128 / NWG;
   static constexpr int ROWB = D * 2;
   static constexpr int NCHUNK = ROWB / 128;
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * ROWB;
   static constexpr int KSTEPS = ROWB / 32;
-  // TMEM: S^T | dP^T (dS^T bf16 written back into its first columns) | dV | dK
+  // TMEM: S^T | dP^T (dS^T bf16 written back) | dV | dK
   static constexpr int T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D, TMEM_COLS = 512;
   static constexpr int S_K = 0, S_V = TILE, S_Q = 2 * TILE;   // [NQS] Q tiles
   static constexpr int S_DO = S_Q + NQS * TILE;                // [NQS] dO tiles
   static constexpr int S_P = S_DO + NQS * TILE;                // P^T: 128 key rows x 128 queries bf16
   static constexpr int S_STAT = S_P + 128 * 256;               // [NQS] lse2[128], delta[128]
   static constexpr int S_BAR = S_STAT + NQS * 1024;
-  // kv, q_full[NQS], q_empty[NQS], s, s_consumed, dp, p, p_empty, ds, kv_done, done
-  static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NQS, B_S = 1 + 2 * NQS, B_SC = 2 + 2 * NQS,
-                       B_DP = 3 + 2 * NQS, B_P = 4 + 2 * NQS, B_PE = 5 + 2 * NQS,
-                       B_DS = 6 + 2 * NQS, B_KVD = 7 + 2 * NQS, B_DONE = 8 + 2 * NQS,
-                       NBAR = 9 + 2 * NQS;
+  // kv, q_full[NQS] (Q_i and its row statistics), q_empty[NQS], do_full[NQS],
+  // do_empty[NQS], s, s_consumed, dp, p, p_empty, ds, kv_done, done
+  static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NQS, B_OF = 1 + 2 * NQS,
+                       B_OE = 1 + 3 * NQS, B_S = 1 + 4 * NQS, B_SC = 2 + 4 * NQS,
+                       B_DP = 3 + 4 * NQS, B_P = 4 + 4 * NQS, B_PE = 5 + 4 * NQS,
+                       B_DS = 6 + 4 * NQS, B_KVD = 7 + 4 * NQS, B_DONE = 8 + 4 * NQS,
+                       NBAR = 9 + 4 * NQS;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int LAYOUT = S_MISC + 16;
   // dynamic shared memory: the layout plus as much of the 1024-byte alignment
   // slack as the per-block limit leaves (the kernel checks the actual slack)
   static constexpr int SMEM_BYTES = LAYOUT + 1024 <= 232448 ? LAYOUT + 1024 : 232448;
-  static constexpr int THREADS = 320;  // 2 warpgroups (64 query columns each) + producer + MMA
+  static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;  // warp indices
+  static constexpr int THREADS = 128 * NWG + 64;
   static_assert(LAYOUT <= 232448, "shared memory budget");
+  static_assert(NWG % 2 == 0 && D % (8 * NWG) == 0, "dK/dV columns per warpgroup");
 };
 
-template <int D, int NQS>
-__global__ void __launch_bounds__(320, 1)
+template <int D, int NQS, int NWG>
+__global__ void __launch_bounds__(128 * NWG + 64, 1)
     bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p) {
-  using C = BwdKVCfg<D, NQS>;
+  using C = BwdKVCfg<D, NQS, NWG>;
+  constexpr int CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -358,20 +413,22 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < NQS; ++s) {
       mbar_init(BAR(C::B_QF + s), 1);
       mbar_init(BAR(C::B_QE + s), 1);
+      mbar_init(BAR(C::B_OF + s), 1);
+      mbar_init(BAR(C::B_OE + s), 1);
     }
     mbar_init(BAR(C::B_S), 1);
-    mbar_init(BAR(C::B_SC), 8);
+    mbar_init(BAR(C::B_SC), 4 * NWG);
     mbar_init(BAR(C::B_DP), 1);
-    mbar_init(BAR(C::B_P), 8);
+    mbar_init(BAR(C::B_P), 4 * NWG);
     mbar_init(BAR(C::B_PE), 1);
-    mbar_init(BAR(C::B_DS), 8);
+    mbar_init(BAR(C::B_DS), 4 * NWG);
     mbar_init(BAR(C::B_KVD), 1);
     mbar_init(BAR(C::B_DONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == C::MMA) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -381,38 +438,41 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 
-  if (warp < 8) {
+  if (warp < 4 * NWG) {
     // ---------------------------------------- P^T, dS^T rows (thread j = key row j)
-    const int par = warp >> 2;           // query columns [64 par, 64 par + 64) of each tile
+    const int par = warp >> 2;           // query columns [CW par, CW par + CW) of each tile
     const int j = threadIdx.x & 127;
     const int jg = k0 + j;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t st_addr = tmem + lane_base + C::T_ST + 64 * par;
-    const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + 64 * par;
-    // this thread's 128-byte row of P^T in the 128-byte-swizzled chunk of its columns
-    uint8_t* prow = smem + C::S_P + par * C::CHUNK + j * 128;
+    const uint32_t st_addr = tmem + lane_base + C::T_ST + CW * par;
+    const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + CW * par;
+    // this thread's part of its 128-byte P^T row in the 128-byte-swizzled
+    // chunk holding its columns: 16-byte granules g0 .. g0 + CW/8 - 1
+    uint8_t* prow = smem + C::S_P + ((CW * par) / 64) * C::CHUNK + j * 128;
+    const int g0 = ((CW * par) % 64) / 8;
     const int swz = j & 7;
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int stage = it % NQS;
       if (!W.wait_warp(BAR(C::B_S), it & 1, 130)) { ok = false; break; }
-      if (j == 0) ETA_TRACE_AT(tcta, par, it, 0);
+      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 0);
       tc_fence_after();
-      float pr[64];
-      tmem_load_row<64>(st_addr, pr);
+      float pr[CW];
+      tmem_load_row<CW>(st_addr, pr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_SC));  // S^T may be overwritten
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::S_STAT + stage * 1024) + 64 * par;
+      const float* lse2 =
+          reinterpret_cast<const float*>(smem + C::S_STAT + stage * 1024) + CW * par;
       const float* dlt = lse2 + 128;
-      const int ig0 = qtile_of(it) * C::BR + 64 * par;
+      const int ig0 = qtile_of(it) * C::BR + CW * par;
       // window: query ig0 + i sees key jg iff jg - wr <= ig0 + i <= jg + wl
       const int ilo = p.wr < 0 ? -(1 << 30) : jg - p.wr - ig0;
       const int ihi = p.wl < 0 ? (1 << 30) : jg + p.wl - ig0;
       const float2 c2 = make_float2(p.c, p.c);
-      if (ilo <= 0 && ihi >= 63) {
+      if (ilo <= 0 && ihi >= CW - 1) {
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
+        for (int i = 0; i < CW; i += 2) {
           const float2 l2 = *reinterpret_cast<const float2*>(lse2 + i);
           const float2 x = ffma2(make_float2(pr[i], pr[i + 1]), c2, make_float2(-l2.x, -l2.y));
           pr[i] = ex2(x.x);
@@ -420,7 +480,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
+        for (int i = 0; i < CW; i += 2) {
           const float2 l2 = *reinterpret_cast<const float2*>(lse2 + i);
           const float2 x = ffma2(make_float2(pr[i], pr[i + 1]), c2, make_float2(-l2.x, -l2.y));
           pr[i] = (i < ilo || i > ihi) ? 0.f : ex2(x.x);
@@ -430,22 +490,22 @@ __global__ void __launch_bounds__(320, 1)
       // the dV MMA of the previous tile must be done reading P^T
       if (!W.wait_warp(BAR(C::B_PE), (it & 1) ^ 1, 133)) { ok = false; break; }
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < CW / 8; ++g) {
         const uint4 w = make_uint4(pack_bf16x2(pr[8 * g + 0], pr[8 * g + 1]),
                                    pack_bf16x2(pr[8 * g + 2], pr[8 * g + 3]),
                                    pack_bf16x2(pr[8 * g + 4], pr[8 * g + 5]),
                                    pack_bf16x2(pr[8 * g + 6], pr[8 * g + 7]));
-        *reinterpret_cast<uint4*>(prow + ((g ^ swz) << 4)) = w;
+        *reinterpret_cast<uint4*>(prow + (((g0 + g) ^ swz) << 4)) = w;
       }
       fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_P));
-      if (j == 0) ETA_TRACE_AT(tcta, par, it, 1);
+      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 1);
       if (!W.wait_warp(BAR(C::B_DP), it & 1, 131)) { ok = false; break; }
-      if (j == 0) ETA_TRACE_AT(tcta, par, it, 2);
+      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 2);
       tc_fence_after();
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < CW / 32; ++h2) {
         uint32_t rd[32];
         tmem_ld32(dpt_addr + 32 * h2, rd);
         tmem_wait_ld();
@@ -457,7 +517,7 @@ __global__ void __launch_bounds__(320, 1)
           const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
           dk[i / 2] = pack_bf16x2(pr[c] * g.x, pr[c + 1] * g.y);
         }
-        // dS^T of columns [32 h2, 32 h2 + 32) -> dP^T columns 16 h2 .. 16 h2 + 15
+        // dS^T of columns [32 h2, 32 h2 + 32) -> packed columns 16 h2 .. 16 h2 + 15
         // (already read: each half lies below the columns still to be loaded)
         tmem_st16(dpt_addr + 16 * h2, dk);
       }
@@ -465,49 +525,27 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DS));
-      if (j == 0) ETA_TRACE_AT(tcta, par, it, 3);
+      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 3);
     }
+    // epilogue: the first NWG/2 warpgroups store dV, the others dK (x scale),
+    // D / (NWG/2) columns each
+    constexpr int NG = NWG / 2, DC = D / NG;
+    const int which = par / NG, part = par % NG;
+    __nv_bfloat16* row =
+        which == 0 ? static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
+                         static_cast<long long>(jg) * p.dvsn + DC * part
+                   : static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
+                         static_cast<long long>(jg) * p.dksn + DC * part;
+    const bool valid = jg < p.N;
     if (ok && n > 0 && W.wait_warp(BAR(C::B_KVD), 0, 132)) {
       tc_fence_after();
-      // even warpgroup stores dV, odd warpgroup stores dK (x scale)
-      const bool valid = jg < p.N;
-      __nv_bfloat16* row =
-          par == 0 ? static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
-                         static_cast<long long>(jg) * p.dvsn
-                   : static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
-                         static_cast<long long>(jg) * p.dksn;
-      const float mul = par ? p.scale : 1.f;
-      const uint32_t col = par ? C::T_DK : C::T_DV;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + col + 32 * c, r);
-        tmem_wait_ld();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(row + 32 * c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(u2f(r[8 * v + 0]) * mul, u2f(r[8 * v + 1]) * mul);
-            w.y = pack_bf16x2(u2f(r[8 * v + 2]) * mul, u2f(r[8 * v + 3]) * mul);
-            w.z = pack_bf16x2(u2f(r[8 * v + 4]) * mul, u2f(r[8 * v + 5]) * mul);
-            w.w = pack_bf16x2(u2f(r[8 * v + 6]) * mul, u2f(r[8 * v + 7]) * mul);
-            dst[v] = w;
-          }
-        }
-      }
-    } else if (n == 0) {
+      tmem_row_to_bf16<DC>(tmem + lane_base + (which ? C::T_DK : C::T_DV) + DC * part, row,
+                           which ? p.scale : 1.f, valid);
+    } else if (n == 0 && valid) {
       // no query sees these keys: their gradients are zero
-      const bool valid = jg < p.N;
-      __nv_bfloat16* row =
-          par == 0 ? static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
-                         static_cast<long long>(jg) * p.dvsn
-                   : static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
-                         static_cast<long long>(jg) * p.dksn;
-      if (valid)
-        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
+      for (int c = 0; c < DC / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
     }
-  } else if (warp == 8) {
+  } else if (warp == C::PRODUCER) {
     // ---------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -519,19 +557,26 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_4d(sbase + C::S_K + c * C::CHUNK, &tm_k, BAR(C::B_KV), c * 64, k0, hk, b);
         tma_load_4d(sbase + C::S_V + c * C::CHUNK, &tm_v, BAR(C::B_KV), c * 64, k0, hk, b);
       }
-      int it = 0;
+      // dO_i and Q_i have their own barriers: dO_i's slot frees earlier (after
+      // dV) and is refilled first; Q_i (needed first, by S^T) follows.
+      int it = 0, issued_do = 0;
       for (; it < n; ++it) {
         const int stage = it % NQS;
-        if (!W.wait(BAR(C::B_QE + stage), ((it / NQS) & 1) ^ 1, 140)) break;
-        ETA_TRACE_AT(tcta, 3, it, 0);
+        const uint32_t par_empty = ((it / NQS) & 1) ^ 1;
         const int h = head_of(it);
         const int ig0 = qtile_of(it) * C::BR;
+        if (!W.wait(BAR(C::B_OE + stage), par_empty, 143)) break;
+        const uint32_t ofull = BAR(C::B_OF + stage);
+        mbar_expect_tx(ofull, C::TILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sbase + C::S_DO + stage * C::TILE + c * C::CHUNK, &tm_do, ofull, c * 64, ig0, h, b);
+        issued_do = it + 1;
+        if (!W.wait(BAR(C::B_QE + stage), par_empty, 140)) break;
+        ETA_TRACE_AT(tcta, 3, it, 0);
         const uint32_t full = BAR(C::B_QF + stage);
-        mbar_expect_tx(full, 2 * C::TILE + 1024);
-        for (int c = 0; c < C::NCHUNK; ++c) {
+        mbar_expect_tx(full, C::TILE + 1024);
+        for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full, c * 64, ig0, h, b);
-          tma_load_4d(sbase + C::S_DO + stage * C::TILE + c * C::CHUNK, &tm_do, full, c * 64, ig0, h, b);
-        }
         const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
         bulk_load(sbase + C::S_STAT + stage * 1024, p.lse2 + srow, 512, full);
         bulk_load(sbase + C::S_STAT + stage * 1024 + 512, p.delta + srow, 512, full);
@@ -542,86 +587,92 @@ __global__ void __launch_bounds__(320, 1)
         const int last = s + ((issued - 1 - s) / NQS) * NQS;
         W.drain(BAR(C::B_QF + s), static_cast<uint32_t>(last / NQS) & 1u, 142);
       }
+      for (int s = 0; s < NQS && s < issued_do; ++s) {
+        const int last = s + ((issued_do - 1 - s) / NQS) * NQS;
+        W.drain(BAR(C::B_OF + s), static_cast<uint32_t>(last / NQS) & 1u, 144);
+      }
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ---------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_make(128, 128, 1u, false, false);  // S^T, dP^T
-      constexpr uint32_t id_kv = idesc_make(128, D, 1u, false, true);    // dV, dK
-      const SDesc dK = sdesc_base(sbase + C::S_K, 16, 1024);
-      const SDesc dV = sdesc_base(sbase + C::S_V, 16, 1024);
-      const SDesc dP = sdesc_base(sbase + C::S_P, 16, 1024);
-      auto issue_s = [&](int it) -> bool {
-        const int stage = it % NQS;
-        if (!W.wait(BAR(C::B_QF + stage), (it / NQS) & 1, 150)) return false;
-        tc_fence_after();
-        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, 16, 1024);
+  } else if (warp == C::MMA) {
+    // ---------------------------------------- MMA issuer (whole warp, one elected lane issues)
+    constexpr uint32_t id_s = idesc_make(128, 128, 1u, false, false);  // S^T, dP^T
+    constexpr uint32_t id_kv = idesc_make(128, D, 1u, false, true);    // dV, dK
+    const SDesc dK = sdesc_base(sbase + C::S_K, 16, 1024);
+    const SDesc dV = sdesc_base(sbase + C::S_V, 16, 1024);
+    const SDesc dP = sdesc_base(sbase + C::S_P, 16, 1024);
+    auto issue_s = [&](int it) -> bool {
+      const int stage = it % NQS;
+      if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 150)) return false;
+      tc_fence_after();
+      const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          mma_ss<false>(tmem + C::T_ST, sdesc_at(dK, off), sdesc_at(dq, off), id_s, ks > 0);
-        }
-        mma_commit(BAR(C::B_S));
-        return true;
-      };
-      auto issue_dp = [&](int it) {
-        const int stage = it % NQS;
-        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          mma_ss<false>(tmem + C::T_DPT, sdesc_at(dV, off), sdesc_at(ddo, off), id_s, ks > 0);
-        }
-        mma_commit(BAR(C::B_DP));
-      };
-      bool ok = W.wait(BAR(C::B_KV), 0, 151);
-      if (ok && n > 0) {
-        ok = issue_s(0);
-        if (ok) issue_dp(0);
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+        mma_ss_w(tmem + C::T_ST, sdesc_at(dK, off), sdesc_at(dq, off), id_s, ks > 0);
       }
-      for (int it = 0; ok && it < n; ++it) {
-        const int stage = it % NQS;
-        const uint32_t acc0 = it > 0 ? 1u : 0u;
-        ETA_TRACE_AT(tcta, 2, it, 0);
-        // S^T of the next tile once the softmax has loaded this one
-        if (it + 1 < n) {
-          if (!W.wait(BAR(C::B_SC), it & 1, 155)) { ok = false; break; }
-          if (!issue_s(it + 1)) { ok = false; break; }
-        }
-        ETA_TRACE_AT(tcta, 2, it, 1);
-        // dV += P^T dO_i: A = P^T (K-major shared memory), B = dO_i (MN-major)
-        if (!W.wait(BAR(C::B_P), it & 1, 152)) { ok = false; break; }
-        ETA_TRACE_AT(tcta, 2, it, 2);
-        tc_fence_after();
-        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, C::CHUNK, 1024);
+      mma_commit_w(BAR(C::B_S));
+      return true;
+    };
+    auto issue_dp = [&](int it) -> bool {
+      const int stage = it % NQS;
+      if (!W.wait_warp(BAR(C::B_OF + stage), (it / NQS) & 1, 156)) return false;
+      tc_fence_after();
+      const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss<false>(tmem + C::T_DV, sdesc_at(dP, (ks >> 2) * C::CHUNK + (ks & 3) * 32),
-                        sdesc_at(ddo, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-        mma_commit(BAR(C::B_PE));
-        // dK += dS^T Q_i: dS^T of query column k at dP^T column 64 (k / 64) + (k % 64) / 2
-        if (!W.wait(BAR(C::B_DS), it & 1, 153)) { ok = false; break; }
-        ETA_TRACE_AT(tcta, 2, it, 3);
-        tc_fence_after();
-        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, C::CHUNK, 1024);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ts<false>(tmem + C::T_DK, tmem + C::T_DPT + 64 * (ks >> 2) + 8 * (ks & 3),
-                        sdesc_at(dq, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-        mma_commit(BAR(C::B_QE + stage));
-        if (it + 1 < n) issue_dp(it + 1);
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
+        mma_ss_w(tmem + C::T_DPT, sdesc_at(dV, off), sdesc_at(ddo, off), id_s, ks > 0);
       }
-      if (ok) mma_commit(BAR(C::B_KVD));
-      mma_commit(BAR(C::B_DONE));
-      W.drain(BAR(C::B_DONE), 0, 154);
+      mma_commit_w(BAR(C::B_DP));
+      return true;
+    };
+    bool ok = W.wait_warp(BAR(C::B_KV), 0, 151);
+    if (ok && n > 0) ok = issue_s(0) && issue_dp(0);
+    for (int it = 0; ok && it < n; ++it) {
+      const int stage = it % NQS;
+      const uint32_t acc0 = it > 0 ? 1u : 0u;
+      ETA_TRACE_AT(tcta, 2, it, 0);
+      // S^T of the next tile once the elementwise warps have loaded this one
+      if (it + 1 < n) {
+        if (!W.wait_warp(BAR(C::B_SC), it & 1, 155)) { ok = false; break; }
+        ETA_TRACE_AT(tcta, 3, it, 1);
+        if (!issue_s(it + 1)) { ok = false; break; }
+      }
+      ETA_TRACE_AT(tcta, 2, it, 1);
+      // dV += P^T dO_i: A = P^T (K-major shared memory), B = dO_i (MN-major)
+      if (!W.wait_warp(BAR(C::B_P), it & 1, 152)) { ok = false; break; }
+      ETA_TRACE_AT(tcta, 2, it, 2);
+      tc_fence_after();
+      const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, C::CHUNK, 1024);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ss_w(tmem + C::T_DV, sdesc_at(dP, (ks >> 2) * C::CHUNK + (ks & 3) * 32),
+                 sdesc_at(ddo, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
+      mma_commit_w(BAR(C::B_PE));
+      mma_commit_w(BAR(C::B_OE + stage));  // dO_i is not read again
+      ETA_TRACE_AT(tcta, 3, it, 2);
+      // dK += dS^T Q_i with dS^T read from TMEM
+      if (!W.wait_warp(BAR(C::B_DS), it & 1, 153)) { ok = false; break; }
+      ETA_TRACE_AT(tcta, 2, it, 3);
+      tc_fence_after();
+      const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, C::CHUNK, 1024);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts_w(tmem + C::T_DK, tmem + C::T_DPT + packed_col<CW>(ks), sdesc_at(dq, ks * 2048),
+                 id_kv, ks > 0 ? 1u : acc0);
+      mma_commit_w(BAR(C::B_QE + stage));  // Q_i (and its statistics) are not read again
+      if (it + 1 < n && !issue_dp(it + 1)) { ok = false; break; }
+      ETA_TRACE_AT(tcta, 3, it, 3);
     }
+    if (ok) mma_commit_w(BAR(C::B_KVD));
+    mma_commit_w(BAR(C::B_DONE));
+    W.drain(BAR(C::B_DONE), 0, 154);
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
