@@ -15,7 +15,8 @@
 // Kernels:
 //  * bwd_preprocess_kernel: Delta = rowsum(dO * O) and lse2 = lse * log2(e)
 //    per row (rows past N padded with Delta = 0, lse2 = +inf so that their P
-//    is exactly 0), and zeroes the fp32 dQ scratch.  One warp per row.
+//    is exactly 0), and zeroes the fp32 dQ scratch (head dimension 256).
+//    D/8 threads per row.  Shared with the kernels of bwd_split.cuh.
 //  * bwd_dkdv_kernel: one CTA per (batch, key/value head, 128-row key tile,
 //    128-column slice of D); loops over the query heads of the GQA group and
 //    the 64-row query tiles (causal: only tiles at or below the diagonal).
@@ -100,47 +101,29 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------- preprocess
+// D/8 threads per row, each reading 16 bytes of O and of dO; a block of 256
+// threads covers 256 / (D/8) rows.  Rows past N get Delta = 0, lse2 = +inf.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) {
-  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  constexpr int TPR = D / 8;  // threads per row (8, 16 or 32)
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = t / TPR;  // over B * Hq * Npad
+  const int part = static_cast<int>(t % TPR);
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
-  if (warp >= rows) return;
-  const int bh = static_cast<int>(warp / p.Npad);
-  const int i = static_cast<int>(warp % p.Npad);
+  // (the launch covers exactly rows * TPR threads; the guard keeps every lane
+  // in the shuffles below either way)
+  const bool in_range = row < rows;
+  const int bh = static_cast<int>(row / p.Npad);
+  const int i = static_cast<int>(row % p.Npad);
   const int b = bh / p.Hq, h = bh % p.Hq;
-  if (i >= p.N) {
-    if (lane == 0) {
-      p.delta[warp] = 0.f;
-      p.lse2[warp] = INFINITY;
-    }
-    return;
-  }
-  constexpr int PER = D / 32;  // elements per lane (2, 4 or 8)
-  const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(p.o) + b * p.osb + h * p.osh + i * p.osn;
-  const __nv_bfloat16* drow =
-      static_cast<const __nv_bfloat16*>(p.dout) + b * p.dosb + h * p.dosh + i * p.dosn;
   float acc = 0.f;
-  if constexpr (PER == 2) {
-    const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(orow + lane * 2));
-    const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(drow + lane * 2));
-    acc = fmaf(of.x, df.x, acc);
-    acc = fmaf(of.y, df.y, acc);
-  } else if constexpr (PER == 4) {
-    const uint2 ov = *reinterpret_cast<const uint2*>(orow + lane * 4);
-    const uint2 dv = *reinterpret_cast<const uint2*>(drow + lane * 4);
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float2 of = __bfloat1622float2(o2[e]);
-      const float2 df = __bfloat1622float2(d2[e]);
-      acc = fmaf(of.x, df.x, acc);
-      acc = fmaf(of.y, df.y, acc);
-    }
-  } else {
-    const uint4 ov = *reinterpret_cast<const uint4*>(orow + lane * 8);
-    const uint4 dv = *reinterpret_cast<const uint4*>(drow + lane * 8);
+  if (in_range && i < p.N) {
+    const uint4 ov = *reinterpret_cast<const uint4*>(
+        static_cast<const __nv_bfloat16*>(p.o) + b * p.osb + h * p.osh +
+        static_cast<long long>(i) * p.osn + 8 * part);
+    const uint4 dv = *reinterpret_cast<const uint4*>(
+        static_cast<const __nv_bfloat16*>(p.dout) + b * p.dosb + h * p.dosh +
+        static_cast<long long>(i) * p.dosn + 8 * part);
     const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
@@ -150,18 +133,20 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) 
       acc = fmaf(of.x, df.x, acc);
       acc = fmaf(of.y, df.y, acc);
     }
+    // zero this part of the fp32 dQ scratch row (when dQ is accumulated there)
+    if (p.dqacc) {
+      float4* z = reinterpret_cast<float4*>(p.dqacc + (static_cast<long long>(bh) * p.N + i) * D +
+                                            8 * part);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  // zero this row of the fp32 dQ scratch (when dQ is accumulated there)
-  if (p.dqacc) {
-    float4* zrow = reinterpret_cast<float4*>(p.dqacc + (static_cast<long long>(bh) * p.N + i) * D);
-#pragma unroll
-    for (int e = lane; e < D / 4; e += 32) zrow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  if (lane == 0) {
-    p.delta[warp] = acc;
-    p.lse2[warp] = p.lse[static_cast<long long>(bh) * p.N + i] * 1.4426950408889634f;
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (in_range && part == 0) {
+    p.delta[row] = acc;
+    p.lse2[row] = i < p.N ? p.lse[static_cast<long long>(bh) * p.N + i] * 1.4426950408889634f
+                          : INFINITY;
   }
 }
 
