@@ -20,7 +20,6 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libattn.so")
 
 SOURCES = ["attn_api.cu"]
-HEADERS = ["ptx.cuh", "fwd.cuh", "fwd_fp32.cuh", "bwd.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,7 +37,8 @@ def _nvcc() -> str:
 
 
 def _inputs():
-    files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
+    headers = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
+    files = [os.path.join(CSRC, s) for s in SOURCES + headers]
     files.append(os.path.join(INCLUDE, "attn.h"))
     files.append(os.path.abspath(__file__))
     return files

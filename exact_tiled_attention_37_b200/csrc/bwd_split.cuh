@@ -82,10 +82,13 @@ struct BwdQCfg {
   static constexpr int T_S = 0, T_DP = 256, T_DQ = 384, TMEM_COLS = 512;
   static constexpr int SMEM_Q = 0, SMEM_DO = TILE, SMEM_KV = 2 * TILE;
   static constexpr int SMEM_BAR = SMEM_KV + NS * TILE;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], dp_full, ds_full, dq_done, done, dp_consumed
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], dp_full, ds_full[2], dq_done, done,
+  // dp_consumed.  ds_full alternates by key tile: a warp may arrive for tile
+  // u + 1 (it needs only dP(u) loaded by every warp, not dS(u) written)
+  // before the last warp arrives for tile u.
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS, B_DP = 3 + 2 * NS,
-                       B_DS = 4 + 2 * NS, B_DQ = 5 + 2 * NS, B_DONE = 6 + 2 * NS,
-                       B_DPC = 7 + 2 * NS, NBAR = 8 + 2 * NS;
+                       B_DS = 4 + 2 * NS, B_DQ = 6 + 2 * NS, B_DONE = 7 + 2 * NS,
+                       B_DPC = 8 + 2 * NS, NBAR = 9 + 2 * NS;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
   static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;  // warp indices
@@ -133,7 +136,8 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     mbar_init(BAR(C::B_S + 0), 1);
     mbar_init(BAR(C::B_S + 1), 1);
     mbar_init(BAR(C::B_DP), 1);
-    mbar_init(BAR(C::B_DS), 4 * NWG);
+    mbar_init(BAR(C::B_DS + 0), 4 * NWG);
+    mbar_init(BAR(C::B_DS + 1), 4 * NWG);
     mbar_init(BAR(C::B_DPC), 4 * NWG);
     mbar_init(BAR(C::B_DQ), 1);
     mbar_init(BAR(C::B_DONE), 1);
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_DS));
+      if (lane == 0) mbar_arrive(BAR(C::B_DS + (u & 1)));
       if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 3);
     }
     if (ok && n > 0 && W.wait_warp(BAR(C::B_DQ), 0, 102)) {
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       }
       ETA_FTRACE_AT(tcta, 2, u, 2);
       // dS(u) is in S[u % 2]
-      if (!W.wait_warp(BAR(C::B_DS), u & 1, 123)) { ok = false; break; }
+      if (!W.wait_warp(BAR(C::B_DS + (u & 1)), (u >> 1) & 1, 123)) { ok = false; break; }
       ETA_FTRACE_AT(tcta, 2, u, 0);
       tc_fence_after();
       // dQ += dS K_u: A = dS from TMEM, B = K_u as an MN-major operand (N = D, K = 128 keys)

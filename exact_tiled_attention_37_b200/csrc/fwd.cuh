@@ -530,16 +530,18 @@ struct SingleCfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_KV = QTILE;
   static constexpr int SMEM_BAR = SMEM_KV + NS * KTILE;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full, pv_done, o_full, done
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done, o_full, done.
+  // p_full alternates by key tile: S(j+1) is computed before P(j) is complete,
+  // so a warp may arrive for tile j + 1 before the last warp arrives for j.
   static constexpr int BAR_Q = 0;
   static constexpr int BAR_KVF = 1;
   static constexpr int BAR_KVE = 1 + NS;
   static constexpr int BAR_S = 1 + 2 * NS;
   static constexpr int BAR_P = 3 + 2 * NS;
-  static constexpr int BAR_PV = 4 + 2 * NS;
-  static constexpr int BAR_O = 5 + 2 * NS;
-  static constexpr int BAR_DONE = 6 + 2 * NS;
-  static constexpr int NBAR = 7 + 2 * NS;
+  static constexpr int BAR_PV = 5 + 2 * NS;
+  static constexpr int BAR_O = 6 + 2 * NS;
+  static constexpr int BAR_DONE = 7 + 2 * NS;
+  static constexpr int NBAR = 8 + 2 * NS;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
   static constexpr int THREADS = 256;
@@ -583,7 +585,8 @@ __global__ void __launch_bounds__(256, 1)
     }
     mbar_init(BAR(C::BAR_S + 0), 1);
     mbar_init(BAR(C::BAR_S + 1), 1);
-    mbar_init(BAR(C::BAR_P), 4);
+    mbar_init(BAR(C::BAR_P + 0), 4);
+    mbar_init(BAR(C::BAR_P + 1), 4);
     mbar_init(BAR(C::BAR_PV), 1);
     mbar_init(BAR(C::BAR_O), 1);
     mbar_init(BAR(C::BAR_DONE), 1);
@@ -628,7 +631,7 @@ __global__ void __launch_bounds__(256, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::BAR_P));
+      if (lane == 0) mbar_arrive(BAR(C::BAR_P + (j & 1)));
     }
     if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
       tc_fence_after();
@@ -705,7 +708,7 @@ __global__ void __launch_bounds__(256, 1)
           mma_commit(BAR(C::BAR_S + ((j + 1) & 1)));
           mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
         }
-        if (!W.wait(BAR(C::BAR_P), j & 1, 43)) { ok = false; break; }
+        if (!W.wait(BAR(C::BAR_P + (j & 1)), (j >> 1) & 1, 43)) { ok = false; break; }
         if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 44)) { ok = false; break; }
         tc_fence_after();
         issue_pv(j & 1, vslot(j), j > 0);
