@@ -38,6 +38,15 @@ sliding-window attention; twiscan MHA search: a 112-token local window):
 a negative bound is unbounded on that side.  ``causal`` is the same as
 ``window=(-1, 0)`` and both may be combined.
 
+Block-sparse attention, the other mask variant the pages name (FlashAttention
+(Metal Port) README, Documentation section: block sparsity as a customisation
+of the basic algorithm; FlashPrefill V2 finding on the FlashAttention entity
+page: block-sparse prefill): ``block_mask`` [B, Hq, T, T] (T = ceil(N / block))
+lets query i see key j only when ``block_mask[b, h, i // block, j // block]``
+is nonzero, on top of the causal/window mask.  A query row that sees no key
+at all has ``O = 0`` and ``lse = -inf`` (its softmax has no terms) and passes
+no gradient.
+
 Precision: every input is upcast to float64 first; numpy/OpenBLAS does the
 matrix products (a library primitive used as one step, no fusion).
 """
@@ -75,8 +84,11 @@ def _check_shapes(q, k, v):
 
 
 def _scores(q_rows: np.ndarray, k_all: np.ndarray, row_ids: np.ndarray,
-            causal: bool, scale: float, window=None) -> np.ndarray:
-    """Scaled, masked scores for the given query rows against every key."""
+            causal: bool, scale: float, window=None, block_mask=None,
+            block: int = 128) -> np.ndarray:
+    """Scaled, masked scores for the given query rows against every key.
+
+    ``block_mask``: this (batch, head)'s [T, T] tile mask, or None."""
     s = scale * (q_rows @ k_all.T)
     cols = np.arange(k_all.shape[0])[None, :]
     rows = row_ids[:, None]
@@ -88,20 +100,33 @@ def _scores(q_rows: np.ndarray, k_all: np.ndarray, row_ids: np.ndarray,
             s = np.where(cols < rows - wl, -np.inf, s)
         if wr >= 0:
             s = np.where(cols > rows + wr, -np.inf, s)
+    if block_mask is not None:
+        bm = np.asarray(block_mask) != 0
+        allowed = bm[row_ids // block][:, np.arange(k_all.shape[0]) // block]
+        s = np.where(allowed, s, -np.inf)
     return s
 
 
 def softmax_probs(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
-    """Full-row softmax of a score block; returns (P, lse) with lse natural-log."""
+    """Full-row softmax of a score block; returns (P, lse) with lse natural-log.
+
+    A row whose scores are all -inf (no visible key) gets P = 0, lse = -inf."""
     m = np.max(s, axis=1, keepdims=True)
-    e = np.exp(s - m)
+    empty = ~np.isfinite(m)
+    e = np.exp(s - np.where(empty, 0.0, m))
     z = np.sum(e, axis=1, keepdims=True)
-    p = e / z
-    lse = (m + np.log(z))[:, 0]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p = np.where(empty, 0.0, e / np.where(empty, 1.0, z))
+        lse = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, z)))[:, 0]
     return p, lse
 
 
-def attention_fwd(q, k, v, causal: bool, scale: float, window=None):
+def _bm(block_mask, b, h):
+    return None if block_mask is None else np.asarray(block_mask)[b, h]
+
+
+def attention_fwd(q, k, v, causal: bool, scale: float, window=None, block_mask=None,
+                  block: int = 128):
     """O [B,Hq,N,D] and lse [B,Hq,N] in float64 for the whole problem."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     b_, hq, hkv, n, d = _check_shapes(q, k, v)
@@ -113,14 +138,16 @@ def attention_fwd(q, k, v, causal: bool, scale: float, window=None):
             hk = h // g
             for r0 in range(0, n, _ROW_BLOCK):
                 rows = np.arange(r0, min(n, r0 + _ROW_BLOCK))
-                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale, window)
+                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale, window,
+                            _bm(block_mask, b, h), block)
                 p, l = softmax_probs(s)
                 o[b, h, rows] = p @ v[b, hk]
                 lse[b, h, rows] = l
     return o, lse
 
 
-def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows, window=None):
+def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows, window=None,
+                       block_mask=None, block: int = 128):
     """O and lse of selected query rows of one (batch, query head) only.
 
     Rows of attention are independent, so this is the same definition
@@ -133,12 +160,13 @@ def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows
     qr = _f64(q[b, h][rows])
     kk = _f64(k[b, hk])
     vv = _f64(v[b, hk])
-    s = _scores(qr, kk, rows, causal, scale, window)
+    s = _scores(qr, kk, rows, causal, scale, window, _bm(block_mask, b, h), block)
     p, l = softmax_probs(s)
     return p @ vv, l
 
 
-def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None, window=None):
+def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None, window=None,
+                  block_mask=None, block: int = 128):
     """(dQ, dK, dV) in float64 from the plain softmax Jacobian.
 
     ``heads``: optional iterable of (b, h_kv) pairs to restrict the work to
@@ -161,7 +189,8 @@ def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None, window=No
             dq_h = np.empty((n, d))
             for r0 in range(0, n, _ROW_BLOCK):
                 rows = np.arange(r0, min(n, r0 + _ROW_BLOCK))
-                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale, window)
+                s = _scores(q[b, h, rows], k[b, hk], rows, causal, scale, window,
+                            _bm(block_mask, b, h), block)
                 p, _ = softmax_probs(s)
                 dO = do[b, h, rows]
                 dv_acc += p.T @ dO

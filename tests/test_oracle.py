@@ -262,7 +262,8 @@ def _run_pins():
 def test_mutants_are_caught(monkeypatch):
     assert _run_pins() == []
 
-    def off_by_one_mask(q_rows, k_all, row_ids, causal, scale, window=None):
+    def off_by_one_mask(q_rows, k_all, row_ids, causal, scale, window=None, block_mask=None,
+                        block=128):
         s = scale * (q_rows @ k_all.T)
         if causal:
             cols = np.arange(k_all.shape[0])
@@ -270,8 +271,10 @@ def test_mutants_are_caught(monkeypatch):
             s[:, 0] = np.where(np.isinf(s[:, 0]), 0.0, s[:, 0])
         return s
 
-    def dropped_scale(q_rows, k_all, row_ids, causal, scale, window=None):
-        return oa.__dict__["_orig_scores"](q_rows, k_all, row_ids, causal, 1.0, window)
+    def dropped_scale(q_rows, k_all, row_ids, causal, scale, window=None, block_mask=None,
+                      block=128):
+        return oa.__dict__["_orig_scores"](q_rows, k_all, row_ids, causal, 1.0, window,
+                                           block_mask, block)
 
     def lse_without_max(s):
         m = np.max(s, axis=1, keepdims=True)
@@ -397,3 +400,123 @@ def test_window_backward_finite_differences(window):
                        - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
         err = np.max(np.abs(fd - g)) / max(np.max(np.abs(g)), 1e-30)
         assert err < 1e-6, (name, err)
+
+
+# ---------------------------------------------------------------- block-sparse masks
+
+
+def _brute_block(q, k, v, bm, blk, scale, causal):
+    """Explicit loops over (i, j) for one head: the block-mask definition written out."""
+    n = q.shape[0]
+    o = np.zeros_like(v)
+    lse = np.full(n, -np.inf)
+    for i in range(n):
+        js = [j for j in range(n) if bm[i // blk][j // blk] and (not causal or j <= i)]
+        if not js:
+            continue  # no visible key: O = 0, lse = -inf
+        sc = [scale * float(q[i] @ k[j]) for j in js]
+        mx = max(sc)
+        w = [math.exp(x - mx) for x in sc]
+        tot = sum(w)
+        o[i] = sum(wj * v[j] for wj, j in zip(w, js)) / tot
+        lse[i] = mx + math.log(tot)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_matches_explicit_loops(causal):
+    n, d, blk = 10, 4, 3  # 4 x 4 tiles, ragged last tile
+    q, k, v = rnd((n, d), 80), rnd((n, d), 81), rnd((n, d), 82)
+    bm = np.array([[1, 0, 1, 0], [0, 1, 0, 0], [1, 1, 0, 1], [0, 0, 0, 1]], dtype=np.uint8)
+    o, lse = oracle.attention_fwd(q[None, None], k[None, None], v[None, None], causal, 0.6,
+                                  block_mask=bm[None, None], block=blk)
+    o_b, lse_b = _brute_block(q, k, v, bm, blk, 0.6, causal)
+    np.testing.assert_allclose(o[0, 0], o_b, atol=1e-13)
+    np.testing.assert_array_equal(np.isinf(lse[0, 0]), np.isinf(lse_b))
+    fin = np.isfinite(lse_b)
+    np.testing.assert_allclose(lse[0, 0][fin], lse_b[fin], atol=1e-13)
+
+
+def test_block_mask_special_cases():
+    b, h, n, d, blk = 1, 2, 12, 5, 4
+    q, k, v = rnd((b, h, n, d), 83), rnd((b, h, n, d), 84), rnd((b, h, n, d), 85)
+    t = n // blk
+    full, lf = fwd(q, k, v, False, 0.45)
+    caus, lc = fwd(q, k, v, True, 0.45)
+    ones = np.ones((b, h, t, t), np.uint8)
+    lower = np.broadcast_to(np.tril(np.ones((t, t), np.uint8)), (b, h, t, t))
+    for causal, bm, (o_ref, l_ref) in ((False, ones, (full, lf)), (True, ones, (caus, lc)),
+                                       (True, lower, (caus, lc))):
+        o, l = oracle.attention_fwd(q, k, v, causal, 0.45, block_mask=bm, block=blk)
+        np.testing.assert_allclose(o, o_ref, atol=1e-13)
+        np.testing.assert_allclose(l, l_ref, atol=1e-13)
+    # block-diagonal mask = independent attention on each tile of rows
+    diag = np.broadcast_to(np.eye(t, dtype=np.uint8), (b, h, t, t))
+    o, l = oracle.attention_fwd(q, k, v, False, 0.45, block_mask=diag, block=blk)
+    for s in range(t):
+        sl = slice(s * blk, (s + 1) * blk)
+        o_s, l_s = fwd(q[:, :, sl], k[:, :, sl], v[:, :, sl], False, 0.45)
+        np.testing.assert_allclose(o[:, :, sl], o_s, atol=1e-13)
+        np.testing.assert_allclose(l[:, :, sl], l_s, atol=1e-13)
+
+
+def test_block_mask_empty_rows():
+    # query tile 1 sees no key tile: O = 0, lse = -inf, no gradient through it
+    b, h, n, d, blk = 1, 1, 8, 3, 4
+    q, k, v, do = (rnd((b, h, n, d), s) for s in (86, 87, 88, 89))
+    bm = np.array([[[[1, 1], [0, 0]]]], np.uint8)
+    o, l = oracle.attention_fwd(q, k, v, False, 0.5, block_mask=bm, block=blk)
+    assert np.all(o[0, 0, 4:] == 0.0) and np.all(l[0, 0, 4:] == -np.inf)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, False, 0.5, block_mask=bm, block=blk)
+    assert np.all(dq[0, 0, 4:] == 0.0)
+    # the other rows are plain attention over all keys, unaffected by dO of empty rows
+    do2 = do.copy()
+    do2[0, 0, 4:] = 17.0
+    dq2, dk2, dv2 = oracle.attention_bwd(q, k, v, do2, False, 0.5, block_mask=bm, block=blk)
+    np.testing.assert_allclose(dk2, dk, atol=1e-14)
+    np.testing.assert_allclose(dv2, dv, atol=1e-14)
+    o_full, _ = fwd(q, k, v, False, 0.5)
+    np.testing.assert_allclose(o[0, 0, :4], o_full[0, 0, :4], atol=1e-13)
+
+
+def test_block_mask_backward_finite_differences():
+    n, d, scale, h, blk = 6, 3, 0.8, 1e-6, 2
+    q, k, v, do = (rnd((1, 2, n, d), s) for s in (90, 91, 92, 93))
+    k, v = k[:, :1], v[:, :1]
+    bm = np.array([[[[1, 0, 1], [1, 1, 0], [0, 1, 1]], [[0, 1, 0], [1, 0, 1], [1, 1, 1]]]],
+                  np.uint8)
+    kw = dict(block_mask=bm, block=blk)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, False, scale, **kw)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.attention_fwd(qq, kk, vv, False, scale, **kw)
+        return float(np.sum(o * do))
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = {"q": q, "k": k, "v": v}
+            args_p[name], args_m[name] = xp, xm
+            fd[idx] = (loss(args_p["q"], args_p["k"], args_p["v"])
+                       - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
+        err = np.max(np.abs(fd - g)) / max(np.max(np.abs(g)), 1e-30)
+        assert err < 1e-6, (name, err)
+
+
+def test_block_mask_transposed_mutant_is_caught(monkeypatch):
+    orig = oa._scores
+
+    def transposed(q_rows, k_all, row_ids, causal, scale, window=None, block_mask=None,
+                   block=128):
+        bm = None if block_mask is None else np.asarray(block_mask).T
+        return orig(q_rows, k_all, row_ids, causal, scale, window, bm, block)
+
+    monkeypatch.setattr(oa, "_scores", transposed)
+    with pytest.raises(AssertionError):
+        test_block_mask_matches_explicit_loops(False)
