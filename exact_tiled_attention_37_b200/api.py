@@ -52,12 +52,27 @@ def _window(causal: bool, window) -> tuple[int, int]:
     return wl, wr
 
 
+def _block_mask(block_mask, B, Hq, N, device) -> ctypes.c_void_p:
+    """Device pointer of a [B, Hq, T, T] uint8 tile mask (T = ceil(N / 128)), or NULL."""
+    if block_mask is None:
+        return ctypes.c_void_p(0)
+    t = (N + 127) // 128
+    if (block_mask.dtype != torch.uint8 or not block_mask.is_cuda
+            or block_mask.device != device or tuple(block_mask.shape) != (B, Hq, t, t)
+            or not block_mask.is_contiguous()):
+        raise ValueError(f"block_mask must be a contiguous uint8 CUDA tensor of shape "
+                         f"{(B, Hq, t, t)} on {device}")
+    return ctypes.c_void_p(block_mask.data_ptr())
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              scale: float | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, window=None):
+             lse: torch.Tensor | None = None, window=None, block_mask=None):
     """O, lse = attention(q, k, v): q [B,Hq,N,D], k/v [B,Hkv,N,D] on one CUDA device.
 
     window=(wl, wr): query i sees keys i - wl .. i + wr (-1 = unbounded side).
+    block_mask: [B,Hq,T,T] uint8 (T = ceil(N/128)); 128x128 tile pairs whose
+    entry is 0 are skipped (rows that see no key get O = 0, lse = -inf).
     Returns O (dtype of q) and lse [B,Hq,N] fp32 (natural log).
     """
     B, Hq, N, D = q.shape
@@ -76,9 +91,10 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
         raise ValueError("lse must be a contiguous fp32 [B, Hq, N] tensor")
     L = _lib.lib()
     wl, wr = _window(causal, window)
-    code = L.attn_fwd_window(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(out, "out"),
+    bm = _block_mask(block_mask, B, Hq, N, q.device)
+    code = L.attn_fwd_masked(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(out, "out"),
                              ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, N, D, _dtype_code(q),
-                             wl, wr, float(scale), _stream(q.device))
+                             wl, wr, bm, float(scale), _stream(q.device))
     _check(code, "attn_fwd")
     return out, lse
 
@@ -88,8 +104,10 @@ def bwd_workspace_bytes(B: int, Hq: int, N: int, D: int) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
-             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, window=None):
-    """dQ, dK, dV of attention from the forward's O and lse and the gradient dO."""
+             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, window=None,
+             block_mask=None):
+    """dQ, dK, dV of attention from the forward's O and lse and the gradient dO
+    (window and block_mask as in attn_fwd)."""
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
     if scale is None:
@@ -109,10 +127,11 @@ def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     if not lse.is_contiguous() or lse.dtype != torch.float32:
         raise ValueError("lse must be contiguous fp32")
     wl, wr = _window(causal, window)
-    code = L.attn_bwd_window(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(o, "o"),
+    bm = _block_mask(block_mask, B, Hq, N, q.device)
+    code = L.attn_bwd_masked(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(o, "o"),
                              ctypes.c_void_p(lse.data_ptr()), _desc(do, "do"), _desc(dq, "dq"),
                              _desc(dk, "dk"), _desc(dv, "dv"), B, Hq, Hkv, N, D,
-                             _dtype_code(q), wl, wr, float(scale),
+                             _dtype_code(q), wl, wr, bm, float(scale),
                              ctypes.c_void_p(workspace.data_ptr()),
                              ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                              _stream(q.device))

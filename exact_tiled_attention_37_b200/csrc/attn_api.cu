@@ -121,6 +121,13 @@ attn_status_t set_smem(Kernel k, int bytes) {
   return ATTN_OK;
 }
 
+template <typename Kernel>
+int kernel_regs(Kernel k) {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return -1;
+  return fa.numRegs;
+}
+
 attn_status_t last_launch() {
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -136,7 +143,13 @@ attn_status_t launch_pingpong(const attn_tensor_t& q, const attn_tensor_t& k,
   if ((s = make_map(&tq, q, B, Hq, N, D, sizeof(T), 128)) != ATTN_OK) return s;
   if ((s = make_map(&tk, k, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
   if ((s = make_map(&tv, v, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
-  auto kern = eta::fwd_pingpong_kernel<T, D, NS>;
+  auto kern = p.bmask ? eta::fwd_pingpong_kernel<T, D, NS, true>
+                      : eta::fwd_pingpong_kernel<T, D, NS, false>;
+  // The kernel moves registers between its warpgroups on the assumption that
+  // it was launched with C::LAUNCH_REGS per thread; never launch otherwise.
+  static const int regs[2] = {kernel_regs(eta::fwd_pingpong_kernel<T, D, NS, false>),
+                              kernel_regs(eta::fwd_pingpong_kernel<T, D, NS, true>)};
+  if (regs[p.bmask ? 1 : 0] != C::LAUNCH_REGS) return ATTN_ERR_CUDA;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
   dim3 grid(Hq, B, (N + 255) / 256);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
@@ -317,6 +330,14 @@ attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
                               float* lse, int B, int Hq, int Hkv, int N, int D,
                               attn_dtype_t dtype, int window_left, int window_right, float scale,
                               void* stream) {
+  return attn_fwd_masked(q, k, v, o, lse, B, Hq, Hkv, N, D, dtype, window_left, window_right,
+                         nullptr, scale, stream);
+}
+
+attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                              float* lse, int B, int Hq, int Hkv, int N, int D,
+                              attn_dtype_t dtype, int window_left, int window_right,
+                              const uint8_t* block_mask, float scale, void* stream) {
   attn_status_t s;
   if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
   if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
@@ -325,6 +346,10 @@ attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
   const bool bf16 = dtype == ATTN_BF16;
   if (bf16 ? !(D == 64 || D == 128 || D == 256) : D != 64) return ATTN_ERR_UNSUPPORTED;
+  if (block_mask) {
+    // block-sparse tiles: bf16 with D <= 128 and at most kMaxMaskTiles tiles
+    if (!bf16 || D > 128 || (N + 127) / 128 > eta::kMaxMaskTiles) return ATTN_ERR_UNSUPPORTED;
+  }
   const int es = bf16 ? 2 : 4;
   if ((s = check_tensor(q, B, Hq, N, es)) != ATTN_OK) return s;
   if ((s = check_tensor(k, B, Hkv, N, es)) != ATTN_OK) return s;
@@ -348,6 +373,8 @@ attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
   p.wait_limit_ns = g_wait_limit_ns.load();
   p.debug_flags = g_debug_flags.load();
+  p.bmask = block_mask;
+  p.nt = (N + 127) / 128;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!bf16) {
@@ -384,6 +411,16 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
                               int D, attn_dtype_t dtype, int window_left, int window_right,
                               float scale, void* workspace, size_t workspace_bytes,
                               void* stream) {
+  return attn_bwd_masked(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, dtype, window_left,
+                         window_right, nullptr, scale, workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                              const float* lse, attn_tensor_t dout, attn_tensor_t dq,
+                              attn_tensor_t dk, attn_tensor_t dv, int B, int Hq, int Hkv, int N,
+                              int D, attn_dtype_t dtype, int window_left, int window_right,
+                              const uint8_t* block_mask, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
   attn_status_t s;
   if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
   if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
@@ -391,6 +428,7 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
   if (!(D == 64 || D == 128 || D == 256)) return ATTN_ERR_UNSUPPORTED;
+  if (block_mask && (D > 128 || (N + 127) / 128 > eta::kMaxMaskTiles)) return ATTN_ERR_UNSUPPORTED;
   const int es = 2;
   const attn_tensor_t* qs[] = {&q, &o, &dout, &dq};
   for (auto* t : qs)
@@ -427,6 +465,8 @@ attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
   p.wait_limit_ns = g_wait_limit_ns.load();
+  p.bmask = block_mask;
+  p.nt = (N + 127) / 128;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // per head dimension: Q/dO stages of the dK/dV kernel, K/V ring slots of
   // the dQ kernel, elementwise warpgroups (measured best on B200)

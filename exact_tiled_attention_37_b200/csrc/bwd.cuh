@@ -98,6 +98,8 @@ struct BwdParams {
   float scale, c;       // c = scale * log2(e)
   int* status;
   unsigned long long wait_limit_ns;
+  const uint8_t* bmask; // block-sparse tile mask [B, Hq, nt, nt] or null (D <= 128 only)
+  int nt;               // ceil(N / 128)
 };
 
 // ---------------------------------------------------------------- preprocess
@@ -145,8 +147,10 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) 
   for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (in_range && part == 0) {
     p.delta[row] = acc;
-    p.lse2[row] = i < p.N ? p.lse[static_cast<long long>(bh) * p.N + i] * 1.4426950408889634f
-                          : INFINITY;
+    // rows past N, and rows that saw no key (lse = -inf), get lse2 = +inf so
+    // that their P is exactly 0
+    const float l = i < p.N ? p.lse[static_cast<long long>(bh) * p.N + i] : -INFINITY;
+    p.lse2[row] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
   }
 }
 

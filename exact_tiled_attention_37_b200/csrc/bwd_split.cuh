@@ -90,7 +90,8 @@ struct BwdQCfg {
                        B_DS = 4 + 2 * NS, B_DQ = 6 + 2 * NS, B_DONE = 7 + 2 * NS,
                        B_DPC = 8 + 2 * NS, NBAR = 9 + 2 * NS;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
-  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
+  static constexpr int SMEM_BITS = SMEM_MISC + 16;  // block-sparse: computed key tiles
+  static constexpr int SMEM_BYTES = SMEM_BITS + 4 * kMaskWords + 1024;
   static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;  // warp indices
   static constexpr int THREADS = 128 * NWG + 64;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -119,7 +120,24 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   const int hk = h / p.group;
   const int q0 = qb * C::BM;
   const int2 ktr = key_tiles(q0, p.N, p.wl, p.wr, C::BN);
-  const int j0 = ktr.x, n = ktr.y - ktr.x;  // key tiles j0 .. j0 + n - 1
+  const int jlo = ktr.x, jhi = ktr.y;  // key tiles in the window range
+  // Block-sparse: bit j marks key tile j as computed for this query tile.
+  const bool sparse = p.bmask != nullptr;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::SMEM_BITS);
+  if (sparse) {
+    for (int wi = warp; wi < kMaskWords; wi += C::THREADS / 32) {
+      const int j = 32 * wi + lane;
+      const bool on = j >= jlo && j < jhi && qb < p.nt &&
+                      p.bmask[((static_cast<long long>(b) * p.Hq + h) * p.nt + qb) * p.nt + j] != 0;
+      const uint32_t w = __ballot_sync(0xffffffffu, on);
+      if (lane == 0) bits[wi] = w;
+    }
+  }
+  // first computed key tile >= j (jhi if none)
+  auto next_key = [&](int j) -> int {
+    j = max(j, jlo);
+    return sparse ? next_bit(bits, j, jhi) : min(j, jhi);
+  };
 #ifdef ETA_TRACE
   const int tcta = (blockIdx.x == 0 && blockIdx.y == 0) ? (qb == 31 ? 0 : (qb == 15 ? 1 : -1)) : -1;
 #else
@@ -154,6 +172,8 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+  // computed key tiles, in increasing order: iteration u handles the u-th
+  const int n = sparse ? bits_below(bits, jhi) : jhi - jlo;
 
   if (warp < 4 * NWG) {
     // ---------------------------------------- dS rows (thread r = query row r), then dQ
@@ -165,7 +185,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     const float lse2 = p.lse2[srow];       // +inf for padded rows: their P is exactly 0
     const float dlt = p.delta[srow];
     bool ok = true;
-    for (int u = 0; u < n; ++u) {
+    for (int u = 0, j = next_key(jlo); u < n; ++u, j = next_key(j + 1)) {
       const int buf = u & 1;
       const uint32_t s_addr = tmem + lane_base + C::T_S + 128 * buf + CW * par;
       if (!W.wait_warp(BAR(C::B_S + buf), (u >> 1) & 1, 100)) { ok = false; break; }
@@ -173,7 +193,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       tc_fence_after();
       float s[CW];
       tmem_load_row<CW>(s_addr, s);
-      const int2 cw = col_window(C::BN * (j0 + u) + CW * par, qrow, p.N, p.wl, p.wr);
+      const int2 cw = col_window(C::BN * j + CW * par, qrow, p.N, p.wl, p.wr);
       const float2 c2 = make_float2(p.c, p.c), nl2 = make_float2(-lse2, -lse2);
       if (cw.x <= 0 && cw.y >= CW) {
 #pragma unroll
@@ -214,13 +234,16 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       if (lane == 0) mbar_arrive(BAR(C::B_DS + (u & 1)));
       if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 3);
     }
+    // dQ * scale in bf16: warpgroup par stores columns [D/NWG par, D/NWG (par + 1))
+    constexpr int DC = D / NWG;
+    __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.dq) + b * p.dqsb + h * p.dqsh +
+                         static_cast<long long>(qrow) * p.dqsn + DC * par;
     if (ok && n > 0 && W.wait_warp(BAR(C::B_DQ), 0, 102)) {
       tc_fence_after();
-      // dQ * scale in bf16: warpgroup par stores columns [D/NWG par, D/NWG (par + 1))
-      constexpr int DC = D / NWG;
-      __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.dq) + b * p.dqsb + h * p.dqsh +
-                           static_cast<long long>(qrow) * p.dqsn + DC * par;
       tmem_row_to_bf16<DC>(tmem + lane_base + C::T_DQ + DC * par, row, p.scale, qrow < p.N);
+    } else if (n == 0 && qrow < p.N) {
+      // no key tile is computed for this query tile: dQ = 0
+      for (int c = 0; c < DC / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
     }
   } else if (warp == C::PRODUCER) {
     // ---------------------------------------- TMA producer
@@ -235,14 +258,14 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         tma_load_4d(sbase + C::SMEM_DO + c * C::CHUNK, &tm_do, BAR(C::B_Q), c * 64, q0, h, b);
       }
       int it = 0;
-      for (int u = 0; u < n && !W.aborted(); ++u) {
+      for (int u = 0, j = next_key(jlo); u < n && !W.aborted(); ++u, j = next_key(j + 1)) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = it % C::NS;
           if (!W.wait(BAR(C::B_KVE + slot), (static_cast<uint32_t>(it / C::NS) & 1u) ^ 1u, 110)) break;
           mbar_expect_tx(BAR(C::B_KVF + slot), C::TILE);
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_4d(sbase + C::SMEM_KV + slot * C::TILE + c * C::CHUNK, kv ? &tm_v : &tm_k,
-                        BAR(C::B_KVF + slot), c * 64, C::BN * (j0 + u), hk, b);
+                        BAR(C::B_KVF + slot), c * 64, C::BN * j, hk, b);
         }
       }
       const int issued = it;
@@ -361,13 +384,16 @@ struct BwdKVCfg {
                        B_DS = 6 + 4 * NQS, B_KVD = 7 + 4 * NQS, B_DONE = 8 + 4 * NQS,
                        NBAR = 9 + 4 * NQS;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
-  static constexpr int LAYOUT = S_MISC + 16;
+  static constexpr int S_META = S_MISC + 16;   // [NQS] entry index of each stage
+  static constexpr int S_CNT = S_META + 16;    // number of computed entries
+  static constexpr int LAYOUT = S_CNT + 16;
   // dynamic shared memory: the layout plus as much of the 1024-byte alignment
   // slack as the per-block limit leaves (the kernel checks the actual slack)
   static constexpr int SMEM_BYTES = LAYOUT + 1024 <= 232448 ? LAYOUT + 1024 : 232448;
   static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;  // warp indices
   static constexpr int THREADS = 128 * NWG + 64;
   static_assert(LAYOUT <= 232448, "shared memory budget");
+  static_assert(NQS <= 4, "stage metadata slots");
   static_assert(NWG % 2 == 0 && D % (8 * NWG) == 0, "dK/dV columns per warpgroup");
 };
 
@@ -402,9 +428,19 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   const int q_hi = p.wl < 0 ? p.N : min(p.N, min(p.N, k0 + C::BC) + p.wl);
   const int i_first = q_lo / C::BR;
   const int per_head = (q_hi + C::BR - 1) / C::BR - i_first;
-  const int n = per_head * p.group;  // iterations: query heads of the group x query tiles
-  auto head_of = [&](int it) { return hk * p.group + it / per_head; };
-  auto qtile_of = [&](int it) { return i_first + it % per_head; };
+  // entries: query heads of the group x query tiles in the window range, in
+  // that order; with a block-sparse mask only the entries whose tile pair is
+  // marked are computed
+  const int E = per_head * p.group;
+  const bool sparse = p.bmask != nullptr;
+  auto head_of = [&](int e) { return hk * p.group + e / per_head; };
+  auto qtile_of = [&](int e) { return i_first + e % per_head; };
+  auto marked = [&](int e) -> bool {
+    return p.bmask[((static_cast<long long>(b) * p.Hq + head_of(e)) * p.nt + qtile_of(e)) * p.nt +
+                   kt] != 0;
+  };
+  volatile int* meta = reinterpret_cast<volatile int*>(smem + C::S_META);
+  int* cnt_smem = reinterpret_cast<int*>(smem + C::S_CNT);
 #ifdef ETA_TRACE
   const int tcta = (blockIdx.x == 0 && blockIdx.y == 0) ? (kt == 0 ? 0 : (kt == 16 ? 1 : -1)) : -1;
 #else
@@ -429,6 +465,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     mbar_init(BAR(C::B_KVD), 1);
     mbar_init(BAR(C::B_DONE), 1);
     *abort_flag = 0u;
+    *cnt_smem = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -441,6 +478,14 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+  int n = E;  // iterations: computed entries
+  if (sparse) {
+    int c = 0;
+    for (int e = threadIdx.x; e < E; e += C::THREADS) c += marked(e) ? 1 : 0;
+    if (c) atomicAdd(cnt_smem, c);
+    __syncthreads();
+    n = *cnt_smem;
+  }
 
   if (warp < 4 * NWG) {
     // ---------------------------------------- P^T, dS^T rows (thread j = key row j)
@@ -459,6 +504,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     for (int it = 0; it < n; ++it) {
       const int stage = it % NQS;
       if (!W.wait_warp(BAR(C::B_S), it & 1, 130)) { ok = false; break; }
+      // (complete already: S^T was computed from this stage) orders the reads of
+      // the stage's entry index and row statistics after the producer's writes
+      if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 134)) { ok = false; break; }
       if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 0);
       tc_fence_after();
       float pr[CW];
@@ -469,7 +517,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       const float* lse2 =
           reinterpret_cast<const float*>(smem + C::S_STAT + stage * 1024) + CW * par;
       const float* dlt = lse2 + 128;
-      const int ig0 = qtile_of(it) * C::BR + CW * par;
+      const int ig0 = qtile_of(meta[stage]) * C::BR + CW * par;
       // window: query ig0 + i sees key jg iff jg - wr <= ig0 + i <= jg + wl
       const int ilo = p.wr < 0 ? -(1 << 30) : jg - p.wr - ig0;
       const int ihi = p.wl < 0 ? (1 << 30) : jg + p.wl - ig0;
@@ -550,7 +598,8 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       for (int c = 0; c < DC / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
     }
   } else if (warp == C::PRODUCER) {
-    // ---------------------------------------- TMA producer
+    // ---------------------------------------- TMA producer (the whole warp scans
+    // 32 entries at a time; lane 0 waits and issues the copies)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -561,34 +610,58 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         tma_load_4d(sbase + C::S_K + c * C::CHUNK, &tm_k, BAR(C::B_KV), c * 64, k0, hk, b);
         tma_load_4d(sbase + C::S_V + c * C::CHUNK, &tm_v, BAR(C::B_KV), c * 64, k0, hk, b);
       }
-      // dO_i and Q_i have their own barriers: dO_i's slot frees earlier (after
-      // dV) and is refilled first; Q_i (needed first, by S^T) follows.
-      int it = 0, issued_do = 0;
-      for (; it < n; ++it) {
-        const int stage = it % NQS;
-        const uint32_t par_empty = ((it / NQS) & 1) ^ 1;
-        const int h = head_of(it);
-        const int ig0 = qtile_of(it) * C::BR;
-        if (!W.wait(BAR(C::B_OE + stage), par_empty, 143)) break;
-        const uint32_t ofull = BAR(C::B_OF + stage);
-        mbar_expect_tx(ofull, C::TILE);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sbase + C::S_DO + stage * C::TILE + c * C::CHUNK, &tm_do, ofull, c * 64, ig0, h, b);
-        issued_do = it + 1;
-        if (!W.wait(BAR(C::B_QE + stage), par_empty, 140)) break;
-        ETA_TRACE_AT(tcta, 3, it, 0);
-        const uint32_t full = BAR(C::B_QF + stage);
-        mbar_expect_tx(full, C::TILE + 1024);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full, c * 64, ig0, h, b);
-        const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
-        bulk_load(sbase + C::S_STAT + stage * 1024, p.lse2 + srow, 512, full);
-        bulk_load(sbase + C::S_STAT + stage * 1024 + 512, p.delta + srow, 512, full);
+    }
+    // dO_i and Q_i have their own barriers: dO_i's slot frees earlier (after
+    // dV) and is refilled first; Q_i (needed first, by S^T) follows.
+    int it = 0, issued_q = 0, issued_do = 0;
+    bool pok = true;
+    for (int base = 0; pok && it < n && base < E; base += 32) {
+      const int e_l = base + lane;
+      const bool on = e_l < E && (!sparse || marked(e_l));
+      uint32_t pend = __ballot_sync(0xffffffffu, on);
+      while (pend != 0u && it < n) {
+        const int e = base + __ffs(pend) - 1;
+        pend &= pend - 1u;
+        if (lane == 0) {
+          const int stage = it % NQS;
+          const uint32_t par_empty = ((it / NQS) & 1) ^ 1;
+          const int h = head_of(e);
+          const int ig0 = qtile_of(e) * C::BR;
+          if (!W.wait(BAR(C::B_OE + stage), par_empty, 143)) {
+            pok = false;
+          } else {
+            const uint32_t ofull = BAR(C::B_OF + stage);
+            mbar_expect_tx(ofull, C::TILE);
+            for (int c = 0; c < C::NCHUNK; ++c)
+              tma_load_4d(sbase + C::S_DO + stage * C::TILE + c * C::CHUNK, &tm_do, ofull, c * 64,
+                          ig0, h, b);
+            issued_do = it + 1;
+            if (!W.wait(BAR(C::B_QE + stage), par_empty, 140)) {
+              pok = false;
+            } else {
+              ETA_TRACE_AT(tcta, 3, it, 0);
+              meta[stage] = e;
+              const uint32_t full = BAR(C::B_QF + stage);
+              mbar_expect_tx(full, C::TILE + 1024);
+              for (int c = 0; c < C::NCHUNK; ++c)
+                tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full, c * 64,
+                            ig0, h, b);
+              const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
+              bulk_load(sbase + C::S_STAT + stage * 1024, p.lse2 + srow, 512, full);
+              bulk_load(sbase + C::S_STAT + stage * 1024 + 512, p.delta + srow, 512, full);
+              issued_q = it + 1;
+            }
+          }
+        }
+        pok = __shfl_sync(0xffffffffu, pok, 0);
+        if (!pok) break;
+        ++it;
       }
+    }
+    if (lane == 0) {
       W.drain(BAR(C::B_KV), 0, 141);
-      const int issued = it;
-      for (int s = 0; s < NQS && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / NQS) * NQS;
+      for (int s = 0; s < NQS && s < issued_q; ++s) {
+        const int last = s + ((issued_q - 1 - s) / NQS) * NQS;
         W.drain(BAR(C::B_QF + s), static_cast<uint32_t>(last / NQS) & 1u, 142);
       }
       for (int s = 0; s < NQS && s < issued_do; ++s) {

@@ -67,7 +67,34 @@ struct FwdParams {
   int* status;       // device status word (4 ints)
   unsigned long long wait_limit_ns;
   int debug_flags;   // bit 0: producer skips the first V tile (timeout test)
+  // block-sparse tile mask [B, Hq, nt, nt] (nonzero = the 128 x 128 tile pair is
+  // computed), or null; nt = ceil(N / 128) <= kMaxMaskTiles
+  const uint8_t* bmask;
+  int nt;
 };
+
+// Longest sequence (in 128-row tiles) a block-sparse mask may describe: the
+// kernels keep one bit per key tile of a query tile in shared memory.
+constexpr int kMaxMaskTiles = 512;
+constexpr int kMaskWords = kMaxMaskTiles / 32;
+
+// Number of set bits of w[] below bit j.
+__device__ __forceinline__ int bits_below(const uint32_t* w, int j) {
+  int c = 0;
+  for (int i = 0; i < (j >> 5); ++i) c += __popc(w[i]);
+  if (j & 31) c += __popc(w[j >> 5] & ((1u << (j & 31)) - 1u));
+  return c;
+}
+
+// Smallest set bit of w[] at or after j, or `end` (bits at or beyond `end` ignored).
+__device__ __forceinline__ int next_bit(const uint32_t* w, int j, int end) {
+  while (j < end) {
+    const uint32_t x = w[j >> 5] >> (j & 31);
+    if (x) return min(end, j + __ffs(x) - 1);
+    j = (j | 31) + 1;
+  }
+  return end;
+}
 
 // Online-softmax update of one row over one tile of BC scores (already masked
 // to -inf where not allowed).  m is the running maximum in raw score units,
@@ -180,7 +207,7 @@ template <typename T, int D>
 __device__ __forceinline__ void store_row(uint32_t o_taddr, const FwdParams& p, int b, int h,
                                           int qrow, float m, float l) {
   const bool valid = qrow < p.N;
-  const float inv_l = 1.f / l;
+  const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no visible key stores O = 0
   char* row = static_cast<char*>(p.o) +
               (static_cast<long long>(b) * p.osb + static_cast<long long>(h) * p.osh +
                static_cast<long long>(qrow) * p.osn) *
@@ -212,7 +239,21 @@ __device__ __forceinline__ void store_row(uint32_t o_taddr, const FwdParams& p, 
     }
   }
   if (valid)
-    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = m * p.scale + logf(l);
+    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] =
+        l > 0.f ? m * p.scale + logf(l) : -INFINITY;
+}
+
+// Epilogue of a row whose query tile computed no key tile: O = 0, lse = -inf.
+template <typename T, int D>
+__device__ __forceinline__ void store_empty_row(const FwdParams& p, int b, int h, int qrow) {
+  if (qrow >= p.N) return;
+  char* row = static_cast<char*>(p.o) +
+              (static_cast<long long>(b) * p.osb + static_cast<long long>(h) * p.osh +
+               static_cast<long long>(qrow) * p.osn) *
+                  static_cast<long long>(sizeof(T));
+  for (int i = 0; i < D * static_cast<int>(sizeof(T)) / 16; ++i)
+    reinterpret_cast<uint4*>(row)[i] = make_uint4(0u, 0u, 0u, 0u);
+  p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = -INFINITY;
 }
 
 // Keys [lo, hi) that query rows [qs, qe) may see under the window (wl, wr)
@@ -277,8 +318,14 @@ struct PingPongCfg {
   static constexpr int BAR_DONE = 7 + 2 * NS;
   static constexpr int NBAR = 8 + 2 * NS;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;  // tmem slot, abort flag
-  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int SMEM_BITS = SMEM_MISC + 16;        // [2][kMaskWords] used-tile bits
+  static constexpr int SMEM_BYTES = SMEM_BITS + 8 * kMaskWords + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
+  // registers per thread: at launch (what the compiler allocates under
+  // __launch_bounds__(384, 1); the host checks it before launching), then
+  // moved to the softmax warpgroups, away from the producer/MMA warpgroup
+  static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, OTHER_REGS = 72;
+  static_assert(THREADS * LAUNCH_REGS == 256 * SOFTMAX_REGS + 128 * OTHER_REGS, "register split");
   // bf16 only: tf32 products would keep 10 mantissa bits, which misses the
   // logsumexp tolerance; fp32 storage goes through fwd_fp32_kernel.
   static_assert(sizeof(T) == 2, "bf16 storage");
@@ -287,7 +334,9 @@ struct PingPongCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <typename T, int D, int NS>
+// SPARSE: built for a block-sparse tile mask (p.bmask); the dense build
+// carries none of the mask bookkeeping.
+template <typename T, int D, int NS, bool SPARSE>
 __global__ void __launch_bounds__(384, 1)
     fwd_pingpong_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -309,18 +358,50 @@ __global__ void __launch_bounds__(384, 1)
   const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / p.group;
   const int q0 = qb * 256;
-  // key tiles [jlo[t], jhi[t]) of each query tile; tile 0's range never starts
+  // key tiles [jlo(t), jhi(t)) of each query tile; tile 0's range never starts
   // or ends after tile 1's, so tile 1 (when it has work) is the last reader of
   // every K/V tile it uses
-  int jlo[2], jhi[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int2 r = key_tiles(q0 + 128 * t, p.N, p.wl, p.wr, 128);
-    jlo[t] = r.x;
-    jhi[t] = r.y;
+  // (scalars, selected by t, so that they stay in registers)
+  const int2 kr0 = key_tiles(q0, p.N, p.wl, p.wr, 128);
+  const int2 kr1 = key_tiles(q0 + 128, p.N, p.wl, p.wr, 128);
+  auto jlo = [&](int t) { return t ? kr1.x : kr0.x; };
+  auto jhi = [&](int t) { return t ? kr1.y : kr0.y; };
+  const bool has1 = kr1.y > kr1.x;
+  const int jmin = kr0.x, jmax = has1 ? kr1.y : kr0.y;
+  // Block-sparse: bit j of bits[t] marks key tile j as computed by query tile t.
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::SMEM_BITS);
+  if constexpr (SPARSE) {
+    for (int wi = warp; wi < 2 * kMaskWords; wi += C::THREADS / 32) {
+      const int t = wi / kMaskWords, j = 32 * (wi % kMaskWords) + lane;
+      const int qt = 2 * qb + t;
+      const bool on = j >= jlo(t) && j < jhi(t) && qt < p.nt &&
+                      p.bmask[((static_cast<long long>(b) * p.Hq + h) * p.nt + qt) * p.nt + j] != 0;
+      const uint32_t w = __ballot_sync(0xffffffffu, on);
+      if (lane == 0) bits[wi] = w;
+    }
   }
-  const bool has1 = jhi[1] > jlo[1];
-  const int jmin = jlo[0], jmax = has1 ? jhi[1] : jhi[0];
+  // key tile j computed by query tile t
+  auto uses = [&](int t, int j) -> bool {
+    if (j < jlo(t) || j >= jhi(t)) return false;
+    if constexpr (!SPARSE) return true;
+    return (bits[t * kMaskWords + (j >> 5)] >> (j & 31)) & 1u;
+  };
+  // first key tile >= j computed by query tile t (jhi(t) if none)
+  auto next_use = [&](int t, int j) -> int {
+    j = max(j, jlo(t));
+    if constexpr (!SPARSE) return min(j, jhi(t));
+    return next_bit(bits + t * kMaskWords, j, jhi(t));
+  };
+  auto in_union = [&](int j) -> bool { return uses(0, j) || uses(1, j); };
+  // first key tile >= j that either query tile computes (jmax if none)
+  auto next_union = [&](int j) -> int {
+    if constexpr (!SPARSE) {
+      for (; j < jmax; ++j)
+        if (in_union(j)) return j;
+      return jmax;
+    }
+    return min(next_use(0, j), next_use(1, j));
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::BAR_Q), 1);
@@ -354,6 +435,13 @@ __global__ void __launch_bounds__(384, 1)
 #endif
   (void)tcta;
 
+  // Registers: the softmax warpgroups hold a 128-float score row; the
+  // producer/MMA warpgroup needs few (no spills in either role).
+  if (warp < 8) {
+    setmaxnreg_inc<C::SOFTMAX_REGS>();
+  } else {
+    setmaxnreg_dec<C::OTHER_REGS>();
+  }
   if (warp < 8) {
     // ------------------------------------------------ softmax / correction / epilogue
     const int t = warp >> 2;
@@ -364,8 +452,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = jlo[t]; j < jhi[t]; ++j) {
-      if (!W.wait_warp(BAR(C::BAR_S + t), (j - jlo[t]) & 1, 10 + t)) { ok = false; break; }
+    int cnt = 0;  // key tiles of this query tile done so far
+    for (int j = next_use(t, jlo(t)); j < jhi(t); j = next_use(t, j + 1), ++cnt) {
+      if (!W.wait_warp(BAR(C::BAR_S + t), cnt & 1, 10 + t)) { ok = false; break; }
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 0);
       tc_fence_after();
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 1);
@@ -379,14 +468,16 @@ __global__ void __launch_bounds__(384, 1)
       const bool rescaled = online_softmax_step<128, kSoftExp8>(s, p.c, m, l, alpha);
       tmem_store_p<128, C::TF32>(s_addr, s);
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 2);
-      if (rescaled && j > jlo[t]) tmem_scale_row<D>(o_addr, alpha);
+      if (rescaled && cnt > 0) tmem_scale_row<D>(o_addr, alpha);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::BAR_P + t));
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 3);
     }
-    if (ok && jhi[t] > jlo[t] && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
+    if (ok && cnt == 0) {
+      store_empty_row<T, D>(p, b, h, qrow);
+    } else if (ok && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
       tc_fence_after();
       store_row<T, D>(o_addr, p, b, h, qrow, m, l);
     }
@@ -404,6 +495,7 @@ __global__ void __launch_bounds__(384, 1)
                       q0 + 128 * t, h, b);
       int it = 0;
       for (int j = jmin; j < jmax && !W.aborted(); ++j) {
+        if (!in_union(j)) continue;  // no query tile of this CTA computes key tile j
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = it % NS;
           const uint32_t ph = static_cast<uint32_t>(it / NS) & 1u;
@@ -430,12 +522,13 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t fmt = C::TF32 ? 2u : 1u;
       constexpr uint32_t idesc_s = idesc_make(128, 128, fmt, false, false);
       constexpr uint32_t idesc_o = idesc_make(128, D, fmt, false, true);
-      // ring position of K_j / V_j (loads start at key tile jmin)
-      auto kslot = [&](int j) { return (2 * (j - jmin)) % NS; };
-      auto kph = [&](int j) { return static_cast<uint32_t>((2 * (j - jmin)) / NS) & 1u; };
-      auto vslot = [&](int j) { return (2 * (j - jmin) + 1) % NS; };
-      auto vph = [&](int j) { return static_cast<uint32_t>((2 * (j - jmin) + 1) / NS) & 1u; };
-      auto uses = [&](int t, int j) { return j >= jlo[t] && j < jhi[t]; };
+      // ring slots of K_j / V_j from j's position among the streamed key tiles
+      // (the producer streams only the tiles that some query tile of this CTA
+      // computes, in increasing order)
+      auto kslot = [&](int pos) { return (2 * pos) % NS; };
+      auto kph = [&](int pos) { return static_cast<uint32_t>((2 * pos) / NS) & 1u; };
+      auto vslot = [&](int pos) { return (2 * pos + 1) % NS; };
+      auto vph = [&](int pos) { return static_cast<uint32_t>((2 * pos + 1) / NS) & 1u; };
       auto issue_s = [&](int t, int slot) {
         const SDesc qa = sdesc_base(sbase + C::SMEM_Q + t * C::TILE, 16, 1024);
         const SDesc kb = sdesc_base(sbase + C::SMEM_KV + slot * C::TILE, 16, 1024);
@@ -455,45 +548,55 @@ __global__ void __launch_bounds__(384, 1)
           mma_ts<C::TF32>(d, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128), idesc_o,
                           ks > 0 ? 1u : acc0);
       };
-      // S_t(j) = Q_t K_j^T; K_j's last reader (tile 1 when it uses K_j) frees its slot
-      auto start_s = [&](int t, int j) -> bool {
-        if (!W.wait(BAR(C::BAR_KVF + kslot(j)), kph(j), 44 + t)) return false;
+      // S_t = Q_t K^T for the key tile at ring position pos
+      auto start_s = [&](int t, int pos) -> bool {
+        if (!W.wait(BAR(C::BAR_KVF + kslot(pos)), kph(pos), 44 + t)) return false;
         tc_fence_after();
-        issue_s(t, kslot(j));
+        issue_s(t, kslot(pos));
         mma_commit(BAR(C::BAR_S + t));
-        if (t == 1 || !uses(1, j)) mma_commit(BAR(C::BAR_KVE + kslot(j)));
         return true;
       };
+      // S_t of a query tile's next key tile is issued right after its P V when
+      // that tile is the next one streamed (always, without a block mask);
+      // otherwise when the loop reaches it, so that no wait can reach past
+      // the tiles the ring holds.
+      int pend[2] = {next_use(0, jmin), next_use(1, jmin)};
+      int cnt[2] = {0, 0};
       bool ok = W.wait(BAR(C::BAR_Q), 0, 40);
-      for (int j = jmin; ok && j < jmax; ++j) {
-        for (int t = 0; ok && t < 2; ++t)
-          if (j == jlo[t] && uses(t, j)) ok = start_s(t, j);
+      for (int j = jmin, pos = 0; ok && j < jmax; ++j) {
+        if (!in_union(j)) continue;
+        if (pend[0] == j && j < jhi(0)) ok = start_s(0, pos);
+        if (ok && pend[1] == j && j < jhi(1)) ok = start_s(1, pos);
         if (!ok) break;
-        if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 42)) { ok = false; break; }
-        if (!uses(0, j) && !uses(1, j)) {
-          // no query tile reads this key tile (cannot happen with windows >= 0:
-          // the two tiles' ranges overlap); hand both slots back
-          if (!W.wait(BAR(C::BAR_KVF + kslot(j)), kph(j), 41)) { ok = false; break; }
-          mbar_arrive(BAR(C::BAR_KVE + kslot(j)));
-          mbar_arrive(BAR(C::BAR_KVE + vslot(j)));
-          continue;
-        }
-        for (int t = 0; ok && t < 2; ++t) {
-          if (!uses(t, j)) continue;
-          if (!W.wait(BAR(C::BAR_P + t), (j - jlo[t]) & 1, 43 + 2 * t)) { ok = false; break; }
-          if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 0);
-          if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 2);
+        // every S(j) is issued: K_j's slot frees once they complete
+        mma_commit(BAR(C::BAR_KVE + kslot(pos)));
+        if (!W.wait(BAR(C::BAR_KVF + vslot(pos)), vph(pos), 42)) { ok = false; break; }
+        const int last_t = uses(1, j) ? 1 : 0;  // the last P V that reads V_j
+        auto pv_step = [&](const int t) -> bool {
+          if (!uses(t, j)) return true;
+          if (!W.wait(BAR(C::BAR_P + t), cnt[t] & 1, 43 + 2 * t)) return false;
+          if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 0);
+          if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 2);
           tc_fence_after();
-          issue_pv(t, vslot(j), j > jlo[t]);
-          if (t == 1 || !uses(1, j)) mma_commit(BAR(C::BAR_KVE + vslot(j)));
-          if (j + 1 < jhi[t]) {
-            ok = start_s(t, j + 1);
-            if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 1);
-            if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo[0], 3);
-          } else {
+          issue_pv(t, vslot(pos), cnt[t] > 0);
+          ++cnt[t];
+          if (t == last_t) mma_commit(BAR(C::BAR_KVE + vslot(pos)));
+          const int nj = next_use(t, j + 1);
+          if (nj >= jhi(t)) {
             mma_commit(BAR(C::BAR_O + t));
+            pend[t] = jhi(t);
+          } else if (next_union(j + 1) == nj) {
+            if (!start_s(t, pos + 1)) return false;
+            pend[t] = -1;
+            if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 1);
+            if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 3);
+          } else {
+            pend[t] = nj;
           }
-        }
+          return true;
+        };
+        if (!pv_step(0) || !pv_step(1)) { ok = false; break; }
+        ++pos;
       }
       // Wait until every MMA this thread issued has finished with TMEM/smem.
       mma_commit(BAR(C::BAR_DONE));

@@ -111,6 +111,26 @@ ATTN_API attn_status_t attn_fwd_window(attn_tensor_t q, attn_tensor_t k, attn_te
                                        int window_right, float scale, void* stream);
 
 /*
+ * Forward with a window (as attn_fwd_window) and a block-sparse tile mask
+ * (FlashAttention (Metal Port) README, Documentation section: block sparsity
+ * as a customisation of the basic algorithm; FlashPrefill V2 finding on the
+ * FlashAttention entity page: block-sparse prefill).
+ *
+ * block_mask: NULL (dense), or a device array of T x T bytes per (batch,
+ * query head), [B][Hq][T][T] contiguous, T = ceil(N / 128): query i sees key
+ * j only when block_mask[b][h][i / 128][j / 128] != 0 (and the window allows
+ * it); tile pairs whose byte is 0 are skipped, not computed.  Owned by the
+ * caller, read during the call's kernels only.  A query row that sees no key
+ * gets o = 0 and lse = -inf.  With a mask: bf16 with D in {64, 128} and
+ * T <= 512 (N <= 65536); anything else is ATTN_ERR_UNSUPPORTED.
+ */
+ATTN_API attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                       attn_tensor_t o, float* lse, int B, int Hq, int Hkv, int N,
+                                       int D, attn_dtype_t dtype, int window_left,
+                                       int window_right, const uint8_t* block_mask, float scale,
+                                       void* stream);
+
+/*
  * Bytes of device workspace attn_bwd needs for these sizes: two fp32 row
  * statistics [B,Hq,N'] (rowsum(dO*O) and lse*log2(e), N' = N rounded up to
  * 128), and for D = 256 also an fp32 dQ accumulator [B,Hq,N,D] (the scratch
@@ -149,6 +169,19 @@ ATTN_API attn_status_t attn_bwd_window(attn_tensor_t q, attn_tensor_t k, attn_te
                                        attn_dtype_t dtype, int window_left, int window_right,
                                        float scale, void* workspace, size_t workspace_bytes,
                                        void* stream);
+
+/*
+ * Backward of attn_fwd_masked: the same window and block_mask (see there);
+ * other arguments as attn_bwd.  Rows that saw no key pass no gradient.  With
+ * a mask: D in {64, 128} and T <= 512, else ATTN_ERR_UNSUPPORTED.
+ */
+ATTN_API attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                       attn_tensor_t o, const float* lse, attn_tensor_t dout,
+                                       attn_tensor_t dq, attn_tensor_t dk, attn_tensor_t dv,
+                                       int B, int Hq, int Hkv, int N, int D,
+                                       attn_dtype_t dtype, int window_left, int window_right,
+                                       const uint8_t* block_mask, float scale, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /*
  * attn_bwd for callers that cannot allocate device memory.

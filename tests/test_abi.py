@@ -85,6 +85,26 @@ def test_fwd_validation_codes(L):
     assert _fwd(L, lse=0x20004) == 3
 
 
+def test_block_mask_validation_codes(L):
+    # refused before anything is launched (no GPU needed): head dim 256, fp32
+    # storage, or more than 512 tiles of 128 rows
+    B, Hq, N, D = 1, 2, 256, 128
+    lse = ctypes.c_void_p(0x20000)
+    bm = ctypes.c_void_p(0x30000)
+
+    def fwd(D=D, dt=0, N=N):
+        t = _t(0x10000, Hq * N * D, N * D, D)
+        return L.attn_fwd_masked(t, t, t, t, lse, B, Hq, Hq, N, D, dt, -1, -1, bm, 0.1, None)
+
+    assert fwd(D=256) == 2
+    assert fwd(D=64, dt=1) == 2
+    assert fwd(N=512 * 128 + 1) == 2
+    t = _t(0x10000, Hq * N * 256, N * 256, 256)
+    ws = L.attn_bwd_workspace_bytes(B, Hq, N, 256)
+    assert L.attn_bwd_masked(t, t, t, t, lse, t, t, t, t, B, Hq, Hq, N, 256, 0, -1, 0, bm, 0.1,
+                             ctypes.c_void_p(0x40000), ws, None) == 2
+
+
 def test_window_validation_codes(L):
     B, Hq, N, D = 1, 2, 256, 128
     t = _t(0x10000, Hq * N * D, N * D, D)
