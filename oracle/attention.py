@@ -59,6 +59,7 @@ __all__ = [
     "attention_fwd",
     "attention_bwd",
     "attention_fwd_rows",
+    "attention_decode",
     "softmax_probs",
 ]
 
@@ -203,3 +204,48 @@ def attention_bwd(q, k, v, do, causal: bool, scale: float, heads=None, window=No
         dk[b, hk] = dk_acc
         dv[b, hk] = dv_acc
     return dq, dk, dv
+
+
+def attention_decode(q, k_pool, v_pool, block_table, seqlens, causal: bool, scale: float,
+                     page: int = 128):
+    """Attention of a few new query tokens against a paged key/value cache.
+
+    The decode step the pages pair with paged KV caches (FlashPrefill V2 and
+    vLLM findings on the FlashAttention entity page: paged KV cache,
+    continuous batching), written out plainly:
+
+    * ``q`` [B, Hq, Sq, D]: the Sq newest tokens of each sequence b;
+    * ``k_pool``, ``v_pool`` [P, page, Hkv, D]: the cache pages; sequence b
+      holds its ``seqlens[b]`` keys in pages ``block_table[b][0..]`` (key t
+      of the sequence is row ``t % page`` of page ``block_table[b][t // page]``);
+    * query token i of sequence b sits at position ``seqlens[b] - Sq + i``;
+      causal lets it see keys at positions <= its own, otherwise it sees all
+      ``seqlens[b]`` keys; a token that sees no key gets O = 0, lse = -inf.
+
+    Returns O [B, Hq, Sq, D] and lse [B, Hq, Sq] (natural log) in float64.
+    """
+    q = _f64(q)
+    kp, vp = _f64(k_pool), _f64(v_pool)
+    b_, hq, sq, d = q.shape
+    hkv = kp.shape[2]
+    g = hq // hkv
+    o = np.zeros((b_, hq, sq, d))
+    lse = np.full((b_, hq, sq), -np.inf)
+    for b in range(b_):
+        n = int(seqlens[b])
+        t = np.arange(n)
+        pages = np.asarray(block_table[b])[t // page]
+        kk = kp[pages, t % page]  # [n, Hkv, D]
+        vv = vp[pages, t % page]
+        pos = n - sq + np.arange(sq)
+        for h in range(hq):
+            hk = h // g
+            s = scale * (q[b, h] @ kk[:, hk].T) if n else np.zeros((sq, 0))
+            if causal:
+                s = np.where(t[None, :] > pos[:, None], -np.inf, s)
+            if n == 0:
+                continue
+            p, l = softmax_probs(s)
+            o[b, h] = p @ vv[:, hk]
+            lse[b, h] = l
+    return o, lse

@@ -520,3 +520,107 @@ def test_block_mask_transposed_mutant_is_caught(monkeypatch):
     monkeypatch.setattr(oa, "_scores", transposed)
     with pytest.raises(AssertionError):
         test_block_mask_matches_explicit_loops(False)
+
+
+# ---------------------------------------------------------------- paged decode
+
+
+def _paged(k, v, page, seed):
+    """Scatter contiguous [B, Hkv, L, D] keys/values into a shuffled page pool."""
+    b_, hkv, n, d = k.shape
+    npg = (n + page - 1) // page
+    total = b_ * npg + 3  # a few unused pages in the pool
+    perm = np.random.default_rng(seed).permutation(total)
+    kp = rnd((total, page, hkv, d), seed + 1)  # garbage in unused rows
+    vp = rnd((total, page, hkv, d), seed + 2)
+    table = np.zeros((b_, npg), np.int64)
+    for b in range(b_):
+        for p in range(npg):
+            pg = perm[b * npg + p]
+            table[b, p] = pg
+            rows = np.arange(p * page, min(n, (p + 1) * page))
+            kp[pg, rows - p * page] = k[b][:, rows].transpose(1, 0, 2)
+            vp[pg, rows - p * page] = v[b][:, rows].transpose(1, 0, 2)
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_full_prefill_equals_attention(causal):
+    # Sq = L: every token is new; bottom-right alignment is then top-left
+    b_, hq, hkv, n, d, page = 2, 4, 2, 11, 5, 4
+    q, k, v = rnd((b_, hq, n, d), 100), rnd((b_, hkv, n, d), 101), rnd((b_, hkv, n, d), 102)
+    kp, vp, table = _paged(k, v, page, 103)
+    o, l = oracle.attention_decode(q, kp, vp, table, [n] * b_, causal, 0.55, page=page)
+    o_r, l_r = fwd(q, k, v, causal, 0.55)
+    np.testing.assert_allclose(o, o_r, atol=1e-13)
+    np.testing.assert_allclose(l, l_r, atol=1e-13)
+
+
+def test_decode_last_tokens_bottom_right_aligned():
+    # Sq newest tokens of length-L sequences = rows L-Sq .. L-1 of full causal attention
+    b_, hq, hkv, d, page, sq = 3, 2, 1, 4, 5, 3
+    lens = [13, 7, 3]
+    n = max(lens)
+    qfull, k, v = rnd((b_, hq, n, d), 110), rnd((b_, hkv, n, d), 111), rnd((b_, hkv, n, d), 112)
+    kp, vp, table = _paged(k, v, page, 113)
+    q = np.zeros((b_, hq, sq, d))
+    for b, L in enumerate(lens):
+        q[b] = qfull[b, :, L - sq:L]
+    o, l = oracle.attention_decode(q, kp, vp, table, lens, True, 0.7, page=page)
+    for b, L in enumerate(lens):
+        for h in range(hq):
+            o_r, l_r = oracle.attention_fwd_rows(qfull[b:b + 1, :, :L], k[b:b + 1, :, :L],
+                                                 v[b:b + 1, :, :L], True, 0.7, 0, h,
+                                                 np.arange(L - sq, L))
+            np.testing.assert_allclose(o[b, h], o_r, atol=1e-13)
+            np.testing.assert_allclose(l[b, h], l_r, atol=1e-13)
+
+
+def test_decode_single_token_explicit_loops_and_empty():
+    b_, hq, hkv, d, page = 2, 2, 2, 3, 4
+    lens = [6, 0]
+    k, v = rnd((b_, hkv, 6, d), 120), rnd((b_, hkv, 6, d), 121)
+    q = rnd((b_, hq, 1, d), 122)
+    kp, vp, table = _paged(k, v, page, 123)
+    for causal in (False, True):
+        o, l = oracle.attention_decode(q, kp, vp, table, lens, causal, 0.9, page=page)
+        for h in range(hq):
+            sc = [0.9 * float(q[0, h, 0] @ k[0, h, j]) for j in range(6)]
+            mx = max(sc)
+            w = [math.exp(x - mx) for x in sc]
+            np.testing.assert_allclose(o[0, h, 0], sum(wj * k_ for wj, k_ in zip(w, v[0, h])) / sum(w),
+                                       atol=1e-13)
+            assert abs(l[0, h, 0] - (mx + math.log(sum(w)))) < 1e-13
+        # an empty sequence: no key, O = 0, lse = -inf
+        assert np.all(o[1] == 0.0) and np.all(l[1] == -np.inf)
+
+
+def test_decode_gqa_and_page_order():
+    b_, hq, hkv, n, d, page, sq = 2, 6, 2, 9, 4, 4, 2
+    q, k, v = rnd((b_, hq, sq, d), 130), rnd((b_, hkv, n, d), 131), rnd((b_, hkv, n, d), 132)
+    kp, vp, table = _paged(k, v, page, 133)
+    kp2, vp2, table2 = _paged(k, v, page, 140)  # another page shuffle
+    o, l = oracle.attention_decode(q, kp, vp, table, [n, n - 2], True, 0.6, page=page)
+    o2, l2 = oracle.attention_decode(q, kp2, vp2, table2, [n, n - 2], True, 0.6, page=page)
+    np.testing.assert_allclose(o, o2, atol=1e-14)
+    np.testing.assert_allclose(l, l2, atol=1e-14)
+    g = hq // hkv
+    kr, vr = np.repeat(k, g, axis=1), np.repeat(v, g, axis=1)
+    kp3, vp3, table3 = _paged(kr, vr, page, 133)
+    o3, l3 = oracle.attention_decode(q, kp3, vp3, table3, [n, n - 2], True, 0.6, page=page)
+    np.testing.assert_allclose(o, o3, atol=1e-13)
+    np.testing.assert_allclose(l, l3, atol=1e-13)
+
+
+def test_decode_top_left_mutant_is_caught(monkeypatch):
+    src = oa.attention_decode
+
+    def top_left(q, k_pool, v_pool, block_table, seqlens, causal, scale, page=128):
+        # wrong alignment: query token i at position i instead of L - Sq + i
+        sq = np.asarray(q).shape[2]
+        o, l = src(q, k_pool, v_pool, block_table, [sq] * len(seqlens), causal, scale, page)
+        return o, l
+
+    monkeypatch.setattr(oracle, "attention_decode", top_left)
+    with pytest.raises(AssertionError):
+        test_decode_last_tokens_bottom_right_aligned()
