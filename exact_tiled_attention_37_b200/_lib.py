@@ -66,6 +66,11 @@ def lib(path: str | None = None) -> ctypes.CDLL:
     L.attn_bwd_masked.restype = i
     L.attn_bwd_masked.argtypes = [T, T, T, T, vp, T, T, T, T, i, i, i, i, i, i, i, i, vp, f, vp,
                                   ctypes.c_size_t, vp]
+    L.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+    L.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.attn_decode_paged.restype = i
+    L.attn_decode_paged.argtypes = [T, T, T, i, vp, i, vp, T, vp, i, i, i, i, i, i, i, f, vp,
+                                    ctypes.c_size_t, vp]
     L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
     L.attn_bwd.restype = i

@@ -154,3 +154,59 @@ def set_wait_limit_ns(ns: int):
 
 def set_debug_flags(flags: int):
     _lib.lib().attn_debug_set_flags(int(flags))
+
+
+def _pool_desc(t: torch.Tensor, name: str) -> AttnTensor:
+    """[P, 128, Hkv, D] page pool -> (ptr, page stride, head stride, row stride)."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dim() != 4 or t.shape[1] != 128 or t.stride(3) != 1:
+        raise ValueError(f"{name} must be [P, 128, Hkv, D] with unit stride on D")
+    sp, sr, sh, _ = t.stride()
+    return AttnTensor(ctypes.c_void_p(t.data_ptr()), sp, sh, sr)
+
+
+def decode_workspace_bytes(B: int, Hq: int, Sq: int, D: int, max_pages: int) -> int:
+    return int(_lib.lib().attn_decode_workspace_bytes(B, Hq, Sq, D, max_pages))
+
+
+def attn_decode(q, k_pool, v_pool, block_table, seqlens, causal: bool = False,
+                scale: float | None = None, out=None, lse=None, workspace=None):
+    """Decode against a paged cache: q [B,Hq,Sq,D] (newest tokens), k_pool/v_pool
+    [P,128,Hkv,D], block_table int32 [B,max_pages], seqlens int32 [B].
+
+    Query token i of sequence b sits at position seqlens[b] - Sq + i.
+    Returns O [B,Hq,Sq,D] (bf16) and lse [B,Hq,Sq] fp32 (natural log)."""
+    B, Hq, Sq, D = q.shape
+    P, _, Hkv, _ = k_pool.shape
+    if v_pool.shape != k_pool.shape or k_pool.shape[3] != D:
+        raise ValueError(f"pool shapes k{tuple(k_pool.shape)} v{tuple(v_pool.shape)} vs q{tuple(q.shape)}")
+    for t, name in ((block_table, "block_table"), (seqlens, "seqlens")):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if block_table.dim() != 2 or block_table.shape[0] != B or seqlens.shape != (B,):
+        raise ValueError("block_table must be [B, max_pages] and seqlens [B]")
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (B, Hq, Sq):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Sq] tensor")
+    L = _lib.lib()
+    need = int(L.attn_decode_workspace_bytes(B, Hq, Sq, D, max_pages))
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    code = L.attn_decode_paged(_desc(q, "q"), _pool_desc(k_pool, "k_pool"),
+                               _pool_desc(v_pool, "v_pool"), P,
+                               ctypes.c_void_p(block_table.data_ptr()), max_pages,
+                               ctypes.c_void_p(seqlens.data_ptr()), _desc(out, "out"),
+                               ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, Sq, D,
+                               _dtype_code(q), int(bool(causal)), float(scale),
+                               ctypes.c_void_p(workspace.data_ptr()),
+                               ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                               _stream(q.device))
+    _check(code, "attn_decode")
+    return out, lse

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -16,6 +17,7 @@
 #include "bwd.cuh"
 #include "bwd_split.cuh"
 #include "fwd.cuh"
+#include "decode.cuh"
 #include "fwd_fp32.cuh"
 
 // Device status word: [0] code, [1] wait site, [2..3] block of the first failure.
@@ -251,6 +253,72 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   return last_launch();
 }
 
+// ---------------------------------------------------------------- decode
+constexpr int kDecodeMaxSplits = 64;
+
+// Splits of the page range per (sequence, key/value head): enough CTAs for
+// about two per SM, at most one per page and kDecodeMaxSplits.
+int decode_splits(int B, int Hkv, int max_pages, int* pages_per_split) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long units = static_cast<long long>(B) * Hkv;
+  int splits = static_cast<int>(std::min<long long>(kDecodeMaxSplits, (2LL * sms + units - 1) / units));
+  splits = std::max(1, std::min(splits, max_pages));
+  const int pps = (max_pages + splits - 1) / splits;
+  *pages_per_split = pps;
+  return (max_pages + pps - 1) / pps;
+}
+
+size_t decode_workspace(int B, int Hq, int Sq, int D, int max_pages) {
+  const size_t rows = static_cast<size_t>(B) * Hq * Sq * std::min(max_pages, kDecodeMaxSplits);
+  return eta::round_up(rows * D * 4, 256) + eta::round_up(rows * 4, 256);
+}
+
+// Page pool [P, 128, Hkv, D] (t.sb: page stride, t.sh: head stride, t.sn: row
+// stride, in elements) as a 4-D TMA map over (D, Hkv, 128 rows, P) with
+// boxes of 64 columns x 128 rows of one head.
+attn_status_t make_pool_map(CUtensorMap* m, const attn_tensor_t& t, int P, int Hkv, int D) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv), 128u,
+                        static_cast<cuuint64_t>(P)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(t.sh) * 2, static_cast<cuuint64_t>(t.sn) * 2,
+                           static_cast<cuuint64_t>(t.sb) * 2};
+  cuuint32_t box[4] = {64u, 1u, 128u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t check_pool(const attn_tensor_t& t, int P, int Hkv) {
+  if (!t.ptr) return ATTN_ERR_INVALID_ARG;
+  if ((P > 1 && t.sb <= 0) || (Hkv > 1 && t.sh <= 0) || t.sn <= 0) return ATTN_ERR_INVALID_ARG;
+  if (t.sb < 0 || t.sh < 0) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return ATTN_ERR_MISALIGNED;
+  if ((t.sb * 2) % 16 || (t.sh * 2) % 16 || (t.sn * 2) % 16) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+template <int D, int NS>
+attn_status_t launch_decode(const attn_tensor_t& kp, const attn_tensor_t& vp, int P,
+                            eta::DecodeParams& p, cudaStream_t st) {
+  using C = eta::DecodeCfg<D, NS>;
+  CUtensorMap tk, tv;
+  attn_status_t s;
+  if ((s = make_pool_map(&tk, kp, P, p.Hkv, D)) != ATTN_OK) return s;
+  if ((s = make_pool_map(&tv, vp, P, p.Hkv, D)) != ATTN_OK) return s;
+  auto kern = eta::decode_kernel<D, NS>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
+  kern<<<dim3(p.splits, p.Hkv, p.B), C::THREADS, C::SMEM_BYTES, st>>>(tk, tv, p);
+  if ((s = last_launch()) != ATTN_OK) return s;
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.Sq;
+  eta::decode_combine_kernel<D><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);
+  return last_launch();
+}
+
 attn_status_t check_sizes(int B, int Hq, int Hkv, int N) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
@@ -389,6 +457,59 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
     case 128: return launch_pingpong<__nv_bfloat16, 128, 4>(q, k, v, p, B, Hq, Hkv, N, st);
     default: return launch_single<256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
   }
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int max_pages) {
+  if (B < 1 || Hq < 1 || Sq < 1 || D < 1 || max_pages < 1) return 0;
+  return decode_workspace(B, Hq, Sq, D, max_pages);
+}
+
+attn_status_t attn_decode_paged(attn_tensor_t q, attn_tensor_t k_pool, attn_tensor_t v_pool,
+                                int num_pages, const int* block_table, int max_pages,
+                                const int* seqlens, attn_tensor_t o, float* lse, int B, int Hq,
+                                int Hkv, int Sq, int D, attn_dtype_t dtype, int causal,
+                                float scale, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  attn_status_t s;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || num_pages < 1 || max_pages < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!block_table || !seqlens || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!workspace) return ATTN_ERR_WORKSPACE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_BF16) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+  if (!(D == 64 || D == 128)) return ATTN_ERR_UNSUPPORTED;
+  if ((Hq / Hkv) * Sq > 128 || B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  if ((s = check_tensor(q, B, Hq, Sq, 2)) != ATTN_OK) return s;
+  if ((s = check_tensor(o, B, Hq, Sq, 2)) != ATTN_OK) return s;
+  if ((s = check_pool(k_pool, num_pages, Hkv)) != ATTN_OK) return s;
+  if ((s = check_pool(v_pool, num_pages, Hkv)) != ATTN_OK) return s;
+  if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < decode_workspace(B, Hq, Sq, D, max_pages)) return ATTN_ERR_WORKSPACE;
+  eta::DecodeParams p;
+  p.q = q.ptr;
+  p.qsb = q.sb; p.qsh = q.sh; p.qsn = q.sn;
+  p.o = o.ptr;
+  p.osb = o.sb; p.osh = o.sh; p.osn = o.sn;
+  p.lse = lse;
+  p.block_table = block_table;
+  p.seqlens = seqlens;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.group = Hq / Hkv;
+  p.max_pages = max_pages;
+  p.splits = decode_splits(B, Hkv, max_pages, &p.pages_per_split);
+  const size_t rows = static_cast<size_t>(B) * Hq * Sq * p.splits;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        eta::round_up(rows * D * 4, 256));
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64) return launch_decode<64, 8>(k_pool, v_pool, num_pages, p, st);
+  return launch_decode<128, 6>(k_pool, v_pool, num_pages, p, st);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D) {

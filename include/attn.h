@@ -214,6 +214,38 @@ ATTN_API attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_t
                                         void* stream);
 
 /*
+ * Decode against a paged key/value cache (FlashAttention entity page:
+ * FlashPrefill V2 and vLLM findings, paged KV cache and continuous batching;
+ * the split-KV / decode step with a logsumexp merge).
+ *
+ * q [B, Hq, Sq, D] holds the Sq newest tokens of each of B sequences; query
+ * token i of sequence b sits at position seqlens[b] - Sq + i.  The keys and
+ * values live in 128-row pages: k_pool and v_pool describe [P, 128, Hkv, D]
+ * pools (num_pages = P) with .sb = page stride, .sh = head stride, .sn = row
+ * stride (elements; unit stride on D; 16-byte multiples).  Key t of sequence
+ * b is row t % 128 of page block_table[b * max_pages + t / 128] (int32 device
+ * array [B][max_pages]); seqlens is an int32 device array [B] with
+ * 0 <= seqlens[b] <= 128 * max_pages.  causal != 0: token i sees keys at
+ * positions <= its own; otherwise all seqlens[b] keys.  Writes o [B, Hq, Sq,
+ * D] (bf16) and lse [B, Hq, Sq] (fp32, natural log, contiguous); a token that
+ * sees no key gets o = 0, lse = -inf.
+ *
+ * The page range of each (sequence, key/value head) is split so that the GPU
+ * gets about two CTAs per SM; each split's partial result goes to the
+ * workspace (attn_decode_workspace_bytes, 256-byte aligned, caller-owned) and
+ * a second kernel merges them.  Requirements: bf16, D in {64, 128},
+ * (Hq / Hkv) * Sq <= 128.  Page ids outside [0, P) read as zeros.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int max_pages);
+ATTN_API attn_status_t attn_decode_paged(attn_tensor_t q, attn_tensor_t k_pool,
+                                         attn_tensor_t v_pool, int num_pages,
+                                         const int* block_table, int max_pages,
+                                         const int* seqlens, attn_tensor_t o, float* lse, int B,
+                                         int Hq, int Hkv, int Sq, int D, attn_dtype_t dtype,
+                                         int causal, float scale, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a kernel's
  * bounded wait gave up; *where, if not NULL, receives the wait site id) or
