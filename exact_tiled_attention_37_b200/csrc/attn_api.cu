@@ -255,15 +255,21 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
 
 // ---------------------------------------------------------------- decode
 constexpr int kDecodeMaxSplits = 64;
+#ifndef ETA_DECODE_CTAS_PER_SM
+#define ETA_DECODE_CTAS_PER_SM 4
+#endif
+constexpr long long kDecodeCtasPerSm = ETA_DECODE_CTAS_PER_SM;
 
 // Splits of the page range per (sequence, key/value head): enough CTAs for
-// about two per SM, at most one per page and kDecodeMaxSplits.
+// about four per SM (in waves of one CTA per SM: fewer left a long tail,
+// measured), at most one per page and kDecodeMaxSplits.
 int decode_splits(int B, int Hkv, int max_pages, int* pages_per_split) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long units = static_cast<long long>(B) * Hkv;
-  int splits = static_cast<int>(std::min<long long>(kDecodeMaxSplits, (2LL * sms + units - 1) / units));
+  int splits = static_cast<int>(
+      std::min<long long>(kDecodeMaxSplits, (kDecodeCtasPerSm * sms + units - 1) / units));
   splits = std::max(1, std::min(splits, max_pages));
   const int pps = (max_pages + splits - 1) / splits;
   *pages_per_split = pps;

@@ -231,7 +231,7 @@ ATTN_API attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_t
  * sees no key gets o = 0, lse = -inf.
  *
  * The page range of each (sequence, key/value head) is split so that the GPU
- * gets about two CTAs per SM; each split's partial result goes to the
+ * gets about four CTAs per SM; each split's partial result goes to the
  * workspace (attn_decode_workspace_bytes, 256-byte aligned, caller-owned) and
  * a second kernel merges them.  Requirements: bf16, D in {64, 128},
  * (Hq / Hkv) * Sq <= 128.  Page ids outside [0, P) read as zeros.
