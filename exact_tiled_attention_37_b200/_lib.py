@@ -66,6 +66,8 @@ def lib(path: str | None = None) -> ctypes.CDLL:
     L.attn_bwd_masked.restype = i
     L.attn_bwd_masked.argtypes = [T, T, T, T, vp, T, T, T, T, i, i, i, i, i, i, i, i, vp, f, vp,
                                   ctypes.c_size_t, vp]
+    L.attn_fwd_fp8.restype = i
+    L.attn_fwd_fp8.argtypes = [T, T, T, T, vp, i, i, i, i, i, f, f, f, i, i, f, vp]
     L.attn_decode_workspace_bytes.restype = ctypes.c_size_t
     L.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
     L.attn_decode_paged.restype = i

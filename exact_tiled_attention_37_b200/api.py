@@ -210,3 +210,30 @@ def attn_decode(q, k_pool, v_pool, block_table, seqlens, causal: bool = False,
                                _stream(q.device))
     _check(code, "attn_decode")
     return out, lse
+
+
+def attn_fwd_fp8(q, k, v, q_scale: float = 1.0, k_scale: float = 1.0, v_scale: float = 1.0,
+                 causal: bool = False, scale: float | None = None, out=None, lse=None,
+                 window=None):
+    """Forward on e4m3 inputs (torch.float8_e4m3fn, D = 128) holding x / scale with
+    per-tensor scales; returns O (bf16) and lse of attention on the dequantised inputs."""
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError(f"{name} must be torch.float8_e4m3fn")
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(q.shape, device=q.device, dtype=torch.bfloat16)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    wl, wr = _window(causal, window)
+    code = _lib.lib().attn_fwd_fp8(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(out, "out"),
+                                   ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, N, D,
+                                   float(q_scale), float(k_scale), float(v_scale), wl, wr,
+                                   float(scale), _stream(q.device))
+    _check(code, "attn_fwd_fp8")
+    return out, lse

@@ -108,7 +108,10 @@ attn_status_t make_map(CUtensorMap* m, const attn_tensor_t& t, int B, int H, int
                            static_cast<cuuint64_t>(sb * es)};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows), 1u, 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+  const CUtensorMapDataType dt = es == 2   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult r = enc(m, dt,
                    4, t.ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -447,6 +450,7 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
   p.wait_limit_ns = g_wait_limit_ns.load();
   p.debug_flags = g_debug_flags.load();
+  p.o_mul = 1.f;
   p.bmask = block_mask;
   p.nt = (N + 127) / 128;
 
@@ -463,6 +467,48 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
     case 128: return launch_pingpong<__nv_bfloat16, 128, 4>(q, k, v, p, B, Hq, Hkv, N, st);
     default: return launch_single<256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
   }
+}
+
+attn_status_t attn_fwd_fp8(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
+                           float* lse, int B, int Hq, int Hkv, int N, int D, float q_scale,
+                           float k_scale, float v_scale, int window_left, int window_right,
+                           float scale, void* stream) {
+  attn_status_t s;
+  if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
+  if ((s = check_sizes(B, Hq, Hkv, N)) != ATTN_OK) return s;
+  if (!lse) return ATTN_ERR_INVALID_ARG;
+  for (float f : {scale, q_scale, k_scale, v_scale})
+    if (!(f > 0.f) || !std::isfinite(f)) return ATTN_ERR_INVALID_ARG;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((s = check_tensor(q, B, Hq, N, 1)) != ATTN_OK) return s;
+  if ((s = check_tensor(k, B, Hkv, N, 1)) != ATTN_OK) return s;
+  if ((s = check_tensor(v, B, Hkv, N, 1)) != ATTN_OK) return s;
+  if ((s = check_tensor(o, B, Hq, N, 2)) != ATTN_OK) return s;
+  if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
+  eta::FwdParams p;
+  p.o = o.ptr;
+  p.lse = lse;
+  p.osb = o.sb;
+  p.osh = o.sh;
+  p.osn = o.sn;
+  p.Hq = Hq;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.wl = window_left >= N ? -1 : window_left;
+  p.wr = window_right >= N ? -1 : window_right;
+  // the per-tensor scales fold into the score scale and the output multiplier
+  const double se = static_cast<double>(scale) * q_scale * k_scale;
+  p.scale = static_cast<float>(se);
+  p.c = static_cast<float>(se * 1.4426950408889634);
+  if (!std::isfinite(p.c) || !(p.scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if ((s = status_ptr(&p.status)) != ATTN_OK) return s;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  p.debug_flags = 0;
+  p.o_mul = v_scale / eta::kP8Scale;
+  p.bmask = nullptr;
+  p.nt = (N + 127) / 128;
+  return launch_pingpong<__nv_fp8_e4m3, 128, 8>(q, k, v, p, B, Hq, Hkv, N,
+                                                static_cast<cudaStream_t>(stream));
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int max_pages) {

@@ -26,6 +26,8 @@
 // grows by more than 2^kRescaleLog2) and the epilogue (O / l, lse).
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace eta {
@@ -67,6 +69,7 @@ struct FwdParams {
   int* status;       // device status word (4 ints)
   unsigned long long wait_limit_ns;
   int debug_flags;   // bit 0: producer skips the first V tile (timeout test)
+  float o_mul;       // output multiplier (1; e4m3 inputs: v_scale / kP8Scale)
   // block-sparse tile mask [B, Hq, nt, nt] (nonzero = the 128 x 128 tile pair is
   // computed), or null; nt = ceil(N / 128) <= kMaxMaskTiles
   const uint8_t* bmask;
@@ -103,7 +106,9 @@ __device__ __forceinline__ int next_bit(const uint32_t* w, int j, int end) {
 // for some row of the warp); alpha is this row's factor for O and l.
 // SOFT8 of every 8 columns take their exponential from the FMA-pipe
 // polynomial instead of the MUFU unit (the two run in parallel).
-template <int BC, int SOFT8>
+// TAU: rescale only when the maximum grows by more than 2^TAU (p <= 2^TAU);
+// e4m3 products need TAU = 0 (p <= 1).
+template <int BC, int SOFT8, int TAU = static_cast<int>(kRescaleLog2)>
 __device__ __forceinline__ bool online_softmax_step(float (&s)[BC], float c, float& m, float& l,
                                                     float& alpha) {
   static_assert(BC % 8 == 0 && SOFT8 % 2 == 0 && SOFT8 <= 8, "column pattern");
@@ -120,7 +125,7 @@ __device__ __forceinline__ bool online_softmax_step(float (&s)[BC], float c, flo
   for (int i = BC - (BC - 12) % 8; i < BC; ++i) mx0 = fmaxf(mx0, s[i]);
   const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
   // +inf when m = -inf and m_new is finite; NaN (false) when both are -inf
-  const bool need = (m_new - m) * c > kRescaleLog2;
+  const bool need = (m_new - m) * c > static_cast<float>(TAU);
   const bool warp_rescale = __any_sync(0xffffffffu, need);
   alpha = 1.f;
   if (warp_rescale) {
@@ -188,6 +193,38 @@ __device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&p)[BC
   }
 }
 
+// e4m3 P for the kind::f8f6f4 P V product, as two terms so that P keeps about
+// 8 significant bits (one e4m3 term has 4): x = p * kP8Scale (p <= 1, so
+// x <= 256, inside e4m3's range; the scale keeps small probabilities out of
+// e4m3's subnormals), hi = e4m3(x), lo = e4m3(x - hi) (the residual, formed
+// in fp16, which holds both exactly enough).  hi goes to the first BC/4
+// columns, lo to the next BC/4, four values per 32-bit column.
+constexpr float kP8Scale = 256.f;
+template <int BC>
+__device__ __forceinline__ void tmem_store_p8(uint32_t taddr, const float (&p)[BC]) {
+  static_assert(BC == 128, "one 128-column row");
+  uint32_t hi[32], lo[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float2 x = make_float2(p[4 * i + 2 * k] * kP8Scale, p[4 * i + 2 * k + 1] * kP8Scale);
+      const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+      const __half2 hf = __half2(__nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3));
+      const __half2 r = __hsub2(__float22half2_rn(x), hf);
+      const __nv_fp8x2_storage_t l =
+          __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(r), __NV_SATFINITE, __NV_E4M3);
+      hw |= static_cast<uint32_t>(h) << (16 * k);
+      lw |= static_cast<uint32_t>(l) << (16 * k);
+    }
+    hi[i] = hw;
+    lo[i] = lw;
+  }
+  tmem_st32(taddr, hi);
+  tmem_st32(taddr + BC / 4, lo);
+}
+
 // Multiplies DC fp32 TMEM columns of this lane by alpha (the correction step).
 template <int DC>
 __device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
@@ -207,7 +244,7 @@ template <typename T, int D>
 __device__ __forceinline__ void store_row(uint32_t o_taddr, const FwdParams& p, int b, int h,
                                           int qrow, float m, float l) {
   const bool valid = qrow < p.N;
-  const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no visible key stores O = 0
+  const float inv_l = l > 0.f ? p.o_mul / l : 0.f;  // a row with no visible key stores O = 0
   char* row = static_cast<char*>(p.o) +
               (static_cast<long long>(b) * p.osb + static_cast<long long>(h) * p.osh +
                static_cast<long long>(qrow) * p.osn) *
@@ -294,6 +331,7 @@ __device__ __forceinline__ int2 key_tiles(int qs, int N, int wl, int wr, int BN)
 template <typename T, int D, int NS>
 struct PingPongCfg {
   static constexpr bool TF32 = sizeof(T) == 4;
+  static constexpr bool FP8 = sizeof(T) == 1;  // e4m3 inputs, kind::f8f6f4 products
   static constexpr int ES = sizeof(T);
   static constexpr int ROWB = D * ES;        // bytes per row
   static constexpr int NCHUNK = ROWB / 128;  // 128-byte swizzle chunks per row
@@ -302,7 +340,8 @@ struct PingPongCfg {
   static constexpr int TILE = 128 * ROWB;
   static constexpr int QK_STEPS = ROWB / 32;
   static constexpr int PV_ROWS = 32 / ES;    // V rows consumed per MMA
-  static constexpr int PV_STEPS = BN / PV_ROWS;
+  // e4m3: P is split into two e4m3 terms (high and residual), each multiplied by V
+  static constexpr int PV_STEPS = (FP8 ? 2 : 1) * BN / PV_ROWS;
   static constexpr int O_COL = 256;          // O0 at 256, O1 at 256 + D
   static constexpr int TMEM_COLS = 512;
   static constexpr int SMEM_Q = 0;
@@ -328,7 +367,7 @@ struct PingPongCfg {
   static_assert(THREADS * LAUNCH_REGS == 256 * SOFTMAX_REGS + 128 * OTHER_REGS, "register split");
   // bf16 only: tf32 products would keep 10 mantissa bits, which misses the
   // logsumexp tolerance; fp32 storage goes through fwd_fp32_kernel.
-  static_assert(sizeof(T) == 2, "bf16 storage");
+  static_assert(sizeof(T) == 2 || sizeof(T) == 1, "bf16 or e4m3 storage");
   static_assert(ROWB % 128 == 0, "row must be whole 128-byte chunks");
   static_assert(256 + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -342,6 +381,7 @@ __global__ void __launch_bounds__(384, 1)
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = PingPongCfg<T, D, NS>;
+  using OutT = std::conditional_t<C::FP8, __nv_bfloat16, T>;  // e4m3 inputs give bf16 O
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -465,8 +505,14 @@ __global__ void __launch_bounds__(384, 1)
       float s[128];
       tmem_load_row<128>(s_addr, s);
       apply_mask<128>(s, col_window(128 * j, qrow, p.N, p.wl, p.wr));
-      const bool rescaled = online_softmax_step<128, kSoftExp8>(s, p.c, m, l, alpha);
-      tmem_store_p<128, C::TF32>(s_addr, s);
+      const bool rescaled =
+          online_softmax_step<128, kSoftExp8, C::FP8 ? 0 : static_cast<int>(kRescaleLog2)>(
+              s, p.c, m, l, alpha);
+      if constexpr (C::FP8) {
+        tmem_store_p8<128>(s_addr, s);
+      } else {
+        tmem_store_p<128, C::TF32>(s_addr, s);
+      }
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 2);
       if (rescaled && cnt > 0) tmem_scale_row<D>(o_addr, alpha);
       tmem_wait_st();
@@ -476,10 +522,10 @@ __global__ void __launch_bounds__(384, 1)
       if (r == 0) ETA_FTRACE_AT(tcta, t, j, 3);
     }
     if (ok && cnt == 0) {
-      store_empty_row<T, D>(p, b, h, qrow);
+      store_empty_row<OutT, D>(p, b, h, qrow);
     } else if (ok && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
       tc_fence_after();
-      store_row<T, D>(o_addr, p, b, h, qrow, m, l);
+      store_row<OutT, D>(o_addr, p, b, h, qrow, m, l);
     }
   } else if (warp == 8) {
     // ------------------------------------------------ TMA producer
@@ -519,7 +565,7 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 9) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t fmt = C::TF32 ? 2u : 1u;
+      constexpr uint32_t fmt = C::FP8 ? 0u : (C::TF32 ? 2u : 1u);
       constexpr uint32_t idesc_s = idesc_make(128, 128, fmt, false, false);
       constexpr uint32_t idesc_o = idesc_make(128, D, fmt, false, true);
       // ring slots of K_j / V_j from j's position among the streamed key tiles
@@ -536,7 +582,11 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
           const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          mma_ss<C::TF32>(d, sdesc_at(qa, off), sdesc_at(kb, off), idesc_s, ks > 0);
+          if constexpr (C::FP8) {
+            mma_ss_f8(d, sdesc_at(qa, off), sdesc_at(kb, off), idesc_s, ks > 0);
+          } else {
+            mma_ss<C::TF32>(d, sdesc_at(qa, off), sdesc_at(kb, off), idesc_s, ks > 0);
+          }
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
@@ -545,8 +595,15 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
         for (int ks = 0; ks < C::PV_STEPS; ++ks)
-          mma_ts<C::TF32>(d, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128), idesc_o,
-                          ks > 0 ? 1u : acc0);
+          if constexpr (C::FP8) {
+            // steps 0-3: high term (TMEM columns 0-31), 4-7: residual (32-63),
+            // both against the same V rows
+            mma_ts_f8(d, a + 8u * ks, sdesc_at(vb, (ks & 3) * C::PV_ROWS * 128), idesc_o,
+                      ks > 0 ? 1u : acc0);
+          } else {
+            mma_ts<C::TF32>(d, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128), idesc_o,
+                            ks > 0 ? 1u : acc0);
+          }
       };
       // S_t = Q_t K^T for the key tile at ring position pos
       auto start_s = [&](int t, int pos) -> bool {

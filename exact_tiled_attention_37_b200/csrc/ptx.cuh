@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace eta {
@@ -229,8 +230,9 @@ __device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t byte_off) {
   return (static_cast<uint64_t>(d.hi) << 32) | static_cast<uint64_t>(d.lo + (byte_off >> 4));
 }
 
-// Instruction descriptor for kind::f16 / kind::tf32 with an f32 accumulator.
-// fmt: 1 = bf16, 2 = tf32.  a_mn / b_mn: operand is MN-major (else K-major).
+// Instruction descriptor for kind::f16 / kind::tf32 / kind::f8f6f4 with an f32
+// accumulator.  fmt: 1 = bf16, 2 = tf32 (kind::f16 / tf32); 0 = e4m3
+// (kind::f8f6f4).  a_mn / b_mn: operand is MN-major (else K-major).
 __host__ __device__ constexpr uint32_t idesc_make(int M, int N, uint32_t fmt, bool a_mn, bool b_mn) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) |
          ((b_mn ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
@@ -272,6 +274,24 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
   }
+}
+
+// kind::f8f6f4 forms (both operands 8-bit floats, fp32 accumulator).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
@@ -447,6 +467,13 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   r.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
   r.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
   return r;
+}
+
+// Four floats to e4m3 (round to nearest even, saturating), first in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

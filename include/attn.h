@@ -214,6 +214,24 @@ ATTN_API attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_t
                                         void* stream);
 
 /*
+ * FP8 forward (FlashAttention entity page: FP8 inference in the FlashPrefill V2
+ * finding; r/mlscaling FA3 item): q, k, v are e4m3 [B, H, N, 128] tensors
+ * (1-byte elements, strides in elements, 16-byte multiples) holding x / scale
+ * for per-tensor scales q_scale, k_scale, v_scale; the result is attention of
+ * the dequantised inputs (q_scale * q, ...) with the given softmax scale and
+ * window (as attn_fwd_window): o [B, Hq, N, 128] bf16 and lse as attn_fwd.
+ * Both products run on e4m3 tensor-core operands (kind::f8f6f4).  P (times
+ * 256) enters P V as two e4m3 terms, its rounding and the rounding's residual,
+ * so it keeps about 8 significant bits (a single e4m3 term keeps 4, which
+ * puts the output's error near 5 % on random inputs).  D = 128 only (else
+ * ATTN_ERR_UNSUPPORTED).
+ */
+ATTN_API attn_status_t attn_fwd_fp8(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
+                                    attn_tensor_t o, float* lse, int B, int Hq, int Hkv, int N,
+                                    int D, float q_scale, float k_scale, float v_scale,
+                                    int window_left, int window_right, float scale, void* stream);
+
+/*
  * Decode against a paged key/value cache (FlashAttention entity page:
  * FlashPrefill V2 and vLLM findings, paged KV cache and continuous batching;
  * the split-KV / decode step with a logsumexp merge).
