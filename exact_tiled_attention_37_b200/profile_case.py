@@ -1,5 +1,7 @@
 """Runs one forward (+ backward) of a named workload through the C ABI, for
 profilers: ``python -m exact_tiled_attention_37_b200.profile_case --workload 2``.
+``--decode`` instead runs a paged decode: 8 sequences of 32768 cached keys,
+Hq=32, Hkv=8, D=128, one new token, the 2048 pages in a seeded random order.
 
 Exits non-zero when a kernel reports a device-side timeout.
 """
@@ -11,8 +13,25 @@ import sys
 
 import torch
 
-from . import attn_bwd, attn_fwd, device_status
+from . import attn_bwd, attn_decode, attn_fwd, device_status
 from .inputs import make_inputs, workload
+
+
+def decode_case(repeat: int) -> int:
+    B, Hq, Hkv, D, L = 8, 32, 8, 128, 32768
+    pages = L // 128
+    g = torch.Generator(device="cuda").manual_seed(3)
+    kp = torch.randn(B * pages, 128, Hkv, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    vp = torch.randn(B * pages, 128, Hkv, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    q = torch.randn(B, Hq, 1, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    table = torch.randperm(B * pages, device="cuda", generator=g).to(torch.int32)
+    seqlens = torch.full((B,), L, device="cuda", dtype=torch.int32)
+    for _ in range(repeat):
+        attn_decode(q, kp, vp, table.reshape(B, pages), seqlens, causal=True)
+    torch.cuda.synchronize()
+    code, where = device_status()
+    print(f"paged decode B={B} Hq={Hq} Hkv={Hkv} L={L}: device status {code} (wait site {where})")
+    return 0 if code == 0 else 1
 
 
 def main(argv=None) -> int:
@@ -20,7 +39,10 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--repeat", type=int, default=1)
     ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--decode", action="store_true")
     args = ap.parse_args(argv)
+    if args.decode:
+        return decode_case(args.repeat)
     w = workload(args.workload)
     causal = w.causal[-1]
     q, k, v, *rest = (t.to("cuda") for t in make_inputs(w, with_do=w.backward))
