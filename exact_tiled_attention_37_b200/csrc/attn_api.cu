@@ -137,6 +137,14 @@ attn_status_t last_launch() {
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Streaming multiprocessors of the current device (148 on a B200).
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
 // ---------------------------------------------------------------- forward
 template <typename T, int D, int NS>
 attn_status_t launch_pingpong(const attn_tensor_t& q, const attn_tensor_t& k,
@@ -249,7 +257,15 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   cudaEvent_t ev1 = static_cast<cudaEvent_t>(g_bwd_ev_stop.exchange(nullptr));
   const bool timed = ev0 && ev1;
   if (timed && cudaEventRecord(ev0, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  kkv<<<dim3(p.Hkv, p.B, tiles), CKV::THREADS, CKV::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+  // persistent: one CTA per SM (at most one per work item)
+  const long long kv_items = static_cast<long long>(p.Hkv) * p.B * tiles;
+  const unsigned kv_ctas = static_cast<unsigned>(std::min<long long>(kv_items, sm_count()));
+  // dK, dV as [B, Hkv, N, D] for the TMA stores of the epilogue ({64, 32} boxes)
+  CUtensorMap tdk, tdv;
+  const attn_tensor_t dk_t{p.dk, p.dksb, p.dksh, p.dksn}, dv_t{p.dv, p.dvsb, p.dvsh, p.dvsn};
+  if ((s = make_map(&tdk, dk_t, p.B, p.Hkv, p.N, D, 2, 32)) != ATTN_OK) return s;
+  if ((s = make_map(&tdv, dv_t, p.B, p.Hkv, p.N, D, 2, 32)) != ATTN_OK) return s;
+  kkv<<<kv_ctas, CKV::THREADS, CKV::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   if ((s = last_launch()) != ATTN_OK) return s;
   if (timed && cudaEventRecord(ev1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   kq<<<dim3(p.Hq, p.B, tiles), CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);

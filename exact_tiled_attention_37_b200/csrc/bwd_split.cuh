@@ -57,6 +57,47 @@ __device__ __forceinline__ void tmem_row_to_bf16(uint32_t taddr, __nv_bfloat16* 
   }
 }
 
+// Epilogue of this warp's 32 TMEM lanes (rows row0 .. row0 + 31 of the
+// output) through TMA stores: NC fp32 columns times mul become bf16, 64
+// columns (one {64, 32} box) at a time, written into the warp's 4 KB staging
+// region in the box's 128-byte-swizzled layout (row i at 128 i, 16-byte unit
+// u at unit u ^ (i & 7)); lane 0 stores each box at (col0 + c, row0, h, b).
+// The last box may still be reading the staging region on return.
+template <int NC>
+__device__ __forceinline__ void tmem_rows_tma_store(uint32_t taddr, uint8_t* stage,
+                                                    const CUtensorMap* m, int col0, int row0,
+                                                    int h, int b, float mul) {
+  static_assert(NC % 64 == 0, "64-column boxes");
+  const int lane = threadIdx.x & 31;
+  uint8_t* srow = stage + lane * 128;
+#pragma unroll 1
+  for (int c = 0; c < NC; c += 64) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(taddr + c, r0);
+    tmem_ld32(taddr + c + 32, r1);
+    tmem_wait_ld();
+    if (c > 0) {
+      if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging region
+      __syncwarp();
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t* x = u < 4 ? r0 + 8 * u : r1 + 8 * (u - 4);
+      const uint4 w = make_uint4(pack_bf16x2(u2f(x[0]) * mul, u2f(x[1]) * mul),
+                                 pack_bf16x2(u2f(x[2]) * mul, u2f(x[3]) * mul),
+                                 pack_bf16x2(u2f(x[4]) * mul, u2f(x[5]) * mul),
+                                 pack_bf16x2(u2f(x[6]) * mul, u2f(x[7]) * mul));
+      *reinterpret_cast<uint4*>(srow + ((u ^ (lane & 7)) << 4)) = w;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_4d(m, smem_u32(stage), col0 + c, row0, h, b);
+      bulk_commit();
+    }
+  }
+}
+
 // Stores CW/2 packed columns (CW = 32 or 64).
 template <int CW>
 __device__ __forceinline__ void tmem_store_packed(uint32_t taddr, const uint32_t (&pk)[CW / 2]) {
@@ -355,6 +396,22 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   }
 }
 
+// Round r of a persistent CTA's static schedule: items sorted by decreasing
+// work are dealt out in snake order (CTA c takes item r G + c in even
+// rounds, r G + G - 1 - c in odd ones, G CTAs), which evens out the per-CTA
+// sums; -1 past the last item.
+__device__ __forceinline__ int snake_item(int r, int cta, int ctas, int items) {
+  const int idx = r * ctas + ((r & 1) ? ctas - 1 - cta : cta);
+  return idx < items ? idx : -1;
+}
+
+// One work item of the dK/dV kernel: a 128-row key tile of one key/value
+// head, and the query tiles (of every query head of its group) that see it.
+struct KVItem {
+  bool valid;
+  int hk, b, kt, k0, i_first, per_head, E;
+};
+
 // ============================================================ dK / dV kernel
 // P^T goes through shared memory (the A operand of dV += P^T dO_i) so that
 // S^T of the next query tile can be computed as soon as the elementwise
@@ -376,17 +433,17 @@ struct BwdKVCfg {
   static constexpr int S_P = S_DO + NQS * TILE;                // P^T: 128 key rows x 128 queries bf16
   static constexpr int S_STAT = S_P + 128 * 256;               // [NQS] lse2[128], delta[128]
   static constexpr int S_BAR = S_STAT + NQS * 1024;
-  // kv, q_full[NQS] (Q_i and its row statistics), q_empty[NQS], do_full[NQS],
-  // do_empty[NQS], s, s_consumed, dp, p, p_empty, ds, kv_done, done
+  // kv (K, V loaded), q_full[NQS] (Q_i and its row statistics), q_empty[NQS],
+  // do_full[NQS], do_empty[NQS], s, s_consumed, dp, p, p_empty, ds,
+  // kv_done (dK, dV complete), done, kv_empty (K, V no longer read)
   static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NQS, B_OF = 1 + 2 * NQS,
                        B_OE = 1 + 3 * NQS, B_S = 1 + 4 * NQS, B_SC = 2 + 4 * NQS,
                        B_DP = 3 + 4 * NQS, B_P = 4 + 4 * NQS, B_PE = 5 + 4 * NQS,
                        B_DS = 6 + 4 * NQS, B_KVD = 7 + 4 * NQS, B_DONE = 8 + 4 * NQS,
-                       NBAR = 9 + 4 * NQS;
+                       B_KVE = 9 + 4 * NQS, NBAR = 10 + 4 * NQS;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int S_META = S_MISC + 16;   // [NQS] entry index of each stage
-  static constexpr int S_CNT = S_META + 16;    // number of computed entries
-  static constexpr int LAYOUT = S_CNT + 16;
+  static constexpr int LAYOUT = S_META + 16;
   // dynamic shared memory: the layout plus as much of the 1024-byte alignment
   // slack as the per-block limit leaves (the kernel checks the actual slack)
   static constexpr int SMEM_BYTES = LAYOUT + 1024 <= 232448 ? LAYOUT + 1024 : 232448;
@@ -401,7 +458,8 @@ template <int D, int NQS, int NWG>
 __global__ void __launch_bounds__(128 * NWG + 64, 1)
     bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using C = BwdKVCfg<D, NQS, NWG>;
   constexpr int CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
@@ -419,30 +477,50 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.z;  // causal key tile 0 (the most work) is dispatched first
-  const int hk = blockIdx.x, b = blockIdx.y;
-  const int k0 = kt * C::BC;
-  // queries that see any key of [k0, k0 + BC): key j is visible to query i iff
-  // j - wr <= i <= j + wl
-  const int q_lo = p.wr < 0 ? 0 : max(0, k0 - p.wr);
-  const int q_hi = p.wl < 0 ? p.N : min(p.N, min(p.N, k0 + C::BC) + p.wl);
-  const int i_first = q_lo / C::BR;
-  const int per_head = (q_hi + C::BR - 1) / C::BR - i_first;
-  // entries: query heads of the group x query tiles in the window range, in
-  // that order; with a block-sparse mask only the entries whose tile pair is
-  // marked are computed
-  const int E = per_head * p.group;
+  // Persistent CTAs: work items (key/value head, batch, key tile) ordered key
+  // tile slowest (causal key tile 0, the most work, first) and dealt out in
+  // snake order, one per CTA per round.
+  const int nkt = (p.N + C::BC - 1) / C::BC;
+  const int items = p.Hkv * p.B * nkt;
   const bool sparse = p.bmask != nullptr;
-  auto head_of = [&](int e) { return hk * p.group + e / per_head; };
-  auto qtile_of = [&](int e) { return i_first + e % per_head; };
-  auto marked = [&](int e) -> bool {
-    return p.bmask[((static_cast<long long>(b) * p.Hq + head_of(e)) * p.nt + qtile_of(e)) * p.nt +
-                   kt] != 0;
+  auto item_of = [&](int r) -> KVItem {
+    const int w = snake_item(r, blockIdx.x, gridDim.x, items);
+    KVItem I;
+    I.valid = w >= 0;
+    if (!I.valid) return I;
+    I.kt = w / (p.Hkv * p.B);
+    I.b = (w / p.Hkv) % p.B;
+    I.hk = w % p.Hkv;
+    I.k0 = I.kt * C::BC;
+    // queries that see any key of [k0, k0 + BC): key j is visible to query i
+    // iff j - wr <= i <= j + wl
+    const int q_lo = p.wr < 0 ? 0 : max(0, I.k0 - p.wr);
+    const int q_hi = p.wl < 0 ? p.N : min(p.N, min(p.N, I.k0 + C::BC) + p.wl);
+    I.i_first = q_lo / C::BR;
+    I.per_head = (q_hi + C::BR - 1) / C::BR - I.i_first;
+    // entries: query heads of the group x query tiles in the window range, in
+    // that order; with a block-sparse mask only the marked tile pairs count
+    I.E = I.per_head * p.group;
+    return I;
+  };
+  auto head_of = [&](const KVItem& I, int e) { return I.hk * p.group + e / I.per_head; };
+  auto qtile_of = [&](const KVItem& I, int e) { return I.i_first + e % I.per_head; };
+  auto marked = [&](const KVItem& I, int e) -> bool {
+    return p.bmask[((static_cast<long long>(I.b) * p.Hq + head_of(I, e)) * p.nt + qtile_of(I, e)) *
+                       p.nt +
+                   I.kt] != 0;
+  };
+  // computed entries of an item (whole warp)
+  auto count = [&](const KVItem& I) -> int {
+    if (!sparse) return I.E;
+    int c = 0;
+    for (int base = 0; base < I.E; base += 32)
+      c += __popc(__ballot_sync(0xffffffffu, base + lane < I.E && marked(I, base + lane)));
+    return c;
   };
   volatile int* meta = reinterpret_cast<volatile int*>(smem + C::S_META);
-  int* cnt_smem = reinterpret_cast<int*>(smem + C::S_CNT);
 #ifdef ETA_TRACE
-  const int tcta = (blockIdx.x == 0 && blockIdx.y == 0) ? (kt == 0 ? 0 : (kt == 16 ? 1 : -1)) : -1;
+  const int tcta = blockIdx.x == 0 ? 0 : (blockIdx.x == 1 ? 1 : -1);
 #else
   const int tcta = -1;
 #endif
@@ -450,6 +528,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_KV), 1);
+    mbar_init(BAR(C::B_KVE), 1);
     for (int s = 0; s < NQS; ++s) {
       mbar_init(BAR(C::B_QF + s), 1);
       mbar_init(BAR(C::B_QE + s), 1);
@@ -465,7 +544,6 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     mbar_init(BAR(C::B_KVD), 1);
     mbar_init(BAR(C::B_DONE), 1);
     *abort_flag = 0u;
-    *cnt_smem = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -478,20 +556,14 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
-  int n = E;  // iterations: computed entries
-  if (sparse) {
-    int c = 0;
-    for (int e = threadIdx.x; e < E; e += C::THREADS) c += marked(e) ? 1 : 0;
-    if (c) atomicAdd(cnt_smem, c);
-    __syncthreads();
-    n = *cnt_smem;
-  }
+  // Barrier phases run on across items: g counts computed entries (query
+  // tiles) of all items so far, and the K/V and dK/dV barriers count items
+  // that compute at least one entry.
 
   if (warp < 4 * NWG) {
     // ---------------------------------------- P^T, dS^T rows (thread j = key row j)
     const int par = warp >> 2;           // query columns [CW par, CW par + CW) of each tile
     const int j = threadIdx.x & 127;
-    const int jg = k0 + j;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t st_addr = tmem + lane_base + C::T_ST + CW * par;
     const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + CW * par;
@@ -500,103 +572,133 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     uint8_t* prow = smem + C::S_P + ((CW * par) / 64) * C::CHUNK + j * 128;
     const int g0 = ((CW * par) % 64) / 8;
     const int swz = j & 7;
+    // NWG = 2: this warp's P^T rows (32 rows x 128 bytes) also stage its
+    // dK/dV rows for the TMA stores of the epilogue
+    constexpr bool kTmaEpi = NWG == 2;
+    uint8_t* stage = smem + C::S_P + par * C::CHUNK + (warp & 3) * 32 * 128;
+    bool store_pending = false;  // a TMA store may still read `stage`
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      const int stage = it % NQS;
-      if (!W.wait_warp(BAR(C::B_S), it & 1, 130)) { ok = false; break; }
-      // (complete already: S^T was computed from this stage) orders the reads of
-      // the stage's entry index and row statistics after the producer's writes
-      if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 134)) { ok = false; break; }
-      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 0);
-      tc_fence_after();
-      float pr[CW];
-      tmem_load_row<CW>(st_addr, pr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_SC));  // S^T may be overwritten
-      const float* lse2 =
-          reinterpret_cast<const float*>(smem + C::S_STAT + stage * 1024) + CW * par;
-      const float* dlt = lse2 + 128;
-      const int ig0 = qtile_of(meta[stage]) * C::BR + CW * par;
-      // window: query ig0 + i sees key jg iff jg - wr <= ig0 + i <= jg + wl
-      const int ilo = p.wr < 0 ? -(1 << 30) : jg - p.wr - ig0;
-      const int ihi = p.wl < 0 ? (1 << 30) : jg + p.wl - ig0;
-      const float2 c2 = make_float2(p.c, p.c);
-      if (ilo <= 0 && ihi >= CW - 1) {
+    int g = 0, nkvd = 0;
+    for (int r = 0; ok; ++r) {
+      const KVItem I = item_of(r);
+      if (!I.valid) break;
+      const int n = count(I);
+      const int jg = I.k0 + j;
+      for (int it = 0; it < n; ++it, ++g) {
+        const int stage = g % NQS;
+        if (!W.wait_warp(BAR(C::B_S), g & 1, 130)) { ok = false; break; }
+        // (complete already: S^T was computed from this stage) orders the reads of
+        // the stage's entry index and row statistics after the producer's writes
+        if (!W.wait_warp(BAR(C::B_QF + stage), (g / NQS) & 1, 134)) { ok = false; break; }
+        if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 0);
+        tc_fence_after();
+        float pr[CW];
+        tmem_load_row<CW>(st_addr, pr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_SC));  // S^T may be overwritten
+        const float* lse2 =
+            reinterpret_cast<const float*>(smem + C::S_STAT + stage * 1024) + CW * par;
+        const float* dlt = lse2 + 128;
+        const int ig0 = qtile_of(I, meta[stage]) * C::BR + CW * par;
+        // window: query ig0 + i sees key jg iff jg - wr <= ig0 + i <= jg + wl
+        const int ilo = p.wr < 0 ? -(1 << 30) : jg - p.wr - ig0;
+        const int ihi = p.wl < 0 ? (1 << 30) : jg + p.wl - ig0;
+        const float2 c2 = make_float2(p.c, p.c);
+        if (ilo <= 0 && ihi >= CW - 1) {
 #pragma unroll
-        for (int i = 0; i < CW; i += 2) {
-          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + i);
-          const float2 x = ffma2(make_float2(pr[i], pr[i + 1]), c2, make_float2(-l2.x, -l2.y));
-          pr[i] = ex2(x.x);
-          pr[i + 1] = ex2(x.y);
+          for (int i = 0; i < CW; i += 2) {
+            const float2 l2 = *reinterpret_cast<const float2*>(lse2 + i);
+            const float2 x = ffma2(make_float2(pr[i], pr[i + 1]), c2, make_float2(-l2.x, -l2.y));
+            pr[i] = ex2(x.x);
+            pr[i + 1] = ex2(x.y);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < CW; i += 2) {
+            const float2 l2 = *reinterpret_cast<const float2*>(lse2 + i);
+            const float2 x = ffma2(make_float2(pr[i], pr[i + 1]), c2, make_float2(-l2.x, -l2.y));
+            pr[i] = (i < ilo || i > ihi) ? 0.f : ex2(x.x);
+            pr[i + 1] = (i + 1 < ilo || i + 1 > ihi) ? 0.f : ex2(x.y);
+          }
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < CW; i += 2) {
-          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + i);
-          const float2 x = ffma2(make_float2(pr[i], pr[i + 1]), c2, make_float2(-l2.x, -l2.y));
-          pr[i] = (i < ilo || i > ihi) ? 0.f : ex2(x.x);
-          pr[i + 1] = (i + 1 < ilo || i + 1 > ihi) ? 0.f : ex2(x.y);
+        // the dV MMA of the previous tile must be done reading P^T (and the
+        // epilogue's TMA stores with the staging rows)
+        if (!W.wait_warp(BAR(C::B_PE), (g & 1) ^ 1, 133)) { ok = false; break; }
+        if (kTmaEpi && store_pending) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          store_pending = false;
         }
-      }
-      // the dV MMA of the previous tile must be done reading P^T
-      if (!W.wait_warp(BAR(C::B_PE), (it & 1) ^ 1, 133)) { ok = false; break; }
 #pragma unroll
-      for (int g = 0; g < CW / 8; ++g) {
-        const uint4 w = make_uint4(pack_bf16x2(pr[8 * g + 0], pr[8 * g + 1]),
-                                   pack_bf16x2(pr[8 * g + 2], pr[8 * g + 3]),
-                                   pack_bf16x2(pr[8 * g + 4], pr[8 * g + 5]),
-                                   pack_bf16x2(pr[8 * g + 6], pr[8 * g + 7]));
-        *reinterpret_cast<uint4*>(prow + (((g0 + g) ^ swz) << 4)) = w;
-      }
-      fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_P));
-      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 1);
-      if (!W.wait_warp(BAR(C::B_DP), it & 1, 131)) { ok = false; break; }
-      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 2);
-      tc_fence_after();
-#pragma unroll
-      for (int h2 = 0; h2 < CW / 32; ++h2) {
-        uint32_t rd[32];
-        tmem_ld32(dpt_addr + 32 * h2, rd);
-        tmem_wait_ld();
-        uint32_t dk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int c = 32 * h2 + i;
-          const float2 dd = *reinterpret_cast<const float2*>(dlt + c);
-          const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
-          dk[i / 2] = pack_bf16x2(pr[c] * g.x, pr[c + 1] * g.y);
+        for (int gr = 0; gr < CW / 8; ++gr) {
+          const uint4 w = make_uint4(pack_bf16x2(pr[8 * gr + 0], pr[8 * gr + 1]),
+                                     pack_bf16x2(pr[8 * gr + 2], pr[8 * gr + 3]),
+                                     pack_bf16x2(pr[8 * gr + 4], pr[8 * gr + 5]),
+                                     pack_bf16x2(pr[8 * gr + 6], pr[8 * gr + 7]));
+          *reinterpret_cast<uint4*>(prow + (((g0 + gr) ^ swz) << 4)) = w;
         }
-        // dS^T of columns [32 h2, 32 h2 + 32) -> packed columns 16 h2 .. 16 h2 + 15
-        // (already read: each half lies below the columns still to be loaded)
-        tmem_st16(dpt_addr + 16 * h2, dk);
+        fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_P));
+        if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 1);
+        if (!W.wait_warp(BAR(C::B_DP), g & 1, 131)) { ok = false; break; }
+        if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 2);
+        tc_fence_after();
+#pragma unroll
+        for (int h2 = 0; h2 < CW / 32; ++h2) {
+          uint32_t rd[32];
+          tmem_ld32(dpt_addr + 32 * h2, rd);
+          tmem_wait_ld();
+          uint32_t dk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const int c = 32 * h2 + i;
+            const float2 dd = *reinterpret_cast<const float2*>(dlt + c);
+            const float2 gd = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
+            dk[i / 2] = pack_bf16x2(pr[c] * gd.x, pr[c + 1] * gd.y);
+          }
+          // dS^T of columns [32 h2, 32 h2 + 32) -> packed columns 16 h2 .. 16 h2 + 15
+          // (already read: each half lies below the columns still to be loaded)
+          tmem_st16(dpt_addr + 16 * h2, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_DS));
+        if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 3);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_DS));
-      if (j == 0) ETA_TRACE_AT(tcta, par & 1, it, 3);
+      if (!ok) break;
+      // epilogue: the first NWG/2 warpgroups store dV, the others dK (x scale),
+      // D / (NWG/2) columns each
+      constexpr int NG = NWG / 2, DC = D / NG;
+      const int which = par / NG, part = par % NG;
+      __nv_bfloat16* row =
+          which == 0 ? static_cast<__nv_bfloat16*>(p.dv) + I.b * p.dvsb + I.hk * p.dvsh +
+                           static_cast<long long>(jg) * p.dvsn + DC * part
+                     : static_cast<__nv_bfloat16*>(p.dk) + I.b * p.dksb + I.hk * p.dksh +
+                           static_cast<long long>(jg) * p.dksn + DC * part;
+      const bool valid = jg < p.N;
+      if (n > 0) {
+        if (!W.wait_warp(BAR(C::B_KVD), nkvd & 1, 132)) { ok = false; break; }
+        ++nkvd;
+        tc_fence_after();
+        const uint32_t src = tmem + lane_base + (which ? C::T_DK : C::T_DV) + DC * part;
+        if constexpr (kTmaEpi) {
+          tmem_rows_tma_store<DC>(src, stage, which ? &tm_dk : &tm_dv, DC * part,
+                                  I.k0 + (warp & 3) * 32, I.hk, I.b, which ? p.scale : 1.f);
+          store_pending = true;
+        } else {
+          tmem_row_to_bf16<DC>(src, row, which ? p.scale : 1.f, valid);
+        }
+      } else if (valid) {
+        // no query sees these keys: their gradients are zero
+        for (int c = 0; c < DC / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
-    // epilogue: the first NWG/2 warpgroups store dV, the others dK (x scale),
-    // D / (NWG/2) columns each
-    constexpr int NG = NWG / 2, DC = D / NG;
-    const int which = par / NG, part = par % NG;
-    __nv_bfloat16* row =
-        which == 0 ? static_cast<__nv_bfloat16*>(p.dv) + b * p.dvsb + hk * p.dvsh +
-                         static_cast<long long>(jg) * p.dvsn + DC * part
-                   : static_cast<__nv_bfloat16*>(p.dk) + b * p.dksb + hk * p.dksh +
-                         static_cast<long long>(jg) * p.dksn + DC * part;
-    const bool valid = jg < p.N;
-    if (ok && n > 0 && W.wait_warp(BAR(C::B_KVD), 0, 132)) {
-      tc_fence_after();
-      tmem_row_to_bf16<DC>(tmem + lane_base + (which ? C::T_DK : C::T_DV) + DC * part, row,
-                           which ? p.scale : 1.f, valid);
-    } else if (n == 0 && valid) {
-      // no query sees these keys: their gradients are zero
-      for (int c = 0; c < DC / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
-    }
+    // the staging rows must stay untouched until the last TMA store has read them
+    if (kTmaEpi && store_pending && lane == 0) bulk_wait_read_all();
+    __syncwarp();
   } else if (warp == C::PRODUCER) {
     // ---------------------------------------- TMA producer (the whole warp scans
     // 32 entries at a time; lane 0 waits and issues the copies)
@@ -605,61 +707,79 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_expect_tx(BAR(C::B_KV), 2 * C::TILE);
-      for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d(sbase + C::S_K + c * C::CHUNK, &tm_k, BAR(C::B_KV), c * 64, k0, hk, b);
-        tma_load_4d(sbase + C::S_V + c * C::CHUNK, &tm_v, BAR(C::B_KV), c * 64, k0, hk, b);
-      }
     }
     // dO_i and Q_i have their own barriers: dO_i's slot frees earlier (after
-    // dV) and is refilled first; Q_i (needed first, by S^T) follows.
-    int it = 0, issued_q = 0, issued_do = 0;
+    // dV) and is refilled first; Q_i (needed first, by S^T) follows.  An
+    // item's K and V are loaded (once the previous item's last S^T and dP^T
+    // are done with them) before its first computed entry.
+    int g = 0, m = 0, issued_q = 0, issued_do = 0;
     bool pok = true;
-    for (int base = 0; pok && it < n && base < E; base += 32) {
-      const int e_l = base + lane;
-      const bool on = e_l < E && (!sparse || marked(e_l));
-      uint32_t pend = __ballot_sync(0xffffffffu, on);
-      while (pend != 0u && it < n) {
-        const int e = base + __ffs(pend) - 1;
-        pend &= pend - 1u;
-        if (lane == 0) {
-          const int stage = it % NQS;
-          const uint32_t par_empty = ((it / NQS) & 1) ^ 1;
-          const int h = head_of(e);
-          const int ig0 = qtile_of(e) * C::BR;
-          if (!W.wait(BAR(C::B_OE + stage), par_empty, 143)) {
-            pok = false;
-          } else {
-            const uint32_t ofull = BAR(C::B_OF + stage);
-            mbar_expect_tx(ofull, C::TILE);
-            for (int c = 0; c < C::NCHUNK; ++c)
-              tma_load_4d(sbase + C::S_DO + stage * C::TILE + c * C::CHUNK, &tm_do, ofull, c * 64,
-                          ig0, h, b);
-            issued_do = it + 1;
-            if (!W.wait(BAR(C::B_QE + stage), par_empty, 140)) {
+    for (int r = 0; pok; ++r) {
+      const KVItem I = item_of(r);
+      if (!I.valid) break;
+      bool kv_loaded = false;
+      for (int base = 0; pok && base < I.E; base += 32) {
+        const int e_l = base + lane;
+        const bool on = e_l < I.E && (!sparse || marked(I, e_l));
+        uint32_t pend = __ballot_sync(0xffffffffu, on);
+        while (pend != 0u) {
+          const int e = base + __ffs(pend) - 1;
+          pend &= pend - 1u;
+          if (lane == 0) {
+            if (!kv_loaded) {
+              if (m > 0 && !W.wait(BAR(C::B_KVE), (m - 1) & 1, 145)) {
+                pok = false;
+              } else {
+                mbar_expect_tx(BAR(C::B_KV), 2 * C::TILE);
+                for (int c = 0; c < C::NCHUNK; ++c) {
+                  tma_load_4d(sbase + C::S_K + c * C::CHUNK, &tm_k, BAR(C::B_KV), c * 64, I.k0,
+                              I.hk, I.b);
+                  tma_load_4d(sbase + C::S_V + c * C::CHUNK, &tm_v, BAR(C::B_KV), c * 64, I.k0,
+                              I.hk, I.b);
+                }
+                ++m;
+              }
+              kv_loaded = true;
+            }
+            const int stage = g % NQS;
+            const uint32_t par_empty = ((g / NQS) & 1) ^ 1;
+            const int h = head_of(I, e);
+            const int ig0 = qtile_of(I, e) * C::BR;
+            if (!pok) {
+            } else if (!W.wait(BAR(C::B_OE + stage), par_empty, 143)) {
               pok = false;
             } else {
-              ETA_TRACE_AT(tcta, 3, it, 0);
-              meta[stage] = e;
-              const uint32_t full = BAR(C::B_QF + stage);
-              mbar_expect_tx(full, C::TILE + 1024);
+              const uint32_t ofull = BAR(C::B_OF + stage);
+              mbar_expect_tx(ofull, C::TILE);
               for (int c = 0; c < C::NCHUNK; ++c)
-                tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full, c * 64,
-                            ig0, h, b);
-              const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
-              bulk_load(sbase + C::S_STAT + stage * 1024, p.lse2 + srow, 512, full);
-              bulk_load(sbase + C::S_STAT + stage * 1024 + 512, p.delta + srow, 512, full);
-              issued_q = it + 1;
+                tma_load_4d(sbase + C::S_DO + stage * C::TILE + c * C::CHUNK, &tm_do, ofull,
+                            c * 64, ig0, h, I.b);
+              issued_do = g + 1;
+              if (!W.wait(BAR(C::B_QE + stage), par_empty, 140)) {
+                pok = false;
+              } else {
+                ETA_TRACE_AT(tcta, 3, g, 0);
+                meta[stage] = e;
+                const uint32_t full = BAR(C::B_QF + stage);
+                mbar_expect_tx(full, C::TILE + 1024);
+                for (int c = 0; c < C::NCHUNK; ++c)
+                  tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full,
+                              c * 64, ig0, h, I.b);
+                const long long srow = static_cast<long long>(I.b * p.Hq + h) * p.Npad + ig0;
+                bulk_load(sbase + C::S_STAT + stage * 1024, p.lse2 + srow, 512, full);
+                bulk_load(sbase + C::S_STAT + stage * 1024 + 512, p.delta + srow, 512, full);
+                issued_q = g + 1;
+              }
             }
           }
+          pok = __shfl_sync(0xffffffffu, pok, 0);
+          if (!pok) break;
+          ++g;
         }
-        pok = __shfl_sync(0xffffffffu, pok, 0);
-        if (!pok) break;
-        ++it;
       }
     }
     if (lane == 0) {
-      W.drain(BAR(C::B_KV), 0, 141);
+      if (m > 0) W.drain(BAR(C::B_KV), static_cast<uint32_t>(m - 1) & 1u, 141);
       for (int s = 0; s < NQS && s < issued_q; ++s) {
         const int last = s + ((issued_q - 1 - s) / NQS) * NQS;
         W.drain(BAR(C::B_QF + s), static_cast<uint32_t>(last / NQS) & 1u, 142);
@@ -677,9 +797,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     const SDesc dK = sdesc_base(sbase + C::S_K, 16, 1024);
     const SDesc dV = sdesc_base(sbase + C::S_V, 16, 1024);
     const SDesc dP = sdesc_base(sbase + C::S_P, 16, 1024);
-    auto issue_s = [&](int it) -> bool {
-      const int stage = it % NQS;
-      if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 150)) return false;
+    auto issue_s = [&](int g) -> bool {
+      const int stage = g % NQS;
+      if (!W.wait_warp(BAR(C::B_QF + stage), (g / NQS) & 1, 150)) return false;
       tc_fence_after();
       const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, 16, 1024);
 #pragma unroll
@@ -690,9 +810,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       mma_commit_w(BAR(C::B_S));
       return true;
     };
-    auto issue_dp = [&](int it) -> bool {
-      const int stage = it % NQS;
-      if (!W.wait_warp(BAR(C::B_OF + stage), (it / NQS) & 1, 156)) return false;
+    auto issue_dp = [&](int g) -> bool {
+      const int stage = g % NQS;
+      if (!W.wait_warp(BAR(C::B_OF + stage), (g / NQS) & 1, 156)) return false;
       tc_fence_after();
       const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, 16, 1024);
 #pragma unroll
@@ -703,45 +823,61 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       mma_commit_w(BAR(C::B_DP));
       return true;
     };
-    bool ok = W.wait_warp(BAR(C::B_KV), 0, 151);
-    if (ok && n > 0) ok = issue_s(0) && issue_dp(0);
-    for (int it = 0; ok && it < n; ++it) {
-      const int stage = it % NQS;
-      const uint32_t acc0 = it > 0 ? 1u : 0u;
-      ETA_TRACE_AT(tcta, 2, it, 0);
-      // S^T of the next tile once the elementwise warps have loaded this one
-      if (it + 1 < n) {
-        if (!W.wait_warp(BAR(C::B_SC), it & 1, 155)) { ok = false; break; }
-        ETA_TRACE_AT(tcta, 3, it, 1);
-        if (!issue_s(it + 1)) { ok = false; break; }
+    bool ok = true;
+    int g = 0, nkv = 0;
+    for (int r = 0; ok; ++r) {
+      const KVItem I = item_of(r);
+      if (!I.valid) break;
+      const int n = count(I);
+      if (n == 0) continue;
+      if (!W.wait_warp(BAR(C::B_KV), nkv & 1, 151)) { ok = false; break; }
+      ++nkv;
+      // the item's first S^T overwrites S^T of the previous item's last entry
+      if (g > 0 && !W.wait_warp(BAR(C::B_SC), (g - 1) & 1, 157)) { ok = false; break; }
+      if (!issue_s(g) || !issue_dp(g)) { ok = false; break; }
+      if (n == 1) mma_commit_w(BAR(C::B_KVE));  // K and V are not read again
+      for (int it = 0; it < n; ++it, ++g) {
+        const int stage = g % NQS;
+        const uint32_t acc0 = it > 0 ? 1u : 0u;
+        ETA_TRACE_AT(tcta, 2, g, 0);
+        // S^T of the next tile once the elementwise warps have loaded this one
+        if (it + 1 < n) {
+          if (!W.wait_warp(BAR(C::B_SC), g & 1, 155)) { ok = false; break; }
+          ETA_TRACE_AT(tcta, 3, g, 1);
+          if (!issue_s(g + 1)) { ok = false; break; }
+        }
+        ETA_TRACE_AT(tcta, 2, g, 1);
+        // dV += P^T dO_i: A = P^T (K-major shared memory), B = dO_i (MN-major)
+        if (!W.wait_warp(BAR(C::B_P), g & 1, 152)) { ok = false; break; }
+        ETA_TRACE_AT(tcta, 2, g, 2);
+        tc_fence_after();
+        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, C::CHUNK, 1024);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss_w(tmem + C::T_DV, sdesc_at(dP, (ks >> 2) * C::CHUNK + (ks & 3) * 32),
+                   sdesc_at(ddo, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
+        mma_commit_w(BAR(C::B_PE));
+        mma_commit_w(BAR(C::B_OE + stage));  // dO_i is not read again
+        ETA_TRACE_AT(tcta, 3, g, 2);
+        // dK += dS^T Q_i with dS^T read from TMEM
+        if (!W.wait_warp(BAR(C::B_DS), g & 1, 153)) { ok = false; break; }
+        ETA_TRACE_AT(tcta, 2, g, 3);
+        tc_fence_after();
+        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, C::CHUNK, 1024);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_w(tmem + C::T_DK, tmem + C::T_DPT + packed_col<CW>(ks), sdesc_at(dq, ks * 2048),
+                   id_kv, ks > 0 ? 1u : acc0);
+        mma_commit_w(BAR(C::B_QE + stage));  // Q_i (and its statistics) are not read again
+        if (it + 1 < n) {
+          if (!issue_dp(g + 1)) { ok = false; break; }
+          if (it + 2 == n) mma_commit_w(BAR(C::B_KVE));  // K and V are not read again
+        }
+        ETA_TRACE_AT(tcta, 3, g, 3);
       }
-      ETA_TRACE_AT(tcta, 2, it, 1);
-      // dV += P^T dO_i: A = P^T (K-major shared memory), B = dO_i (MN-major)
-      if (!W.wait_warp(BAR(C::B_P), it & 1, 152)) { ok = false; break; }
-      ETA_TRACE_AT(tcta, 2, it, 2);
-      tc_fence_after();
-      const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::TILE, C::CHUNK, 1024);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_ss_w(tmem + C::T_DV, sdesc_at(dP, (ks >> 2) * C::CHUNK + (ks & 3) * 32),
-                 sdesc_at(ddo, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-      mma_commit_w(BAR(C::B_PE));
-      mma_commit_w(BAR(C::B_OE + stage));  // dO_i is not read again
-      ETA_TRACE_AT(tcta, 3, it, 2);
-      // dK += dS^T Q_i with dS^T read from TMEM
-      if (!W.wait_warp(BAR(C::B_DS), it & 1, 153)) { ok = false; break; }
-      ETA_TRACE_AT(tcta, 2, it, 3);
-      tc_fence_after();
-      const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::TILE, C::CHUNK, 1024);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_ts_w(tmem + C::T_DK, tmem + C::T_DPT + packed_col<CW>(ks), sdesc_at(dq, ks * 2048),
-                 id_kv, ks > 0 ? 1u : acc0);
-      mma_commit_w(BAR(C::B_QE + stage));  // Q_i (and its statistics) are not read again
-      if (it + 1 < n && !issue_dp(it + 1)) { ok = false; break; }
-      ETA_TRACE_AT(tcta, 3, it, 3);
+      if (!ok) break;
+      mma_commit_w(BAR(C::B_KVD));  // dK, dV of this item complete
     }
-    if (ok) mma_commit_w(BAR(C::B_KVD));
     mma_commit_w(BAR(C::B_DONE));
     W.drain(BAR(C::B_DONE), 0, 154);
     __syncwarp();

@@ -166,6 +166,17 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// 4-D tiled store of a shared-memory box to the tensor described by `m` at
+// coordinates (c0, c1, c2, c3), in the issuing thread's bulk group; elements
+// outside the tensor are skipped.  Coordinates must be non-negative.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, uint32_t ssrc, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(ssrc), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 // Tiled bulk reduction (fp32 add) of a shared-memory box into the 3-D tensor
 // described by `m` at coordinates (c0, c1, c2); elements outside the tensor
 // are skipped.  Coordinates must be non-negative.
