@@ -165,7 +165,11 @@ attn_status_t launch_pingpong(const attn_tensor_t& q, const attn_tensor_t& k,
   if (regs[p.bmask ? 1 : 0] != C::LAUNCH_REGS) return ATTN_ERR_CUDA;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
   dim3 grid(Hq, B, (N + 255) / 256);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  // O as [B, Hq, N, D] bf16 for the TMA stores of the epilogue ({64, 32} boxes)
+  CUtensorMap to;
+  const attn_tensor_t o_t{p.o, p.osb, p.osh, p.osn};
+  if ((s = make_map(&to, o_t, B, Hq, N, D, 2, 32)) != ATTN_OK) return s;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, to, p);
   return last_launch();
 }
 
@@ -268,7 +272,10 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   kkv<<<kv_ctas, CKV::THREADS, CKV::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   if ((s = last_launch()) != ATTN_OK) return s;
   if (timed && cudaEventRecord(ev1, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  kq<<<dim3(p.Hq, p.B, tiles), CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, p);
+  CUtensorMap tdq;
+  const attn_tensor_t dq_t{p.dq, p.dqsb, p.dqsh, p.dqsn};
+  if ((s = make_map(&tdq, dq_t, p.B, p.Hq, p.N, D, 2, 32)) != ATTN_OK) return s;
+  kq<<<dim3(p.Hq, p.B, tiles), CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
   return last_launch();
 }
 

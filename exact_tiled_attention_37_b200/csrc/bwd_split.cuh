@@ -57,47 +57,6 @@ __device__ __forceinline__ void tmem_row_to_bf16(uint32_t taddr, __nv_bfloat16* 
   }
 }
 
-// Epilogue of this warp's 32 TMEM lanes (rows row0 .. row0 + 31 of the
-// output) through TMA stores: NC fp32 columns times mul become bf16, 64
-// columns (one {64, 32} box) at a time, written into the warp's 4 KB staging
-// region in the box's 128-byte-swizzled layout (row i at 128 i, 16-byte unit
-// u at unit u ^ (i & 7)); lane 0 stores each box at (col0 + c, row0, h, b).
-// The last box may still be reading the staging region on return.
-template <int NC>
-__device__ __forceinline__ void tmem_rows_tma_store(uint32_t taddr, uint8_t* stage,
-                                                    const CUtensorMap* m, int col0, int row0,
-                                                    int h, int b, float mul) {
-  static_assert(NC % 64 == 0, "64-column boxes");
-  const int lane = threadIdx.x & 31;
-  uint8_t* srow = stage + lane * 128;
-#pragma unroll 1
-  for (int c = 0; c < NC; c += 64) {
-    uint32_t r0[32], r1[32];
-    tmem_ld32(taddr + c, r0);
-    tmem_ld32(taddr + c + 32, r1);
-    tmem_wait_ld();
-    if (c > 0) {
-      if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging region
-      __syncwarp();
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const uint32_t* x = u < 4 ? r0 + 8 * u : r1 + 8 * (u - 4);
-      const uint4 w = make_uint4(pack_bf16x2(u2f(x[0]) * mul, u2f(x[1]) * mul),
-                                 pack_bf16x2(u2f(x[2]) * mul, u2f(x[3]) * mul),
-                                 pack_bf16x2(u2f(x[4]) * mul, u2f(x[5]) * mul),
-                                 pack_bf16x2(u2f(x[6]) * mul, u2f(x[7]) * mul));
-      *reinterpret_cast<uint4*>(srow + ((u ^ (lane & 7)) << 4)) = w;
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_4d(m, smem_u32(stage), col0 + c, row0, h, b);
-      bulk_commit();
-    }
-  }
-}
-
 // Stores CW/2 packed columns (CW = 32 or 64).
 template <int CW>
 __device__ __forceinline__ void tmem_store_packed(uint32_t taddr, const uint32_t (&pk)[CW / 2]) {
@@ -143,6 +102,7 @@ template <int D, int NS, int NWG>
 __global__ void __launch_bounds__(128 * NWG + 64, 1)
     bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_dq,
                  const BwdParams p) {
   using C = BwdQCfg<D, NS, NWG>;
   constexpr int CW = C::CW;
@@ -281,7 +241,17 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
                          static_cast<long long>(qrow) * p.dqsn + DC * par;
     if (ok && n > 0 && W.wait_warp(BAR(C::B_DQ), 0, 102)) {
       tc_fence_after();
-      tmem_row_to_bf16<DC>(tmem + lane_base + C::T_DQ + DC * par, row, p.scale, qrow < p.N);
+      if constexpr (DC == 64) {
+        // through TMA stores, staged in this warp's rows of Q's chunk `par`
+        // (every MMA reading Q is complete)
+        uint8_t* stage = smem + C::SMEM_Q + par * C::CHUNK + (warp & 3) * 32 * 128;
+        tmem_rows_tma_store<DC>(tmem + lane_base + C::T_DQ + DC * par, stage, &tm_dq, DC * par,
+                                q0 + (warp & 3) * 32, h, b, p.scale);
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      } else {
+        tmem_row_to_bf16<DC>(tmem + lane_base + C::T_DQ + DC * par, row, p.scale, qrow < p.N);
+      }
     } else if (n == 0 && qrow < p.N) {
       // no key tile is computed for this query tile: dQ = 0
       for (int c = 0; c < DC / 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);

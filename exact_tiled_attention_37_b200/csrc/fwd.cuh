@@ -379,7 +379,8 @@ template <typename T, int D, int NS, bool SPARSE>
 __global__ void __launch_bounds__(384, 1)
     fwd_pingpong_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using C = PingPongCfg<T, D, NS>;
   using OutT = std::conditional_t<C::FP8, __nv_bfloat16, T>;  // e4m3 inputs give bf16 O
   extern __shared__ uint8_t smem_raw[];
@@ -525,7 +526,20 @@ __global__ void __launch_bounds__(384, 1)
       store_empty_row<OutT, D>(p, b, h, qrow);
     } else if (ok && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
       tc_fence_after();
-      store_row<OutT, D>(o_addr, p, b, h, qrow, m, l);
+      if constexpr (!C::FP8) {
+        // O / l through TMA stores, staged in this warp's rows of Q_t (every
+        // MMA reading Q_t is complete)
+        uint8_t* stage = smem + C::SMEM_Q + t * C::TILE + (warp & 3) * 32 * 128;
+        tmem_rows_tma_store<D>(o_addr, stage, &tm_o, 0, q0 + 128 * t + (warp & 3) * 32, h, b,
+                               l > 0.f ? p.o_mul / l : 0.f);
+        if (qrow < p.N)
+          p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] =
+              l > 0.f ? m * p.scale + logf(l) : -INFINITY;
+        if (lane == 0) bulk_wait_read_all();  // the staging rows stay valid until read
+        __syncwarp();
+      } else {
+        store_row<OutT, D>(o_addr, p, b, h, qrow, m, l);
+      }
     }
   } else if (warp == 8) {
     // ------------------------------------------------ TMA producer

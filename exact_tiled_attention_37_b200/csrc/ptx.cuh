@@ -492,5 +492,47 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Epilogue of this warp's 32 TMEM lanes (rows row0 .. row0 + 31 of the
+// output) through TMA stores: NC fp32 columns times mul become bf16, 64
+// columns (one {64, 32} box) at a time, written into the warp's 4 KB staging
+// region in the box's 128-byte-swizzled layout (row i at 128 i, 16-byte unit
+// u at unit u ^ (i & 7)); lane 0 stores each box at (col0 + c, row0, h, b).
+// The last box may still be reading the staging region on return.
+template <int NC>
+__device__ __forceinline__ void tmem_rows_tma_store(uint32_t taddr, uint8_t* stage,
+                                                    const CUtensorMap* m, int col0, int row0,
+                                                    int h, int b, float mul) {
+  static_assert(NC % 64 == 0, "64-column boxes");
+  const int lane = threadIdx.x & 31;
+  uint8_t* srow = stage + lane * 128;
+#pragma unroll 1
+  for (int c = 0; c < NC; c += 64) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(taddr + c, r0);
+    tmem_ld32(taddr + c + 32, r1);
+    tmem_wait_ld();
+    if (c > 0) {
+      if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging region
+      __syncwarp();
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t* x = u < 4 ? r0 + 8 * u : r1 + 8 * (u - 4);
+      const uint4 w = make_uint4(pack_bf16x2(u2f(x[0]) * mul, u2f(x[1]) * mul),
+                                 pack_bf16x2(u2f(x[2]) * mul, u2f(x[3]) * mul),
+                                 pack_bf16x2(u2f(x[4]) * mul, u2f(x[5]) * mul),
+                                 pack_bf16x2(u2f(x[6]) * mul, u2f(x[7]) * mul));
+      *reinterpret_cast<uint4*>(srow + ((u ^ (lane & 7)) << 4)) = w;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_4d(m, smem_u32(stage), col0 + c, row0, h, b);
+      bulk_commit();
+    }
+  }
+}
+
+
 
 }  // namespace eta
