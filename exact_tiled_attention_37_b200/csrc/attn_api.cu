@@ -183,7 +183,8 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
   if ((s = make_map(&tq, q, B, Hq, N, D, 2, 128)) != ATTN_OK) return s;
   if ((s = make_map(&tk, k, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
   if ((s = make_map(&tv, v, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
-  auto kern = eta::fwd_single_kernel<D, BC, NS>;
+  auto kern = p.bmask ? eta::fwd_single_kernel<D, BC, NS, true>
+                      : eta::fwd_single_kernel<D, BC, NS, false>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
   dim3 grid(Hq, B, (N + 127) / 128);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
@@ -485,9 +486,13 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
         static_cast<const float*>(v.ptr), q.sb, q.sh, q.sn, k.sb, k.sh, k.sn, v.sb, v.sh, v.sn, p);
     return last_launch();
   }
+  // One query tile per CTA with 64-key tiles and a double-buffered S; at
+  // D <= 128 two CTAs share an SM (faster than the two-tile ping-pong CTA,
+  // measured: each CTA's S(j+1) runs while its softmax of S(j) does, and one
+  // CTA's loads and epilogue overlap the other's products).
   switch (D) {
-    case 64: return launch_pingpong<__nv_bfloat16, 64, 6>(q, k, v, p, B, Hq, Hkv, N, st);
-    case 128: return launch_pingpong<__nv_bfloat16, 128, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+    case 64: return launch_single<64, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
+    case 128: return launch_single<128, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
     default: return launch_single<256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
   }
 }

@@ -699,8 +699,10 @@ struct SingleCfg {
   static constexpr int QK_STEPS = ROWB / 32;
   static constexpr int PV_STEPS = BC / 16;
   static constexpr int S_COL = 0;            // S buffers at 0 and BC
-  static constexpr int O_COL = 256;
-  static constexpr int TMEM_COLS = 512;
+  // D <= 128: S[2] | O in 256 columns, so that two CTAs share an SM's TMEM
+  static constexpr int CTAS_PER_SM = D <= 128 ? 2 : 1;
+  static constexpr int O_COL = D <= 128 ? 2 * BC : 256;
+  static constexpr int TMEM_COLS = D <= 128 ? 256 : 512;
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_KV = QTILE;
   static constexpr int SMEM_BAR = SMEM_KV + NS * KTILE;
@@ -717,18 +719,25 @@ struct SingleCfg {
   static constexpr int BAR_DONE = 7 + 2 * NS;
   static constexpr int NBAR = 8 + 2 * NS;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
-  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
+  static constexpr int SMEM_BITS = SMEM_MISC + 16;  // block-sparse: marked 128-key blocks
+  static constexpr int SMEM_BYTES = SMEM_BITS + 4 * kMaskWords + 1024;
   static constexpr int THREADS = 256;
   static_assert(2 * BC <= O_COL && O_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // two co-resident CTAs: 228 KB of shared memory per SM, 1 KB reserved per CTA
+  static_assert(CTAS_PER_SM == 1 || CTAS_PER_SM * (SMEM_BYTES + 1024) <= 233472,
+                "two CTAs per SM");
 };
 
-template <int D, int BC, int NS>
-__global__ void __launch_bounds__(256, 1)
+// SPARSE: built for a block-sparse tile mask (p.bmask, 128 x 128 tile pairs):
+// the BC-key tiles of unmarked 128-key blocks are skipped.
+template <int D, int BC, int NS, bool SPARSE>
+__global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     fwd_single_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = SingleCfg<D, BC, NS>;
+  static_assert(!SPARSE || 128 % BC == 0, "key tiles within 128-key mask blocks");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -745,11 +754,35 @@ __global__ void __launch_bounds__(256, 1)
   const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / p.group;
   const int q0 = qb * 128;
-  // key tiles j0 .. j0 + n - 1 are visible to this query tile; loop counters
-  // below run over 0 .. n - 1
+  // key tiles [j0, j1) are visible to this query tile; the loops below run a
+  // counter u over the computed ones (all of them without a block mask)
   const int2 ktr = key_tiles(q0, p.N, p.wl, p.wr, BC);
-  const int j0 = ktr.x;
-  const int n = ktr.y - ktr.x;
+  const int j0 = ktr.x, j1 = ktr.y;
+  constexpr int TPB = 128 / BC;  // key tiles per 128-key mask block
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::SMEM_BITS);
+  if constexpr (SPARSE) {
+    // bit kb: 128-key block kb is marked for this query tile (published to
+    // every warp by the __syncthreads below)
+    for (int wi = warp; wi < kMaskWords; wi += C::THREADS / 32) {
+      const int kb = 32 * wi + lane;
+      const bool on = kb < p.nt && qb < p.nt &&
+                      p.bmask[((static_cast<long long>(b) * p.Hq + h) * p.nt + qb) * p.nt + kb] != 0;
+      const uint32_t w = __ballot_sync(0xffffffffu, on);
+      if (lane == 0) bits[wi] = w;
+    }
+  }
+  // first computed key tile >= j (j1 if none)
+  auto next_tile = [&](int j) -> int {
+    j = max(j, j0);
+    if constexpr (!SPARSE) return min(j, j1);
+    while (j < j1) {
+      const int kb = next_bit(bits, j / TPB, (j1 + TPB - 1) / TPB);
+      if (kb * TPB >= j1) return j1;
+      j = max(j, kb * TPB);
+      if ((bits[(j / TPB) >> 5] >> ((j / TPB) & 31)) & 1u) return j;
+    }
+    return j1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::BAR_Q), 1);
@@ -777,6 +810,8 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+  int n = 0;  // computed key tiles
+  for (int j = next_tile(j0); j < j1; j = next_tile(j + 1)) ++n;
 
   if (warp < 4) {
     const int r = threadIdx.x & 127;
@@ -785,29 +820,31 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t o_addr = tmem + lane_base + C::O_COL;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int buf = j & 1;
+    for (int u = 0, j = next_tile(j0); u < n; ++u, j = next_tile(j + 1)) {
+      const int buf = u & 1;
       const uint32_t s_addr = tmem + lane_base + C::S_COL + BC * buf;
-      if (!W.wait_warp(BAR(C::BAR_S + buf), (j >> 1) & 1, 10)) { ok = false; break; }
+      if (!W.wait_warp(BAR(C::BAR_S + buf), (u >> 1) & 1, 10)) { ok = false; break; }
       tc_fence_after();
       float s[BC];
       tmem_load_row<BC>(s_addr, s);
-      apply_mask<BC>(s, col_window(BC * (j0 + j), qrow, p.N, p.wl, p.wr));
+      apply_mask<BC>(s, col_window(BC * j, qrow, p.N, p.wl, p.wr));
       float alpha;
       const bool rescaled = online_softmax_step<BC, 0>(s, p.c, m, l, alpha);
       tmem_store_p<BC, false>(s_addr, s);
-      if (rescaled && j > 0) {
-        // O must hold every P V product up to tile j-1 before it is rescaled.
-        if (!W.wait_warp(BAR(C::BAR_PV), (j - 1) & 1, 11)) { ok = false; break; }
+      if (rescaled && u > 0) {
+        // O must hold every P V product up to tile u-1 before it is rescaled.
+        if (!W.wait_warp(BAR(C::BAR_PV), (u - 1) & 1, 11)) { ok = false; break; }
         tc_fence_after();
         tmem_scale_row<D>(o_addr, alpha);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::BAR_P + (j & 1)));
+      if (lane == 0) mbar_arrive(BAR(C::BAR_P + (u & 1)));
     }
-    if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
+    if (ok && n == 0) {
+      store_empty_row<__nv_bfloat16, D>(p, b, h, qrow);
+    } else if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
       tc_fence_after();
       store_row<__nv_bfloat16, D>(o_addr, p, b, h, qrow, m, l);
     }
@@ -820,16 +857,16 @@ __global__ void __launch_bounds__(256, 1)
       for (int c = 0; c < C::NCHUNK; ++c)
         tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * 64, q0, h, b);
       int it = 0;
-      for (int j = 0; j < n && !W.aborted(); ++j) {
+      for (int u = 0, j = next_tile(j0); u < n && !W.aborted(); ++u, j = next_tile(j + 1)) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = it % NS;
           const uint32_t ph = static_cast<uint32_t>(it / NS) & 1u;
           if (!W.wait(BAR(C::BAR_KVE + slot), ph ^ 1u, 30)) break;
-          if ((p.debug_flags & 1) && kv == 1 && j == 0) continue;
+          if ((p.debug_flags & 1) && kv == 1 && u == 0) continue;
           mbar_expect_tx(BAR(C::BAR_KVF + slot), C::KTILE);
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_4d(sbase + C::SMEM_KV + slot * C::KTILE + c * C::KCHUNK, kv ? &tm_v : &tm_k,
-                        BAR(C::BAR_KVF + slot), c * 64, BC * (j0 + j), hk, b);
+                        BAR(C::BAR_KVF + slot), c * 64, BC * j, hk, b);
         }
       }
       const int issued = it;
@@ -868,7 +905,8 @@ __global__ void __launch_bounds__(256, 1)
           mma_ts<false>(tmem + C::O_COL, a + 8u * ks, sdesc_at(vb, ks * 16 * 128), idesc_o,
                         ks > 0 ? 1u : acc0);
       };
-      bool ok = W.wait(BAR(C::BAR_Q), 0, 40) && W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
+      bool ok = n > 0 && W.wait(BAR(C::BAR_Q), 0, 40) &&
+                W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
       if (ok) {
         tc_fence_after();
         issue_s(0, kslot(0));
