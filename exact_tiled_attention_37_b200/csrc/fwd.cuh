@@ -11,13 +11,16 @@
 // GPUs" finding on the FlashAttention entity page).
 //
 // Two kernels:
+//  * fwd_single_kernel: one 128-row query tile per CTA, 64-row K/V tiles
+//    through a TMA ring and a double-buffered S, so that S(j+1) = Q K_{j+1}^T
+//    runs while the row softmax works on S(j).  TMEM: S0 | S1 | O.  At
+//    D <= 128 these take 256 columns and two CTAs share an SM (one CTA's
+//    loads and epilogue overlap the other's products); at D = 256 O needs
+//    256 columns and one CTA runs per SM.  Used for bf16 D = 64, 128, 256.
 //  * fwd_pingpong_kernel: one CTA owns two 128-row query tiles of one
 //    (batch, head) and streams 128-row K/V tiles through a TMA ring.  While the
 //    softmax warpgroup of one query tile works, the tensor core runs the other
-//    tile's MMAs.  TMEM: S0 | S1 | O0 | O1.  Used for bf16 D = 64, 128.
-//  * fwd_single_kernel: one 128-row query tile, 64-row K/V tiles and a double
-//    buffered S so that S(j+1) = Q K_{j+1}^T runs while row softmax works on
-//    S(j).  TMEM: S0 | S1 | O (D = 256 columns).  Used for bf16 D = 256.
+//    tile's MMAs.  TMEM: S0 | S1 | O0 | O1.  Used for the e4m3 forward.
 //
 // Roles (warp-specialised): a TMA producer warp, an MMA warp (one elected
 // thread issues every tcgen05.mma), and 128-thread softmax warpgroups in
