@@ -187,7 +187,10 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
                       : eta::fwd_single_kernel<D, BC, NS, false>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
   dim3 grid(Hq, B, (N + 127) / 128);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  CUtensorMap to;  // O as [B, Hq, N, D] bf16 ({64, 32} boxes) for TMA-store epilogues
+  const attn_tensor_t o_t{p.o, p.osb, p.osh, p.osn};
+  if ((s = make_map(&to, o_t, B, Hq, N, D, 2, 32)) != ATTN_OK) return s;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, to, p);
   return last_launch();
 }
 

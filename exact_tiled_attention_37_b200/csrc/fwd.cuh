@@ -738,7 +738,8 @@ template <int D, int BC, int NS, bool SPARSE>
 __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     fwd_single_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using C = SingleCfg<D, BC, NS>;
   static_assert(!SPARSE || 128 % BC == 0, "key tiles within 128-key mask blocks");
   extern __shared__ uint8_t smem_raw[];
@@ -832,7 +833,7 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       tmem_load_row<BC>(s_addr, s);
       apply_mask<BC>(s, col_window(BC * j, qrow, p.N, p.wl, p.wr));
       float alpha;
-      const bool rescaled = online_softmax_step<BC, 0>(s, p.c, m, l, alpha);
+      const bool rescaled = online_softmax_step<BC, kSoftExp8>(s, p.c, m, l, alpha);
       tmem_store_p<BC, false>(s_addr, s);
       if (rescaled && u > 0) {
         // O must hold every P V product up to tile u-1 before it is rescaled.
@@ -849,7 +850,16 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       store_empty_row<__nv_bfloat16, D>(p, b, h, qrow);
     } else if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
       tc_fence_after();
-      store_row<__nv_bfloat16, D>(o_addr, p, b, h, qrow, m, l);
+      // O / l through TMA stores ({64, 32} boxes), staged in this warp's rows
+      // of Q's first chunk (every MMA reading Q is complete)
+      uint8_t* stage = smem + C::SMEM_Q + warp * 32 * 128;
+      tmem_rows_tma_store<D>(o_addr, stage, &tm_o, 0, q0 + warp * 32, h, b,
+                             l > 0.f ? p.o_mul / l : 0.f);
+      if (qrow < p.N)
+        p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] =
+            l > 0.f ? m * p.scale + logf(l) : -INFINITY;
+      if (lane == 0) bulk_wait_read_all();  // the staging rows stay valid until read
+      __syncwarp();
     }
   } else if (warp == 4) {
     if (lane == 0) {
