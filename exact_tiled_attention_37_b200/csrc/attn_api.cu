@@ -126,13 +126,6 @@ attn_status_t set_smem(Kernel k, int bytes) {
   return ATTN_OK;
 }
 
-template <typename Kernel>
-int kernel_regs(Kernel k) {
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return -1;
-  return fa.numRegs;
-}
-
 attn_status_t last_launch() {
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -146,45 +139,18 @@ int sm_count() {
 }
 
 // ---------------------------------------------------------------- forward
-template <typename T, int D, int NS>
-attn_status_t launch_pingpong(const attn_tensor_t& q, const attn_tensor_t& k,
-                              const attn_tensor_t& v, const eta::FwdParams& p, int B, int Hq,
-                              int Hkv, int N, cudaStream_t st) {
-  using C = eta::PingPongCfg<T, D, NS>;
-  CUtensorMap tq, tk, tv;
-  attn_status_t s;
-  if ((s = make_map(&tq, q, B, Hq, N, D, sizeof(T), 128)) != ATTN_OK) return s;
-  if ((s = make_map(&tk, k, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
-  if ((s = make_map(&tv, v, B, Hkv, N, D, sizeof(T), 128)) != ATTN_OK) return s;
-  auto kern = p.bmask ? eta::fwd_pingpong_kernel<T, D, NS, true>
-                      : eta::fwd_pingpong_kernel<T, D, NS, false>;
-  // The kernel moves registers between its warpgroups on the assumption that
-  // it was launched with C::LAUNCH_REGS per thread; never launch otherwise.
-  static const int regs[2] = {kernel_regs(eta::fwd_pingpong_kernel<T, D, NS, false>),
-                              kernel_regs(eta::fwd_pingpong_kernel<T, D, NS, true>)};
-  if (regs[p.bmask ? 1 : 0] != C::LAUNCH_REGS) return ATTN_ERR_CUDA;
-  if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
-  dim3 grid(Hq, B, (N + 255) / 256);
-  // O as [B, Hq, N, D] bf16 for the TMA stores of the epilogue ({64, 32} boxes)
-  CUtensorMap to;
-  const attn_tensor_t o_t{p.o, p.osb, p.osh, p.osn};
-  if ((s = make_map(&to, o_t, B, Hq, N, D, 2, 32)) != ATTN_OK) return s;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, to, p);
-  return last_launch();
-}
-
-template <int D, int BC, int NS>
+template <typename T, int D, int BC, int NS>
 attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, const attn_tensor_t& v,
                             const eta::FwdParams& p, int B, int Hq, int Hkv, int N,
                             cudaStream_t st) {
-  using C = eta::SingleCfg<D, BC, NS>;
+  using C = eta::SingleCfg<T, D, BC, NS>;
   CUtensorMap tq, tk, tv;
   attn_status_t s;
-  if ((s = make_map(&tq, q, B, Hq, N, D, 2, 128)) != ATTN_OK) return s;
-  if ((s = make_map(&tk, k, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
-  if ((s = make_map(&tv, v, B, Hkv, N, D, 2, BC)) != ATTN_OK) return s;
-  auto kern = p.bmask ? eta::fwd_single_kernel<D, BC, NS, true>
-                      : eta::fwd_single_kernel<D, BC, NS, false>;
+  if ((s = make_map(&tq, q, B, Hq, N, D, sizeof(T), 128)) != ATTN_OK) return s;
+  if ((s = make_map(&tk, k, B, Hkv, N, D, sizeof(T), BC)) != ATTN_OK) return s;
+  if ((s = make_map(&tv, v, B, Hkv, N, D, sizeof(T), BC)) != ATTN_OK) return s;
+  auto kern = p.bmask ? eta::fwd_single_kernel<T, D, BC, NS, true>
+                      : eta::fwd_single_kernel<T, D, BC, NS, false>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
   dim3 grid(Hq, B, (N + 127) / 128);
   CUtensorMap to;  // O as [B, Hq, N, D] bf16 ({64, 32} boxes) for TMA-store epilogues
@@ -494,9 +460,9 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   // measured: each CTA's S(j+1) runs while its softmax of S(j) does, and one
   // CTA's loads and epilogue overlap the other's products).
   switch (D) {
-    case 64: return launch_single<64, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
-    case 128: return launch_single<128, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
-    default: return launch_single<256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+    case 64: return launch_single<__nv_bfloat16, 64, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
+    case 128: return launch_single<__nv_bfloat16, 128, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+    default: return launch_single<__nv_bfloat16, 256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
   }
 }
 
@@ -538,8 +504,8 @@ attn_status_t attn_fwd_fp8(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, at
   p.o_mul = v_scale / eta::kP8Scale;
   p.bmask = nullptr;
   p.nt = (N + 127) / 128;
-  return launch_pingpong<__nv_fp8_e4m3, 128, 8>(q, k, v, p, B, Hq, Hkv, N,
-                                                static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return launch_single<__nv_fp8_e4m3, 128, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int max_pages) {

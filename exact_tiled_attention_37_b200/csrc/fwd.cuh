@@ -10,17 +10,12 @@
 // as in the "FlashAttention-4: Algorithm and Kernel Pipelining for Blackwell
 // GPUs" finding on the FlashAttention entity page).
 //
-// Two kernels:
-//  * fwd_single_kernel: one 128-row query tile per CTA, 64-row K/V tiles
-//    through a TMA ring and a double-buffered S, so that S(j+1) = Q K_{j+1}^T
-//    runs while the row softmax works on S(j).  TMEM: S0 | S1 | O.  At
-//    D <= 128 these take 256 columns and two CTAs share an SM (one CTA's
-//    loads and epilogue overlap the other's products); at D = 256 O needs
-//    256 columns and one CTA runs per SM.  Used for bf16 D = 64, 128, 256.
-//  * fwd_pingpong_kernel: one CTA owns two 128-row query tiles of one
-//    (batch, head) and streams 128-row K/V tiles through a TMA ring.  While the
-//    softmax warpgroup of one query tile works, the tensor core runs the other
-//    tile's MMAs.  TMEM: S0 | S1 | O0 | O1.  Used for the e4m3 forward.
+// The kernel, fwd_single_kernel: one 128-row query tile per CTA, 64-row K/V
+// tiles through a TMA ring and a double-buffered S, so that S(j+1) =
+// Q K_{j+1}^T runs while the row softmax works on S(j).  TMEM: S0 | S1 | O.
+// At D <= 128 these take 256 columns and two CTAs share an SM (one CTA's
+// loads and epilogue overlap the other's products); at D = 256 O needs 256
+// columns and one CTA runs per SM.  bf16 at D = 64, 128, 256; e4m3 at D = 128.
 //
 // Roles (warp-specialised): a TMA producer warp, an MMA warp (one elected
 // thread issues every tcgen05.mma), and 128-thread softmax warpgroups in
@@ -205,10 +200,10 @@ __device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&p)[BC
 constexpr float kP8Scale = 256.f;
 template <int BC>
 __device__ __forceinline__ void tmem_store_p8(uint32_t taddr, const float (&p)[BC]) {
-  static_assert(BC == 128, "one 128-column row");
-  uint32_t hi[32], lo[32];
+  static_assert(BC == 128 || BC == 64, "32 or 16 columns per term");
+  uint32_t hi[BC / 4], lo[BC / 4];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < BC / 4; ++i) {
     uint32_t hw = 0u, lw = 0u;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -224,8 +219,13 @@ __device__ __forceinline__ void tmem_store_p8(uint32_t taddr, const float (&p)[B
     hi[i] = hw;
     lo[i] = lw;
   }
-  tmem_st32(taddr, hi);
-  tmem_st32(taddr + BC / 4, lo);
+  if constexpr (BC == 128) {
+    tmem_st32(taddr, hi);
+    tmem_st32(taddr + BC / 4, lo);
+  } else {
+    tmem_st16(taddr, hi);
+    tmem_st16(taddr + BC / 4, lo);
+  }
 }
 
 // Multiplies DC fp32 TMEM columns of this lane by alpha (the correction step).
@@ -240,47 +240,6 @@ __device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(u2f(r[i]) * alpha);
     tmem_st32(taddr + 32 * c, r);
   }
-}
-
-// Epilogue of one row: O = O_acc / l written to global memory as T, lse.
-template <typename T, int D>
-__device__ __forceinline__ void store_row(uint32_t o_taddr, const FwdParams& p, int b, int h,
-                                          int qrow, float m, float l) {
-  const bool valid = qrow < p.N;
-  const float inv_l = l > 0.f ? p.o_mul / l : 0.f;  // a row with no visible key stores O = 0
-  char* row = static_cast<char*>(p.o) +
-              (static_cast<long long>(b) * p.osb + static_cast<long long>(h) * p.osh +
-               static_cast<long long>(qrow) * p.osn) *
-                  static_cast<long long>(sizeof(T));
-#pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld32(o_taddr + 32 * c, r);
-    tmem_wait_ld();
-    if (valid) {
-      if constexpr (sizeof(T) == 2) {
-        uint4* dst = reinterpret_cast<uint4*>(row + 64 * c);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 w;
-          w.x = pack_bf16x2(u2f(r[8 * v + 0]) * inv_l, u2f(r[8 * v + 1]) * inv_l);
-          w.y = pack_bf16x2(u2f(r[8 * v + 2]) * inv_l, u2f(r[8 * v + 3]) * inv_l);
-          w.z = pack_bf16x2(u2f(r[8 * v + 4]) * inv_l, u2f(r[8 * v + 5]) * inv_l);
-          w.w = pack_bf16x2(u2f(r[8 * v + 6]) * inv_l, u2f(r[8 * v + 7]) * inv_l);
-          dst[v] = w;
-        }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(row + 128 * c);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_float4(u2f(r[4 * v]) * inv_l, u2f(r[4 * v + 1]) * inv_l,
-                               u2f(r[4 * v + 2]) * inv_l, u2f(r[4 * v + 3]) * inv_l);
-      }
-    }
-  }
-  if (valid)
-    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] =
-        l > 0.f ? m * p.scale + logf(l) : -INFINITY;
 }
 
 // Epilogue of a row whose query tile computed no key tile: O = 0, lse = -inf.
@@ -329,370 +288,12 @@ __device__ __forceinline__ int2 key_tiles(int qs, int N, int wl, int wr, int BN)
 }
 
 // =====================================================================
-// Two query tiles per CTA (ping-pong).
-// =====================================================================
-template <typename T, int D, int NS>
-struct PingPongCfg {
-  static constexpr bool TF32 = sizeof(T) == 4;
-  static constexpr bool FP8 = sizeof(T) == 1;  // e4m3 inputs, kind::f8f6f4 products
-  static constexpr int ES = sizeof(T);
-  static constexpr int ROWB = D * ES;        // bytes per row
-  static constexpr int NCHUNK = ROWB / 128;  // 128-byte swizzle chunks per row
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int CHUNK = 128 * 128;    // bytes of one chunk of a 128-row tile
-  static constexpr int TILE = 128 * ROWB;
-  static constexpr int QK_STEPS = ROWB / 32;
-  static constexpr int PV_ROWS = 32 / ES;    // V rows consumed per MMA
-  // e4m3: P is split into two e4m3 terms (high and residual), each multiplied by V
-  static constexpr int PV_STEPS = (FP8 ? 2 : 1) * BN / PV_ROWS;
-  static constexpr int O_COL = 256;          // O0 at 256, O1 at 256 + D
-  static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_Q = 0;
-  static constexpr int SMEM_KV = 2 * TILE;
-  static constexpr int SMEM_BAR = SMEM_KV + NS * TILE;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_full[2], done
-  static constexpr int BAR_Q = 0;
-  static constexpr int BAR_KVF = 1;
-  static constexpr int BAR_KVE = 1 + NS;
-  static constexpr int BAR_S = 1 + 2 * NS;
-  static constexpr int BAR_P = 3 + 2 * NS;
-  static constexpr int BAR_O = 5 + 2 * NS;
-  static constexpr int BAR_DONE = 7 + 2 * NS;
-  static constexpr int NBAR = 8 + 2 * NS;
-  static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;  // tmem slot, abort flag
-  static constexpr int SMEM_BITS = SMEM_MISC + 16;        // [2][kMaskWords] used-tile bits
-  static constexpr int SMEM_BYTES = SMEM_BITS + 8 * kMaskWords + 1024;  // + alignment slack
-  static constexpr int THREADS = 384;
-  // registers per thread: at launch (what the compiler allocates under
-  // __launch_bounds__(384, 1); the host checks it before launching), then
-  // moved to the softmax warpgroups, away from the producer/MMA warpgroup
-  static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, OTHER_REGS = 72;
-  static_assert(THREADS * LAUNCH_REGS == 256 * SOFTMAX_REGS + 128 * OTHER_REGS, "register split");
-  // bf16 only: tf32 products would keep 10 mantissa bits, which misses the
-  // logsumexp tolerance; fp32 storage goes through fwd_fp32_kernel.
-  static_assert(sizeof(T) == 2 || sizeof(T) == 1, "bf16 or e4m3 storage");
-  static_assert(ROWB % 128 == 0, "row must be whole 128-byte chunks");
-  static_assert(256 + 2 * D <= TMEM_COLS, "TMEM budget");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-};
-
-// SPARSE: built for a block-sparse tile mask (p.bmask); the dense build
-// carries none of the mask bookkeeping.
-template <typename T, int D, int NS, bool SPARSE>
-__global__ void __launch_bounds__(384, 1)
-    fwd_pingpong_kernel(const __grid_constant__ CUtensorMap tm_q,
-                        const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
-  using C = PingPongCfg<T, D, NS>;
-  using OutT = std::conditional_t<C::FP8, __nv_bfloat16, T>;  // e4m3 inputs give bf16 O
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + C::SMEM_BAR;
-  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC);
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::SMEM_MISC + 4);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid (Hq, B, query blocks): the block index varies slowest so that every
-  // head's longest causal CTAs are dispatched first
-  const int qb = gridDim.z - 1 - blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int hk = h / p.group;
-  const int q0 = qb * 256;
-  // key tiles [jlo(t), jhi(t)) of each query tile; tile 0's range never starts
-  // or ends after tile 1's, so tile 1 (when it has work) is the last reader of
-  // every K/V tile it uses
-  // (scalars, selected by t, so that they stay in registers)
-  const int2 kr0 = key_tiles(q0, p.N, p.wl, p.wr, 128);
-  const int2 kr1 = key_tiles(q0 + 128, p.N, p.wl, p.wr, 128);
-  auto jlo = [&](int t) { return t ? kr1.x : kr0.x; };
-  auto jhi = [&](int t) { return t ? kr1.y : kr0.y; };
-  const bool has1 = kr1.y > kr1.x;
-  const int jmin = kr0.x, jmax = has1 ? kr1.y : kr0.y;
-  // Block-sparse: bit j of bits[t] marks key tile j as computed by query tile t.
-  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::SMEM_BITS);
-  if constexpr (SPARSE) {
-    for (int wi = warp; wi < 2 * kMaskWords; wi += C::THREADS / 32) {
-      const int t = wi / kMaskWords, j = 32 * (wi % kMaskWords) + lane;
-      const int qt = 2 * qb + t;
-      const bool on = j >= jlo(t) && j < jhi(t) && qt < p.nt &&
-                      p.bmask[((static_cast<long long>(b) * p.Hq + h) * p.nt + qt) * p.nt + j] != 0;
-      const uint32_t w = __ballot_sync(0xffffffffu, on);
-      if (lane == 0) bits[wi] = w;
-    }
-  }
-  // key tile j computed by query tile t
-  auto uses = [&](int t, int j) -> bool {
-    if (j < jlo(t) || j >= jhi(t)) return false;
-    if constexpr (!SPARSE) return true;
-    return (bits[t * kMaskWords + (j >> 5)] >> (j & 31)) & 1u;
-  };
-  // first key tile >= j computed by query tile t (jhi(t) if none)
-  auto next_use = [&](int t, int j) -> int {
-    j = max(j, jlo(t));
-    if constexpr (!SPARSE) return min(j, jhi(t));
-    return next_bit(bits + t * kMaskWords, j, jhi(t));
-  };
-  auto in_union = [&](int j) -> bool { return uses(0, j) || uses(1, j); };
-  // first key tile >= j that either query tile computes (jmax if none)
-  auto next_union = [&](int j) -> int {
-    if constexpr (!SPARSE) {
-      for (; j < jmax; ++j)
-        if (in_union(j)) return j;
-      return jmax;
-    }
-    return min(next_use(0, j), next_use(1, j));
-  };
-
-  if (threadIdx.x == 0) {
-    mbar_init(BAR(C::BAR_Q), 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(BAR(C::BAR_KVF + s), 1);
-      mbar_init(BAR(C::BAR_KVE + s), 1);
-    }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(BAR(C::BAR_S + t), 1);
-      mbar_init(BAR(C::BAR_P + t), 4);
-      mbar_init(BAR(C::BAR_O + t), 1);
-    }
-    mbar_init(BAR(C::BAR_DONE), 1);
-    *abort_flag = 0u;
-    fence_barrier_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == 9) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const Waiter W{abort_flag, p.status, p.wait_limit_ns};
-#ifdef ETA_TRACE
-  const int tcta = (h == 0 && b == 0) ? (qb == (int)gridDim.z - 1 ? 0 : (qb == (int)gridDim.z / 2 ? 1 : -1)) : -1;
-#else
-  const int tcta = -1;
-#endif
-  (void)tcta;
-
-  // Registers: the softmax warpgroups hold a 128-float score row; the
-  // producer/MMA warpgroup needs few (no spills in either role).
-  if (warp < 8) {
-    setmaxnreg_inc<C::SOFTMAX_REGS>();
-  } else {
-    setmaxnreg_dec<C::OTHER_REGS>();
-  }
-  if (warp < 8) {
-    // ------------------------------------------------ softmax / correction / epilogue
-    const int t = warp >> 2;
-    const int r = threadIdx.x & 127;
-    const int qrow = q0 + 128 * t + r;
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + 128u * t;
-    const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    int cnt = 0;  // key tiles of this query tile done so far
-    for (int j = next_use(t, jlo(t)); j < jhi(t); j = next_use(t, j + 1), ++cnt) {
-      if (!W.wait_warp(BAR(C::BAR_S + t), cnt & 1, 10 + t)) { ok = false; break; }
-      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 0);
-      tc_fence_after();
-      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 1);
-      // The whole 128-score row lives in registers: fully unrolled code with a
-      // few spills measured faster than a spill-free streamed row (which loses
-      // the instruction-level parallelism of the unrolled exp/sum chain).
-      float alpha;
-      float s[128];
-      tmem_load_row<128>(s_addr, s);
-      apply_mask<128>(s, col_window(128 * j, qrow, p.N, p.wl, p.wr));
-      const bool rescaled =
-          online_softmax_step<128, kSoftExp8, C::FP8 ? 0 : static_cast<int>(kRescaleLog2)>(
-              s, p.c, m, l, alpha);
-      if constexpr (C::FP8) {
-        tmem_store_p8<128>(s_addr, s);
-      } else {
-        tmem_store_p<128, C::TF32>(s_addr, s);
-      }
-      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 2);
-      if (rescaled && cnt > 0) tmem_scale_row<D>(o_addr, alpha);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::BAR_P + t));
-      if (r == 0) ETA_FTRACE_AT(tcta, t, j, 3);
-    }
-    if (ok && cnt == 0) {
-      store_empty_row<OutT, D>(p, b, h, qrow);
-    } else if (ok && W.wait_warp(BAR(C::BAR_O + t), 0, 20 + t)) {
-      tc_fence_after();
-      if constexpr (!C::FP8) {
-        // O / l through TMA stores, staged in this warp's rows of Q_t (every
-        // MMA reading Q_t is complete)
-        uint8_t* stage = smem + C::SMEM_Q + t * C::TILE + (warp & 3) * 32 * 128;
-        tmem_rows_tma_store<D>(o_addr, stage, &tm_o, 0, q0 + 128 * t + (warp & 3) * 32, h, b,
-                               l > 0.f ? p.o_mul / l : 0.f);
-        if (qrow < p.N)
-          p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] =
-              l > 0.f ? m * p.scale + logf(l) : -INFINITY;
-        if (lane == 0) bulk_wait_read_all();  // the staging rows stay valid until read
-        __syncwarp();
-      } else {
-        store_row<OutT, D>(o_addr, p, b, h, qrow, m, l);
-      }
-    }
-  } else if (warp == 8) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      constexpr int EPC = 128 / C::ES;  // elements per 128-byte chunk
-      mbar_expect_tx(BAR(C::BAR_Q), 2 * C::TILE);
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sbase + C::SMEM_Q + t * C::TILE + c * C::CHUNK, &tm_q, BAR(C::BAR_Q), c * EPC,
-                      q0 + 128 * t, h, b);
-      int it = 0;
-      for (int j = jmin; j < jmax && !W.aborted(); ++j) {
-        if (!in_union(j)) continue;  // no query tile of this CTA computes key tile j
-        for (int kv = 0; kv < 2; ++kv, ++it) {
-          const int slot = it % NS;
-          const uint32_t ph = static_cast<uint32_t>(it / NS) & 1u;
-          if (!W.wait(BAR(C::BAR_KVE + slot), ph ^ 1u, 30)) break;
-          if ((p.debug_flags & 1) && kv == 1 && j == jmin) continue;  // fault injection: drop V
-          mbar_expect_tx(BAR(C::BAR_KVF + slot), C::TILE);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sbase + C::SMEM_KV + slot * C::TILE + c * C::CHUNK, kv ? &tm_v : &tm_k,
-                        BAR(C::BAR_KVF + slot), c * EPC, 128 * j, hk, b);
-        }
-      }
-      // Let every copy this warp started land before the CTA can exit.
-      const int issued = it;
-      W.drain(BAR(C::BAR_Q), 0, 31);
-      for (int s = 0; s < NS && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / NS) * NS;  // last load into slot s
-        W.drain(BAR(C::BAR_KVF + s), static_cast<uint32_t>(last / NS) & 1u, 32);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t fmt = C::FP8 ? 0u : (C::TF32 ? 2u : 1u);
-      constexpr uint32_t idesc_s = idesc_make(128, 128, fmt, false, false);
-      constexpr uint32_t idesc_o = idesc_make(128, D, fmt, false, true);
-      // ring slots of K_j / V_j from j's position among the streamed key tiles
-      // (the producer streams only the tiles that some query tile of this CTA
-      // computes, in increasing order)
-      auto kslot = [&](int pos) { return (2 * pos) % NS; };
-      auto kph = [&](int pos) { return static_cast<uint32_t>((2 * pos) / NS) & 1u; };
-      auto vslot = [&](int pos) { return (2 * pos + 1) % NS; };
-      auto vph = [&](int pos) { return static_cast<uint32_t>((2 * pos + 1) / NS) & 1u; };
-      auto issue_s = [&](int t, int slot) {
-        const SDesc qa = sdesc_base(sbase + C::SMEM_Q + t * C::TILE, 16, 1024);
-        const SDesc kb = sdesc_base(sbase + C::SMEM_KV + slot * C::TILE, 16, 1024);
-        const uint32_t d = tmem + 128u * t;
-#pragma unroll
-        for (int ks = 0; ks < C::QK_STEPS; ++ks) {
-          const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-          if constexpr (C::FP8) {
-            mma_ss_f8(d, sdesc_at(qa, off), sdesc_at(kb, off), idesc_s, ks > 0);
-          } else {
-            mma_ss<C::TF32>(d, sdesc_at(qa, off), sdesc_at(kb, off), idesc_s, ks > 0);
-          }
-        }
-      };
-      auto issue_pv = [&](int t, int slot, bool acc) {
-        const SDesc vb = sdesc_base(sbase + C::SMEM_KV + slot * C::TILE, C::CHUNK, 1024);
-        const uint32_t d = tmem + C::O_COL + D * t, a = tmem + 128u * t;
-        const uint32_t acc0 = acc ? 1u : 0u;
-#pragma unroll
-        for (int ks = 0; ks < C::PV_STEPS; ++ks)
-          if constexpr (C::FP8) {
-            // steps 0-3: high term (TMEM columns 0-31), 4-7: residual (32-63),
-            // both against the same V rows
-            mma_ts_f8(d, a + 8u * ks, sdesc_at(vb, (ks & 3) * C::PV_ROWS * 128), idesc_o,
-                      ks > 0 ? 1u : acc0);
-          } else {
-            mma_ts<C::TF32>(d, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128), idesc_o,
-                            ks > 0 ? 1u : acc0);
-          }
-      };
-      // S_t = Q_t K^T for the key tile at ring position pos
-      auto start_s = [&](int t, int pos) -> bool {
-        if (!W.wait(BAR(C::BAR_KVF + kslot(pos)), kph(pos), 44 + t)) return false;
-        tc_fence_after();
-        issue_s(t, kslot(pos));
-        mma_commit(BAR(C::BAR_S + t));
-        return true;
-      };
-      // S_t of a query tile's next key tile is issued right after its P V when
-      // that tile is the next one streamed (always, without a block mask);
-      // otherwise when the loop reaches it, so that no wait can reach past
-      // the tiles the ring holds.
-      int pend[2] = {next_use(0, jmin), next_use(1, jmin)};
-      int cnt[2] = {0, 0};
-      bool ok = W.wait(BAR(C::BAR_Q), 0, 40);
-      for (int j = jmin, pos = 0; ok && j < jmax; ++j) {
-        if (!in_union(j)) continue;
-        if (pend[0] == j && j < jhi(0)) ok = start_s(0, pos);
-        if (ok && pend[1] == j && j < jhi(1)) ok = start_s(1, pos);
-        if (!ok) break;
-        // every S(j) is issued: K_j's slot frees once they complete
-        mma_commit(BAR(C::BAR_KVE + kslot(pos)));
-        if (!W.wait(BAR(C::BAR_KVF + vslot(pos)), vph(pos), 42)) { ok = false; break; }
-        const int last_t = uses(1, j) ? 1 : 0;  // the last P V that reads V_j
-        auto pv_step = [&](const int t) -> bool {
-          if (!uses(t, j)) return true;
-          if (!W.wait(BAR(C::BAR_P + t), cnt[t] & 1, 43 + 2 * t)) return false;
-          if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 0);
-          if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 2);
-          tc_fence_after();
-          issue_pv(t, vslot(pos), cnt[t] > 0);
-          ++cnt[t];
-          if (t == last_t) mma_commit(BAR(C::BAR_KVE + vslot(pos)));
-          const int nj = next_use(t, j + 1);
-          if (nj >= jhi(t)) {
-            mma_commit(BAR(C::BAR_O + t));
-            pend[t] = jhi(t);
-          } else if (next_union(j + 1) == nj) {
-            if (!start_s(t, pos + 1)) return false;
-            pend[t] = -1;
-            if (t == 0) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 1);
-            if (t == 1) ETA_FTRACE_AT(tcta, 2, j - jlo(0), 3);
-          } else {
-            pend[t] = nj;
-          }
-          return true;
-        };
-        if (!pv_step(0) || !pv_step(1)) { ok = false; break; }
-        ++pos;
-      }
-      // Wait until every MMA this thread issued has finished with TMEM/smem.
-      mma_commit(BAR(C::BAR_DONE));
-      W.drain(BAR(C::BAR_DONE), 0, 47);
-    }
-    __syncwarp();
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-// =====================================================================
 // One query tile per CTA, double-buffered S (large head dimension).
 // =====================================================================
-template <int D, int BC, int NS>
+template <typename T, int D, int BC, int NS>
 struct SingleCfg {
-  static constexpr int ES = 2;
+  static constexpr bool FP8 = sizeof(T) == 1;  // e4m3 inputs, kind::f8f6f4 products
+  static constexpr int ES = sizeof(T);
   static constexpr int ROWB = D * ES;
   static constexpr int NCHUNK = ROWB / 128;
   static constexpr int QCHUNK = 128 * 128;   // chunk of the 128-row Q tile
@@ -700,7 +301,10 @@ struct SingleCfg {
   static constexpr int QTILE = 128 * ROWB;
   static constexpr int KTILE = BC * ROWB;
   static constexpr int QK_STEPS = ROWB / 32;
-  static constexpr int PV_STEPS = BC / 16;
+  static constexpr int PV_ROWS = 32 / ES;    // V rows consumed per P V step
+  // e4m3: P is split into two e4m3 terms (high and residual), each multiplied by V
+  static constexpr int PV_STEPS = (FP8 ? 2 : 1) * BC / PV_ROWS;
+  static constexpr int EPC = 128 / ES;       // elements per 128-byte chunk
   static constexpr int S_COL = 0;            // S buffers at 0 and BC
   // D <= 128: S[2] | O in 256 columns, so that two CTAs share an SM's TMEM
   static constexpr int CTAS_PER_SM = D <= 128 ? 2 : 1;
@@ -727,6 +331,7 @@ struct SingleCfg {
   static constexpr int THREADS = 256;
   static_assert(2 * BC <= O_COL && O_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(sizeof(T) == 2 || (FP8 && D == 128), "bf16, or e4m3 at D = 128");
   // two co-resident CTAs: 228 KB of shared memory per SM, 1 KB reserved per CTA
   static_assert(CTAS_PER_SM == 1 || CTAS_PER_SM * (SMEM_BYTES + 1024) <= 233472,
                 "two CTAs per SM");
@@ -734,13 +339,13 @@ struct SingleCfg {
 
 // SPARSE: built for a block-sparse tile mask (p.bmask, 128 x 128 tile pairs):
 // the BC-key tiles of unmarked 128-key blocks are skipped.
-template <int D, int BC, int NS, bool SPARSE>
+template <typename T, int D, int BC, int NS, bool SPARSE>
 __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     fwd_single_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
-  using C = SingleCfg<D, BC, NS>;
+  using C = SingleCfg<T, D, BC, NS>;
   static_assert(!SPARSE || 128 % BC == 0, "key tiles within 128-key mask blocks");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -778,14 +383,14 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
   // first computed key tile >= j (j1 if none)
   auto next_tile = [&](int j) -> int {
     j = max(j, j0);
-    if constexpr (!SPARSE) return min(j, j1);
-    while (j < j1) {
+    if constexpr (!SPARSE) {
+      return min(j, j1);
+    } else {
+      if (j >= j1) return j1;
+      // the first marked 128-key block at or after j's own
       const int kb = next_bit(bits, j / TPB, (j1 + TPB - 1) / TPB);
-      if (kb * TPB >= j1) return j1;
-      j = max(j, kb * TPB);
-      if ((bits[(j / TPB) >> 5] >> ((j / TPB) & 31)) & 1u) return j;
+      return kb * TPB >= j1 ? j1 : max(j, kb * TPB);
     }
-    return j1;
   };
 
   if (threadIdx.x == 0) {
@@ -833,8 +438,14 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       tmem_load_row<BC>(s_addr, s);
       apply_mask<BC>(s, col_window(BC * j, qrow, p.N, p.wl, p.wr));
       float alpha;
-      const bool rescaled = online_softmax_step<BC, kSoftExp8>(s, p.c, m, l, alpha);
-      tmem_store_p<BC, false>(s_addr, s);
+      const bool rescaled =
+          online_softmax_step<BC, kSoftExp8, C::FP8 ? 0 : static_cast<int>(kRescaleLog2)>(
+              s, p.c, m, l, alpha);
+      if constexpr (C::FP8) {
+        tmem_store_p8<BC>(s_addr, s);
+      } else {
+        tmem_store_p<BC, false>(s_addr, s);
+      }
       if (rescaled && u > 0) {
         // O must hold every P V product up to tile u-1 before it is rescaled.
         if (!W.wait_warp(BAR(C::BAR_PV), (u - 1) & 1, 11)) { ok = false; break; }
@@ -847,7 +458,7 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       if (lane == 0) mbar_arrive(BAR(C::BAR_P + (u & 1)));
     }
     if (ok && n == 0) {
-      store_empty_row<__nv_bfloat16, D>(p, b, h, qrow);
+      store_empty_row<__nv_bfloat16, D>(p, b, h, qrow);  // O is bf16 for either input
     } else if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
       tc_fence_after();
       // O / l through TMA stores ({64, 32} boxes), staged in this warp's rows
@@ -868,7 +479,8 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       tma_prefetch_desc(&tm_v);
       mbar_expect_tx(BAR(C::BAR_Q), C::QTILE);
       for (int c = 0; c < C::NCHUNK; ++c)
-        tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * 64, q0, h, b);
+        tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * C::EPC, q0, h,
+                    b);
       int it = 0;
       for (int u = 0, j = next_tile(j0); u < n && !W.aborted(); ++u, j = next_tile(j + 1)) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
@@ -879,7 +491,7 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
           mbar_expect_tx(BAR(C::BAR_KVF + slot), C::KTILE);
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_4d(sbase + C::SMEM_KV + slot * C::KTILE + c * C::KCHUNK, kv ? &tm_v : &tm_k,
-                        BAR(C::BAR_KVF + slot), c * 64, BC * j, hk, b);
+                        BAR(C::BAR_KVF + slot), c * C::EPC, BC * j, hk, b);
         }
       }
       const int issued = it;
@@ -892,8 +504,9 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     __syncwarp();
   } else if (warp == 5) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_make(128, BC, 1u, false, false);
-      constexpr uint32_t idesc_o = idesc_make(128, D, 1u, false, true);
+      constexpr uint32_t fmt = C::FP8 ? 0u : 1u;  // e4m3 or bf16
+      constexpr uint32_t idesc_s = idesc_make(128, BC, fmt, false, false);
+      constexpr uint32_t idesc_o = idesc_make(128, D, fmt, false, true);
       auto kslot = [&](int j) { return (2 * j) % NS; };
       auto kph = [&](int j) { return static_cast<uint32_t>((2 * j) / NS) & 1u; };
       auto vslot = [&](int j) { return (2 * j + 1) % NS; };
@@ -906,7 +519,11 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
           const uint32_t qoff = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
           const uint32_t koff = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
-          mma_ss<false>(d, sdesc_at(qa, qoff), sdesc_at(kb, koff), idesc_s, ks > 0);
+          if constexpr (C::FP8) {
+            mma_ss_f8(d, sdesc_at(qa, qoff), sdesc_at(kb, koff), idesc_s, ks > 0);
+          } else {
+            mma_ss<false>(d, sdesc_at(qa, qoff), sdesc_at(kb, koff), idesc_s, ks > 0);
+          }
         }
       };
       auto issue_pv = [&](int buf, int slot, bool acc) {
@@ -914,9 +531,18 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
         const uint32_t a = tmem + C::S_COL + BC * buf;
         const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
-        for (int ks = 0; ks < C::PV_STEPS; ++ks)
-          mma_ts<false>(tmem + C::O_COL, a + 8u * ks, sdesc_at(vb, ks * 16 * 128), idesc_o,
-                        ks > 0 ? 1u : acc0);
+        for (int ks = 0; ks < C::PV_STEPS; ++ks) {
+          if constexpr (C::FP8) {
+            // steps over P's high terms (TMEM columns [0, BC/4)), then its
+            // residuals ([BC/4, BC/2)), both against the same V rows
+            constexpr int VSTEPS = BC / C::PV_ROWS;
+            mma_ts_f8(tmem + C::O_COL, a + 8u * ks,
+                      sdesc_at(vb, (ks % VSTEPS) * C::PV_ROWS * 128), idesc_o, ks > 0 ? 1u : acc0);
+          } else {
+            mma_ts<false>(tmem + C::O_COL, a + 8u * ks, sdesc_at(vb, ks * C::PV_ROWS * 128),
+                          idesc_o, ks > 0 ? 1u : acc0);
+          }
+        }
       };
       bool ok = n > 0 && W.wait(BAR(C::BAR_Q), 0, 40) &&
                 W.wait(BAR(C::BAR_KVF + kslot(0)), kph(0), 41);
