@@ -17,9 +17,9 @@
 // loads and epilogue overlap the other's products); at D = 256 O needs 256
 // columns and one CTA runs per SM.  bf16 at D = 64, 128, 256; e4m3 at D = 128.
 //
-// Roles (warp-specialised): a TMA producer warp, an MMA warp (one elected
-// thread issues every tcgen05.mma), and 128-thread softmax warpgroups in
-// which thread r owns query row r (TMEM lane r).  The softmax warpgroup also
+// Roles (warp-specialised): a TMA producer warp, an MMA warp (one thread
+// issues every tcgen05.mma), and a 128-thread softmax warpgroup in which
+// thread r owns query row r (TMEM lane r).  The softmax warpgroup also
 // does the correction (rescaling the O row in TMEM when its running maximum
 // grows by more than 2^kRescaleLog2) and the epilogue (O / l, lse).
 #pragma once
@@ -35,16 +35,16 @@ namespace eta {
 // identical: O and l always share the same reference maximum).
 constexpr float kRescaleLog2 = 8.0f;
 
-// Columns (of every 8) whose exponential the ping-pong kernel computes with
-// the FMA-pipe polynomial; the rest use the MUFU ex2 unit.
+// Columns (of every 8) whose exponential the forward computes with the
+// FMA-pipe polynomial; the rest use the MUFU ex2 unit (0: measured fastest).
 #ifndef ETA_SOFT_EXP8
 #define ETA_SOFT_EXP8 0
 #endif
 constexpr int kSoftExp8 = ETA_SOFT_EXP8;
 
 #ifdef ETA_TRACE
-// Debug builds only: clock64() timelines of two CTAs of the ping-pong kernel
-// ([cta][role: softmax 0, softmax 1, MMA][key tile][event]).
+// Debug builds only: clock64() timelines of two CTAs of the dQ kernel
+// ([cta][role: elementwise warpgroup 0, 1, MMA][key tile][event]).
 __device__ unsigned long long g_eta_ftrace[2][3][256][4];
 #define ETA_FTRACE_AT(cta, role, it, ev)                                          \
   do {                                                                           \
