@@ -192,12 +192,17 @@ __device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&p)[BC
 }
 
 // e4m3 P for the kind::f8f6f4 P V product, as two terms so that P keeps about
-// 8 significant bits (one e4m3 term has 4): x = p * kP8Scale (p <= 1, so
-// x <= 256, inside e4m3's range; the scale keeps small probabilities out of
+// 8 significant bits (one e4m3 term has 4): x = p * kP8Scale (p <= 2^kP8Tau,
+// so x <= 256, inside e4m3's range; the scale keeps small probabilities out of
 // e4m3's subnormals), hi = e4m3(x), lo = e4m3(x - hi) (the residual, formed
 // in fp16, which holds both exactly enough).  hi goes to the first BC/4
 // columns, lo to the next BC/4, four values per 32-bit column.
-constexpr float kP8Scale = 256.f;
+// e4m3 builds rescale when the row maximum grows by more than 2^kP8Tau, so
+// p <= 2^kP8Tau and p * kP8Scale <= 256 (e4m3's largest finite value is 448).
+// Measured on B200: 2^3 runs 16 % faster than 2^0 (fewer rescales) with
+// max|dO|/max|O| 2.2e-3 against 2.2e-3 (the tolerance is 2e-2).
+constexpr int kP8Tau = 3;
+constexpr float kP8Scale = 256.f / static_cast<float>(1 << kP8Tau);
 template <int BC>
 __device__ __forceinline__ void tmem_store_p8(uint32_t taddr, const float (&p)[BC]) {
   static_assert(BC == 128 || BC == 64, "32 or 16 columns per term");
@@ -439,7 +444,7 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       apply_mask<BC>(s, col_window(BC * j, qrow, p.N, p.wl, p.wr));
       float alpha;
       const bool rescaled =
-          online_softmax_step<BC, kSoftExp8, C::FP8 ? 0 : static_cast<int>(kRescaleLog2)>(
+          online_softmax_step<BC, kSoftExp8, C::FP8 ? kP8Tau : static_cast<int>(kRescaleLog2)>(
               s, p.c, m, l, alpha);
       if constexpr (C::FP8) {
         tmem_store_p8<BC>(s_addr, s);

@@ -221,8 +221,8 @@ ATTN_API attn_status_t attn_bwd_noalloc(attn_tensor_t q, attn_tensor_t k, attn_t
  * the dequantised inputs (q_scale * q, ...) with the given softmax scale and
  * window (as attn_fwd_window): o [B, Hq, N, 128] bf16 and lse as attn_fwd.
  * Both products run on e4m3 tensor-core operands (kind::f8f6f4).  P (times
- * 256) enters P V as two e4m3 terms, its rounding and the rounding's residual,
- * so it keeps about 8 significant bits (a single e4m3 term keeps 4, which
+ * 32, with P <= 8 by the rescale rule) enters P V as two e4m3 terms, its
+ * rounding and the rounding's residual, so it keeps about 8 significant bits (a single e4m3 term keeps 4, which
  * puts the output's error near 5 % on random inputs).  D = 128 only (else
  * ATTN_ERR_UNSUPPORTED).
  */
