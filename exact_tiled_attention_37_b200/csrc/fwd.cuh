@@ -414,6 +414,10 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     *abort_flag = 0u;
     fence_barrier_init();
     fence_proxy_async_smem();
+    // the Q tile's load starts before TMEM allocation and the block-wide sync
+    mbar_expect_tx(BAR(C::BAR_Q), C::QTILE);
+    for (int c = 0; c < C::NCHUNK; ++c)
+      tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * C::EPC, q0, h, b);
   }
   if (warp == 5) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
@@ -479,13 +483,8 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     }
   } else if (warp == 4) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_expect_tx(BAR(C::BAR_Q), C::QTILE);
-      for (int c = 0; c < C::NCHUNK; ++c)
-        tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * C::EPC, q0, h,
-                    b);
       int it = 0;
       for (int u = 0, j = next_tile(j0); u < n && !W.aborted(); ++u, j = next_tile(j + 1)) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
