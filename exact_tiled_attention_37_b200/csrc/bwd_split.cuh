@@ -8,7 +8,10 @@
 //    dS = P (dP - Delta), dQ += dS K_j; dQ is written once, in bf16.
 //  * bwd_kv_kernel (column-parallel): per 128-row key tile, loop over the
 //    query heads of the group x 128-row query tiles: S^T = K Q_i^T,
-//    dP^T = V dO_i^T, P^T, dS^T, dV += P^T dO_i, dK += dS^T Q_i.
+//    dP^T = V dO_i^T, P^T, dS^T, dV += P^T dO_i, dK += dS^T Q_i.  Persistent:
+//    one CTA per SM walks its share of the key tiles (a static snake order
+//    over tiles sorted by work), with barrier phases carried from one key
+//    tile to the next, and writes dK, dV through TMA stores.
 //
 // Both read lse2 = lse log2(e) and Delta = rowsum(dO O) from the
 // preprocess kernel.  All MMAs are M = 128, N = 128 (or D) shapes, issued
