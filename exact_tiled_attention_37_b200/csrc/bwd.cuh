@@ -25,6 +25,10 @@
 //    finally stores dK, dV), and a 128-thread dQ warpgroup (thread d owns
 //    column d of dQ^T: drains dQ_i^T from TMEM and issues coalesced fp32
 //    reductions into the scratch).
+//    Shared memory holds one Q / dO tile, loaded in two parts: the D chunks
+//    outside this CTA's slice are read only by S^T and dP^T, so the next
+//    tile's part is loaded, and its S^T / dP^T steps run, under this tile's
+//    softmax; the slice's own chunks follow once dV and dK are done.
 //  * bwd_dq_finalize_kernel: dQ (bf16, caller's strides) from the scratch.
 //
 // TMEM (512 columns): ST[2] (64 each: S^T, then P^T and dS^T packed) |
@@ -221,7 +225,12 @@ struct BwdCfg {
   static constexpr int B_DQE = 5 + 2 * NQS + 2 * NPB;     // [2]
   static constexpr int B_KVD = 7 + 2 * NQS + 2 * NPB;     // dK/dV accumulated
   static constexpr int B_DONE = 8 + 2 * NQS + 2 * NPB;
-  static constexpr int NBAR = 9 + 2 * NQS + 2 * NPB;
+  // the Q / dO chunks outside this CTA's D slice (read only by S^T and dP^T)
+  // have barriers of their own: they are free again as soon as those two
+  // products are done, while the slice's own chunks wait for dV and dK
+  static constexpr int B_OF = 9 + 2 * NQS + 2 * NPB;
+  static constexpr int B_OE = 10 + 2 * NQS + 2 * NPB;
+  static constexpr int NBAR = 11 + 2 * NQS + 2 * NPB;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = S_MISC + 16 + 1024;
   // warps: 0-3 softmax (query columns 0-31 of every tile), 4-7 dQ drain,
@@ -279,6 +288,7 @@ __global__ void __launch_bounds__(512, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<DFULL, NQS, NPB>;
+  static_assert(NQS == 1 && C::DSPLIT == 2, "one Q/dO stage, split into the two D slices");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -289,12 +299,17 @@ __global__ void __launch_bounds__(512, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid (Hkv * D-slices, B, key tiles): the key tile varies slowest, and
-  // causal tile 0 (the most work) of every head is dispatched first
-  const int kt = blockIdx.z;
-  const int hk = blockIdx.x / C::DSPLIT;
-  const int half = blockIdx.x % C::DSPLIT;
-  const int b = blockIdx.y;
+  // grid (Hkv * D-slices, B, key tiles).  Masked problems: the key tile
+  // varies slowest, so causal tile 0 (the most work) of every head is
+  // dispatched first.  Unmasked problems (equal work per CTA): the key tile
+  // varies fastest, so the CTAs of one head run together and share its Q /
+  // dO tiles and dQ rows in L2.
+  const bool kt_fast = p.wl < 0 && p.wr < 0;
+  const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  const int kt = kt_fast ? lin % gridDim.z : blockIdx.z;
+  const int hk = kt_fast ? lin / gridDim.z / C::DSPLIT % p.Hkv : blockIdx.x / C::DSPLIT;
+  const int half = kt_fast ? lin / gridDim.z % C::DSPLIT : blockIdx.x % C::DSPLIT;
+  const int b = kt_fast ? lin / gridDim.z / C::DSPLIT / p.Hkv : blockIdx.y;
   const int k0 = kt * C::BC;
   // queries that see any key of [k0, k0 + BC): key j is visible to query i iff
   // j - wr <= i <= j + wl
@@ -321,6 +336,8 @@ __global__ void __launch_bounds__(512, 1)
     }
     mbar_init(BAR(C::B_KVD), 1);
     mbar_init(BAR(C::B_DONE), 1);
+    mbar_init(BAR(C::B_OF), 1);
+    mbar_init(BAR(C::B_OE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -469,29 +486,36 @@ __global__ void __launch_bounds__(512, 1)
         tma_load_4d(sbase + C::S_K + c * C::KCHUNK, &tm_k, BAR(C::B_KV), c * 64, k0, hk, b);
         tma_load_4d(sbase + C::S_V + c * C::KCHUNK, &tm_v, BAR(C::B_KV), c * 64, k0, hk, b);
       }
-      int it = 0;
+      // Q / dO chunks 2 half, 2 half + 1 are this CTA's D slice ("own"), the
+      // other two are read only by S^T and dP^T
+      const int c_own = 2 * half, c_oth = 2 - 2 * half;
+      int it = 0, oth_issued = 0;
       for (; it < n; ++it) {
-        const int stage = it % NQS;
-        if (!W.wait(BAR(C::B_QE + stage), ((it / NQS) & 1) ^ 1, 80)) break;
-        ETA_TRACE_AT(tcta, 3, it, 0);
         const int h = head_of(it);
         const int ig0 = qtile_of(it) * C::BR;
-        const uint32_t full = BAR(C::B_QF + stage);
-        mbar_expect_tx(full, 2 * C::QTILE + 512);
-        for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d(sbase + C::S_Q + stage * C::QTILE + c * C::QCHUNK, &tm_q, full, c * 64, ig0, h, b);
-          tma_load_4d(sbase + C::S_DO + stage * C::QTILE + c * C::QCHUNK, &tm_do, full, c * 64, ig0, h, b);
+        if (!W.wait(BAR(C::B_OE), (it & 1) ^ 1, 80)) break;
+        ETA_TRACE_AT(tcta, 3, it, 0);
+        mbar_expect_tx(BAR(C::B_OF), 4 * C::QCHUNK);
+        for (int c = c_oth; c < c_oth + 2; ++c) {
+          tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, BAR(C::B_OF), c * 64, ig0, h, b);
+          tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, BAR(C::B_OF), c * 64, ig0, h, b);
+        }
+        ++oth_issued;
+        if (!W.wait(BAR(C::B_QE), (it & 1) ^ 1, 84)) break;
+        ETA_TRACE_AT(tcta, 3, it, 1);
+        const uint32_t full = BAR(C::B_QF);
+        mbar_expect_tx(full, 4 * C::QCHUNK + 512);
+        for (int c = c_own; c < c_own + 2; ++c) {
+          tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, full, c * 64, ig0, h, b);
+          tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, full, c * 64, ig0, h, b);
         }
         const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
-        bulk_load(sbase + C::S_STAT + stage * 512, p.lse2 + srow, 256, full);
-        bulk_load(sbase + C::S_STAT + stage * 512 + 256, p.delta + srow, 256, full);
+        bulk_load(sbase + C::S_STAT, p.lse2 + srow, 256, full);
+        bulk_load(sbase + C::S_STAT + 256, p.delta + srow, 256, full);
       }
       W.drain(BAR(C::B_KV), 0, 81);
-      const int issued = it;
-      for (int s = 0; s < NQS && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / NQS) * NQS;
-        W.drain(BAR(C::B_QF + s), static_cast<uint32_t>(last / NQS) & 1u, 82);
-      }
+      if (it > 0) W.drain(BAR(C::B_QF), static_cast<uint32_t>(it - 1) & 1u, 82);
+      if (oth_issued > 0) W.drain(BAR(C::B_OF), static_cast<uint32_t>(oth_issued - 1) & 1u, 83);
     }
     __syncwarp();
   } else if (warp == 13) {
@@ -504,55 +528,55 @@ __global__ void __launch_bounds__(512, 1)
       const SDesc dV = sdesc_base(sbase + C::S_V, 16, 1024);
       // K^T for dQ^T: MN-major view of this CTA's D slice of the K tile
       const SDesc dKt = sdesc_base(sbase + C::S_K + half * 2 * C::KCHUNK, C::KCHUNK, 1024);
-      auto issue_sdp = [&](int it) {
-        const int buf = it & 1, stage = it % NQS;
-        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::QTILE, 16, 1024);
-        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::QTILE, 16, 1024);
+      // S^T and dP^T over the two 64-column chunks c0, c0 + 1 of D (8 steps each)
+      auto issue_sdp = [&](int it, int c0, bool first) {
+        const int buf = it & 1;
+        const SDesc dq = sdesc_base(sbase + C::S_Q, 16, 1024);
+        const SDesc ddo = sdesc_base(sbase + C::S_DO, 16, 1024);
         const uint32_t ds = tmem + C::T_ST + 64 * buf, ddp = tmem + C::T_DPT + 64 * buf;
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t ko = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
-          const uint32_t qo = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
-          mma_ss<false>(ds, sdesc_at(dK, ko), sdesc_at(dq, qo), id_s, ks > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (c0 + (kk >> 2)) * C::KCHUNK + (kk & 3) * 32;
+          const uint32_t qo = (c0 + (kk >> 2)) * C::QCHUNK + (kk & 3) * 32;
+          mma_ss<false>(ds, sdesc_at(dK, ko), sdesc_at(dq, qo), id_s, !first || kk > 0);
         }
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t ko = (ks >> 2) * C::KCHUNK + (ks & 3) * 32;
-          const uint32_t qo = (ks >> 2) * C::QCHUNK + (ks & 3) * 32;
-          mma_ss<false>(ddp, sdesc_at(dV, ko), sdesc_at(ddo, qo), id_s, ks > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (c0 + (kk >> 2)) * C::KCHUNK + (kk & 3) * 32;
+          const uint32_t qo = (c0 + (kk >> 2)) * C::QCHUNK + (kk & 3) * 32;
+          mma_ss<false>(ddp, sdesc_at(dV, ko), sdesc_at(ddo, qo), id_s, !first || kk > 0);
         }
       };
-      bool ok = W.wait(BAR(C::B_KV), 0, 90) && (n == 0 || W.wait(BAR(C::B_QF), 0, 91));
+      const int c_own = 2 * half, c_oth = 2 - 2 * half;
+      // tile 0: the other slice's chunks, then this slice's
+      bool ok = W.wait(BAR(C::B_KV), 0, 90) &&
+                (n == 0 || (W.wait(BAR(C::B_OF), 0, 91) && W.wait(BAR(C::B_QF), 0, 96)));
       if (ok && n > 0) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_sdp(0, c_oth, true);
+        mma_commit(BAR(C::B_OE));
+        issue_sdp(0, c_own, false);
         mma_commit(BAR(C::B_SP + 0));
       }
-      // S^T / dP^T of the next iteration go into the other TMEM buffers once
-      // the dQ warpgroup has drained the dQ^T that last used that dP^T buffer.
-      auto issue_next = [&](int it) -> bool {
-        const int b1 = (it + 1) & 1, st1 = (it + 1) % NQS;
-        if (it >= 1 && !W.wait(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1, 92)) return false;
-        if (!W.wait(BAR(C::B_QF + st1), ((it + 1) / NQS) & 1, 93)) return false;
-        tc_fence_after();
-        issue_sdp(it + 1);
-        mma_commit(BAR(C::B_SP + b1));
-        return true;
-      };
       for (int it = 0; ok && it < n; ++it) {
-        const int buf = it & 1, stage = it % NQS, pb = it % NPB;
+        const int buf = it & 1, b1 = (it + 1) & 1, pb = it % NPB;
         ETA_TRACE_AT(tcta, 2, it, 0);
-        // With two Q/dO stages the next tile's products overlap this tile's
-        // softmax; with one stage they must wait for this tile's products.
-        if (NQS > 1 && it + 1 < n && !issue_next(it)) { ok = false; break; }
+        // S^T / dP^T of the next tile over the other slice's chunks run under
+        // this tile's softmax, into the other TMEM buffers once the dQ
+        // warpgroup has drained the dQ^T that last used that dP^T buffer
+        if (it + 1 < n) {
+          if (it >= 1 && !W.wait(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1, 92)) { ok = false; break; }
+          if (!W.wait(BAR(C::B_OF), (it + 1) & 1, 93)) { ok = false; break; }
+          tc_fence_after();
+          issue_sdp(it + 1, c_oth, true);
+          mma_commit(BAR(C::B_OE));
+        }
         ETA_TRACE_AT(tcta, 2, it, 1);
         if (!W.wait(BAR(C::B_DS + pb), (it / NPB) & 1, 94)) { ok = false; break; }
         ETA_TRACE_AT(tcta, 2, it, 2);
         tc_fence_after();
-        const SDesc dq = sdesc_base(sbase + C::S_Q + stage * C::QTILE + half * 2 * C::QCHUNK,
-                                    C::QCHUNK, 1024);
-        const SDesc ddo = sdesc_base(sbase + C::S_DO + stage * C::QTILE + half * 2 * C::QCHUNK,
-                                     C::QCHUNK, 1024);
+        const SDesc dq = sdesc_base(sbase + C::S_Q + half * 2 * C::QCHUNK, C::QCHUNK, 1024);
+        const SDesc ddo = sdesc_base(sbase + C::S_DO + half * 2 * C::QCHUNK, C::QCHUNK, 1024);
         const SDesc dds = sdesc_base(sbase + C::S_DS + pb * C::PTILE, C::PTILE, 1024);
         const uint32_t tst = tmem + C::T_ST + 64 * buf, tdp = tmem + C::T_DPT + 64 * buf;
         const uint32_t acc0 = it > 0 ? 1u : 0u;
@@ -574,10 +598,16 @@ __global__ void __launch_bounds__(512, 1)
         for (int ks = 0; ks < 4; ++ks)
           mma_ts<false>(tmem + C::T_DK, tst + 32 * (ks >> 1) + 16 + 8 * (ks & 1),
                         sdesc_at(dq, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-        mma_commit(BAR(C::B_QE + stage));
+        mma_commit(BAR(C::B_QE));
         mma_commit(BAR(C::B_PE + pb));
         ETA_TRACE_AT(tcta, 2, it, 3);
-        if (NQS == 1 && it + 1 < n && !issue_next(it)) { ok = false; break; }
+        // the next tile's own-slice chunks arrive once dV and dK are done with these
+        if (it + 1 < n) {
+          if (!W.wait(BAR(C::B_QF), (it + 1) & 1, 97)) { ok = false; break; }
+          tc_fence_after();
+          issue_sdp(it + 1, c_own, false);
+          mma_commit(BAR(C::B_SP + b1));
+        }
       }
       if (ok) mma_commit(BAR(C::B_KVD));
       mma_commit(BAR(C::B_DONE));
