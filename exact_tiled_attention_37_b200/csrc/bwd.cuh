@@ -228,9 +228,13 @@ struct BwdCfg {
   // the Q / dO chunks outside this CTA's D slice (read only by S^T and dP^T)
   // have barriers of their own: they are free again as soon as those two
   // products are done, while the slice's own chunks wait for dV and dK
+  // B_QF / B_QE: the slice's own dO chunks and the row statistics (free
+  // after dV); B_WF / B_WE: the slice's own Q chunks (free after dK)
   static constexpr int B_OF = 9 + 2 * NQS + 2 * NPB;
   static constexpr int B_OE = 10 + 2 * NQS + 2 * NPB;
-  static constexpr int NBAR = 11 + 2 * NQS + 2 * NPB;
+  static constexpr int B_WF = 11 + 2 * NQS + 2 * NPB;
+  static constexpr int B_WE = 12 + 2 * NQS + 2 * NPB;
+  static constexpr int NBAR = 13 + 2 * NQS + 2 * NPB;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = S_MISC + 16 + 1024;
   // warps: 0-3 softmax (query columns 0-31 of every tile), 4-7 dQ drain,
@@ -338,6 +342,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(C::B_DONE), 1);
     mbar_init(BAR(C::B_OF), 1);
     mbar_init(BAR(C::B_OE), 1);
+    mbar_init(BAR(C::B_WF), 1);
+    mbar_init(BAR(C::B_WE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(512, 1)
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 
 #ifdef ETA_TRACE
-  const int tcta = (blockIdx.x == 0 && blockIdx.y == 0) ? (kt == 0 ? 0 : (kt == 16 ? 1 : -1)) : -1;
+  const int tcta = lin == 0 ? 0 : (lin == 37 ? 1 : -1);
 #else
   const int tcta = -1;
 #endif
@@ -489,7 +495,7 @@ __global__ void __launch_bounds__(512, 1)
       // Q / dO chunks 2 half, 2 half + 1 are this CTA's D slice ("own"), the
       // other two are read only by S^T and dP^T
       const int c_own = 2 * half, c_oth = 2 - 2 * half;
-      int it = 0, oth_issued = 0;
+      int it = 0, oth_issued = 0, do_issued = 0;
       for (; it < n; ++it) {
         const int h = head_of(it);
         const int ig0 = qtile_of(it) * C::BR;
@@ -503,18 +509,22 @@ __global__ void __launch_bounds__(512, 1)
         ++oth_issued;
         if (!W.wait(BAR(C::B_QE), (it & 1) ^ 1, 84)) break;
         ETA_TRACE_AT(tcta, 3, it, 1);
-        const uint32_t full = BAR(C::B_QF);
-        mbar_expect_tx(full, 4 * C::QCHUNK + 512);
-        for (int c = c_own; c < c_own + 2; ++c) {
-          tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, full, c * 64, ig0, h, b);
-          tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, full, c * 64, ig0, h, b);
-        }
+        mbar_expect_tx(BAR(C::B_QF), 2 * C::QCHUNK + 512);
+        for (int c = c_own; c < c_own + 2; ++c)
+          tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, BAR(C::B_QF), c * 64, ig0, h, b);
         const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
-        bulk_load(sbase + C::S_STAT, p.lse2 + srow, 256, full);
-        bulk_load(sbase + C::S_STAT + 256, p.delta + srow, 256, full);
+        bulk_load(sbase + C::S_STAT, p.lse2 + srow, 256, BAR(C::B_QF));
+        bulk_load(sbase + C::S_STAT + 256, p.delta + srow, 256, BAR(C::B_QF));
+        ++do_issued;
+        if (!W.wait(BAR(C::B_WE), (it & 1) ^ 1, 85)) break;
+        ETA_TRACE_AT(tcta, 3, it, 2);
+        mbar_expect_tx(BAR(C::B_WF), 2 * C::QCHUNK);
+        for (int c = c_own; c < c_own + 2; ++c)
+          tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, BAR(C::B_WF), c * 64, ig0, h, b);
       }
       W.drain(BAR(C::B_KV), 0, 81);
-      if (it > 0) W.drain(BAR(C::B_QF), static_cast<uint32_t>(it - 1) & 1u, 82);
+      if (do_issued > 0) W.drain(BAR(C::B_QF), static_cast<uint32_t>(do_issued - 1) & 1u, 82);
+      if (it > 0) W.drain(BAR(C::B_WF), static_cast<uint32_t>(it - 1) & 1u, 86);
       if (oth_issued > 0) W.drain(BAR(C::B_OF), static_cast<uint32_t>(oth_issued - 1) & 1u, 83);
     }
     __syncwarp();
@@ -528,48 +538,54 @@ __global__ void __launch_bounds__(512, 1)
       const SDesc dV = sdesc_base(sbase + C::S_V, 16, 1024);
       // K^T for dQ^T: MN-major view of this CTA's D slice of the K tile
       const SDesc dKt = sdesc_base(sbase + C::S_K + half * 2 * C::KCHUNK, C::KCHUNK, 1024);
-      // S^T and dP^T over the two 64-column chunks c0, c0 + 1 of D (8 steps each)
-      auto issue_sdp = [&](int it, int c0, bool first) {
-        const int buf = it & 1;
-        const SDesc dq = sdesc_base(sbase + C::S_Q, 16, 1024);
-        const SDesc ddo = sdesc_base(sbase + C::S_DO, 16, 1024);
-        const uint32_t ds = tmem + C::T_ST + 64 * buf, ddp = tmem + C::T_DPT + 64 * buf;
+      // S^T (K Q_i^T) or dP^T (V dO_i^T) over the 64-column chunks c0, c0 + 1
+      // of D (8 steps)
+      auto issue_half = [&](bool dp, int it, int c0, bool first) {
+        const SDesc a = dp ? dV : dK;
+        const SDesc bq = sdesc_base(sbase + (dp ? C::S_DO : C::S_Q), 16, 1024);
+        const uint32_t d = tmem + (dp ? C::T_DPT : C::T_ST) + 64 * (it & 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t ko = (c0 + (kk >> 2)) * C::KCHUNK + (kk & 3) * 32;
           const uint32_t qo = (c0 + (kk >> 2)) * C::QCHUNK + (kk & 3) * 32;
-          mma_ss<false>(ds, sdesc_at(dK, ko), sdesc_at(dq, qo), id_s, !first || kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (c0 + (kk >> 2)) * C::KCHUNK + (kk & 3) * 32;
-          const uint32_t qo = (c0 + (kk >> 2)) * C::QCHUNK + (kk & 3) * 32;
-          mma_ss<false>(ddp, sdesc_at(dV, ko), sdesc_at(ddo, qo), id_s, !first || kk > 0);
+          mma_ss<false>(d, sdesc_at(a, ko), sdesc_at(bq, qo), id_s, !first || kk > 0);
         }
       };
       const int c_own = 2 * half, c_oth = 2 - 2 * half;
-      // tile 0: the other slice's chunks, then this slice's
-      bool ok = W.wait(BAR(C::B_KV), 0, 90) &&
-                (n == 0 || (W.wait(BAR(C::B_OF), 0, 91) && W.wait(BAR(C::B_QF), 0, 96)));
-      if (ok && n > 0) {
+      auto issue_other = [&](int it) {
         tc_fence_after();
-        issue_sdp(0, c_oth, true);
+        issue_half(false, it, c_oth, true);
+        issue_half(true, it, c_oth, true);
         mma_commit(BAR(C::B_OE));
-        issue_sdp(0, c_own, false);
-        mma_commit(BAR(C::B_SP + 0));
+      };
+      // this slice's chunks: dP^T as soon as dO has arrived, then S^T
+      auto issue_own = [&](int it) -> bool {
+        if (!W.wait(BAR(C::B_QF), it & 1, 97)) return false;
+        tc_fence_after();
+        issue_half(true, it, c_own, false);
+        if (!W.wait(BAR(C::B_WF), it & 1, 98)) return false;
+        tc_fence_after();
+        issue_half(false, it, c_own, false);
+        mma_commit(BAR(C::B_SP + (it & 1)));
+        return true;
+      };
+      bool ok = W.wait(BAR(C::B_KV), 0, 90) && (n == 0 || W.wait(BAR(C::B_OF), 0, 91));
+      if (ok && n > 0) {
+        issue_other(0);
+        ok = issue_own(0);
       }
       for (int it = 0; ok && it < n; ++it) {
         const int buf = it & 1, b1 = (it + 1) & 1, pb = it % NPB;
         ETA_TRACE_AT(tcta, 2, it, 0);
-        // S^T / dP^T of the next tile over the other slice's chunks run under
-        // this tile's softmax, into the other TMEM buffers once the dQ
-        // warpgroup has drained the dQ^T that last used that dP^T buffer
-        if (it + 1 < n) {
-          if (it >= 1 && !W.wait(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1, 92)) { ok = false; break; }
-          if (!W.wait(BAR(C::B_OF), (it + 1) & 1, 93)) { ok = false; break; }
-          tc_fence_after();
-          issue_sdp(it + 1, c_oth, true);
-          mma_commit(BAR(C::B_OE));
+        // The next tile's S^T / dP^T over the other slice's chunks go into the
+        // other TMEM buffers (once the dQ warpgroup has drained the dQ^T that
+        // last used that dP^T buffer) and run under this tile's softmax, if
+        // their chunks have landed; otherwise after this tile's products.
+        bool other_issued = false;
+        if (it + 1 < n && (it == 0 || mbar_test(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1)) &&
+            mbar_test(BAR(C::B_OF), (it + 1) & 1)) {
+          issue_other(it + 1);
+          other_issued = true;
         }
         ETA_TRACE_AT(tcta, 2, it, 1);
         if (!W.wait(BAR(C::B_DS + pb), (it / NPB) & 1, 94)) { ok = false; break; }
@@ -580,33 +596,35 @@ __global__ void __launch_bounds__(512, 1)
         const SDesc dds = sdesc_base(sbase + C::S_DS + pb * C::PTILE, C::PTILE, 1024);
         const uint32_t tst = tmem + C::T_ST + 64 * buf, tdp = tmem + C::T_DPT + 64 * buf;
         const uint32_t acc0 = it > 0 ? 1u : 0u;
-        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed dP^T
-        // buffer, first, so that the dQ warpgroup drains it while dV and dK run
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss<false>(tdp, sdesc_at(dKt, ks * 2048), sdesc_at(dds, ks * 2048), id_q, ks > 0);
-        mma_commit(BAR(C::B_DQF + buf));
         // P^T / dS^T of query rows [16 ks, 16 ks + 16) sit at S^T column
         // 32 (ks / 2) + 8 (ks % 2) (+ 16 for dS^T)
-        // dV += P^T dO_i with P^T read from TMEM (K = 64 query rows, 4 steps of 16)
+        // dV += P^T dO_i with P^T read from TMEM (K = 64 query rows, 4 steps of 16);
+        // then the slice's dO chunks and the statistics are free
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_ts<false>(tmem + C::T_DV, tst + 32 * (ks >> 1) + 8 * (ks & 1), sdesc_at(ddo, ks * 2048),
                         id_kv, ks > 0 ? 1u : acc0);
-        // dK += dS^T Q_i with dS^T read from TMEM
+        mma_commit(BAR(C::B_QE));
+        // dK += dS^T Q_i with dS^T read from TMEM; then the slice's Q chunks are free
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_ts<false>(tmem + C::T_DK, tst + 32 * (ks >> 1) + 16 + 8 * (ks & 1),
                         sdesc_at(dq, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-        mma_commit(BAR(C::B_QE));
+        mma_commit(BAR(C::B_WE));
+        // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed dP^T buffer
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss<false>(tdp, sdesc_at(dKt, ks * 2048), sdesc_at(dds, ks * 2048), id_q, ks > 0);
+        mma_commit(BAR(C::B_DQF + buf));
         mma_commit(BAR(C::B_PE + pb));
         ETA_TRACE_AT(tcta, 2, it, 3);
-        // the next tile's own-slice chunks arrive once dV and dK are done with these
         if (it + 1 < n) {
-          if (!W.wait(BAR(C::B_QF), (it + 1) & 1, 97)) { ok = false; break; }
-          tc_fence_after();
-          issue_sdp(it + 1, c_own, false);
-          mma_commit(BAR(C::B_SP + b1));
+          if (!other_issued) {
+            if (it >= 1 && !W.wait(BAR(C::B_DQE + b1), ((it - 1) >> 1) & 1, 92)) { ok = false; break; }
+            if (!W.wait(BAR(C::B_OF), (it + 1) & 1, 93)) { ok = false; break; }
+            issue_other(it + 1);
+          }
+          if (!issue_own(it + 1)) { ok = false; break; }
         }
       }
       if (ok) mma_commit(BAR(C::B_KVD));
