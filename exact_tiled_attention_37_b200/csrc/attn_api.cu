@@ -188,7 +188,7 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
       return ATTN_ERR_CUDA;
   }
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
-  eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
+  eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows / eta::kPrepRows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
   auto kern = eta::bwd_dkdv_kernel<D, NQS, NPB>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
@@ -220,7 +220,7 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   if ((s = make_map(&tk, k, p.B, p.Hkv, p.N, D, 2, 128)) != ATTN_OK) return s;
   if ((s = make_map(&tv, v, p.B, p.Hkv, p.N, D, 2, 128)) != ATTN_OK) return s;
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
-  eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
+  eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows / eta::kPrepRows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
   auto kkv = eta::bwd_kv_kernel<D, NQS, NWG>;
   auto kq = eta::bwd_q_kernel<D, NS, NWG>;

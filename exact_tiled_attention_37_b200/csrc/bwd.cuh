@@ -16,7 +16,7 @@
 //  * bwd_preprocess_kernel: Delta = rowsum(dO * O) and lse2 = lse * log2(e)
 //    per row (rows past N padded with Delta = 0, lse2 = +inf so that their P
 //    is exactly 0), and zeroes the fp32 dQ scratch (head dimension 256).
-//    D/8 threads per row.  Shared with the kernels of bwd_split.cuh.
+//    D/8 threads per group of 4 rows.  Shared with the kernels of bwd_split.cuh.
 //  * bwd_dkdv_kernel: one CTA per (batch, key/value head, 128-row key tile,
 //    128-column slice of D); loops over the query heads of the GQA group and
 //    the 64-row query tiles (causal: only tiles at or below the diagonal).
@@ -25,10 +25,11 @@
 //    finally stores dK, dV), and a 128-thread dQ warpgroup (thread d owns
 //    column d of dQ^T: drains dQ_i^T from TMEM and issues coalesced fp32
 //    reductions into the scratch).
-//    Shared memory holds one Q / dO tile, loaded in two parts: the D chunks
-//    outside this CTA's slice are read only by S^T and dP^T, so the next
-//    tile's part is loaded, and its S^T / dP^T steps run, under this tile's
-//    softmax; the slice's own chunks follow once dV and dK are done.
+//    Shared memory holds one Q / dO tile, loaded in three parts: the D
+//    chunks outside this CTA's slice are read only by S^T and dP^T, so the
+//    next tile's part is loaded, and its S^T / dP^T steps run, under this
+//    tile's softmax; the slice's own dO chunks follow once dV is done, its
+//    Q chunks once dK is done.
 //  * bwd_dq_finalize_kernel: dQ (bf16, caller's strides) from the scratch.
 //
 // TMEM (512 columns): ST[2] (64 each: S^T, then P^T and dS^T packed) |
@@ -107,54 +108,79 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------- preprocess
-// D/8 threads per row, each reading 16 bytes of O and of dO; a block of 256
-// threads covers 256 / (D/8) rows.  Rows past N get Delta = 0, lse2 = +inf.
+// A group of D/8 threads covers kPrepRows consecutive rows, each thread
+// reading 16 bytes of O and of dO per row; all of a thread's loads are issued
+// before the first use, for enough bytes in flight to stream O and dO at HBM
+// speed.  Rows past N get Delta = 0, lse2 = +inf.
+constexpr int kPrepRows = 4;
+static_assert(kBwdRowPad % kPrepRows == 0, "row groups never straddle a head");
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdParams p) {
   constexpr int TPR = D / 8;  // threads per row (8, 16 or 32)
+  constexpr int R = kPrepRows;
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = t / TPR;  // over B * Hq * Npad
+  const long long row0 = t / TPR * R;  // first of R rows over B * Hq * Npad
   const int part = static_cast<int>(t % TPR);
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
-  // (the launch covers exactly rows * TPR threads; the guard keeps every lane
-  // in the shuffles below either way)
-  const bool in_range = row < rows;
-  const int bh = static_cast<int>(row / p.Npad);
-  const int i = static_cast<int>(row % p.Npad);
+  // (Npad is a multiple of R, so the R rows share one (batch, head); the
+  // guard keeps every lane in the shuffles below)
+  const bool in_range = row0 < rows;
+  const int bh = static_cast<int>(row0 / p.Npad);
+  const int i0 = static_cast<int>(row0 % p.Npad);
   const int b = bh / p.Hq, h = bh % p.Hq;
-  float acc = 0.f;
-  if (in_range && i < p.N) {
-    const uint4 ov = *reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(p.o) + b * p.osb + h * p.osh +
-        static_cast<long long>(i) * p.osn + 8 * part);
-    const uint4 dv = *reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(p.dout) + b * p.dosb + h * p.dosh +
-        static_cast<long long>(i) * p.dosn + 8 * part);
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+  const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(p.o) + b * p.osb + h * p.osh +
+                              static_cast<long long>(i0) * p.osn + 8 * part;
+  const __nv_bfloat16* drow = static_cast<const __nv_bfloat16*>(p.dout) + b * p.dosb +
+                              h * p.dosh + static_cast<long long>(i0) * p.dosn + 8 * part;
+  uint4 ov[R], dv[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const bool live = in_range && i0 + r < p.N;
+    ov[r] = live ? *reinterpret_cast<const uint4*>(orow + r * p.osn) : make_uint4(0, 0, 0, 0);
+    dv[r] = live ? *reinterpret_cast<const uint4*>(drow + r * p.dosn) : make_uint4(0, 0, 0, 0);
+  }
+  // zero this part of the fp32 dQ scratch rows (when dQ is accumulated there)
+  if (p.dqacc) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (in_range && i0 + r < p.N) {
+        float4* z = reinterpret_cast<float4*>(
+            p.dqacc + (static_cast<long long>(bh) * p.N + i0 + r) * D + 8 * part);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+  float acc[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[r]);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv[r]);
+    acc[r] = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 of = __bfloat1622float2(o2[e]);
       const float2 df = __bfloat1622float2(d2[e]);
-      acc = fmaf(of.x, df.x, acc);
-      acc = fmaf(of.y, df.y, acc);
+      acc[r] = fmaf(of.x, df.x, acc[r]);
+      acc[r] = fmaf(of.y, df.y, acc[r]);
     }
-    // zero this part of the fp32 dQ scratch row (when dQ is accumulated there)
-    if (p.dqacc) {
-      float4* z = reinterpret_cast<float4*>(p.dqacc + (static_cast<long long>(bh) * p.N + i) * D +
-                                            8 * part);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
 #pragma unroll
-  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (in_range && part == 0) {
-    p.delta[row] = acc;
+    for (int off = TPR / 2; off > 0; off >>= 1)
+      acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
+  }
+  // thread r of the group writes row r
+  if (in_range && part < R) {
+    float a = acc[0];
+#pragma unroll
+    for (int r = 1; r < R; ++r)
+      if (part == r) a = acc[r];
+    const int i = i0 + part;
+    p.delta[row0 + part] = a;
     // rows past N, and rows that saw no key (lse = -inf), get lse2 = +inf so
     // that their P is exactly 0
     const float l = i < p.N ? p.lse[static_cast<long long>(bh) * p.N + i] : -INFINITY;
-    p.lse2[row] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
+    p.lse2[row0 + part] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
   }
 }
 
