@@ -254,13 +254,15 @@ struct BwdCfg {
   // the Q / dO chunks outside this CTA's D slice (read only by S^T and dP^T)
   // have barriers of their own: they are free again as soon as those two
   // products are done, while the slice's own chunks wait for dV and dK
-  // B_QF / B_QE: the slice's own dO chunks and the row statistics (free
-  // after dV); B_WF / B_WE: the slice's own Q chunks (free after dK)
+  // B_WF / B_WE: the slice's own Q chunks and the row statistics (free
+  // after dK); B_QF / B_QE: the slice's own dO chunks (free after dV)
   static constexpr int B_OF = 9 + 2 * NQS + 2 * NPB;
   static constexpr int B_OE = 10 + 2 * NQS + 2 * NPB;
   static constexpr int B_WF = 11 + 2 * NQS + 2 * NPB;
   static constexpr int B_WE = 12 + 2 * NQS + 2 * NPB;
-  static constexpr int NBAR = 13 + 2 * NQS + 2 * NPB;
+  // B_SP[2] signals S^T complete, B_SPD[2] dP^T complete
+  static constexpr int B_SPD = 13 + 2 * NQS + 2 * NPB;   // [2]
+  static constexpr int NBAR = 15 + 2 * NQS + 2 * NPB;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = S_MISC + 16 + 1024;
   // warps: 0-3 softmax (query columns 0-31 of every tile), 4-7 dQ drain,
@@ -270,21 +272,35 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// P^T and dS^T for 32 query columns [c0, c0 + 32) of this thread's key row:
-// loads S^T and dP^T from TMEM, applies exp2 / causal mask / softmax
-// Jacobian, and writes P^T and dS^T as bf16 pairs into the 32 S^T columns it
-// has just read (P^T at columns c0 .. c0 + 15, dS^T at c0 + 16 .. c0 + 31:
-// the A operands of dV += P^T dO and dK += dS^T Q), and dS^T also as a bf16
-// shared-memory row (4 swizzled 16-byte chunks: the B operand of
-// dQ^T = K^T dS^T).  The dP^T columns are left free for dQ^T.
-__device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr, int c0,
-                                             const float* lse2, const float* dlt, float c,
-                                             int ilo, int ihi, uint8_t* drow, int swz) {
-  uint32_t rs[32], rd[32];
+// P^T for 32 query columns [c0, c0 + 32) of this thread's key row: loads S^T
+// from TMEM and applies exp2(S^T c - lse2) and the window mask, into pv.
+__device__ __forceinline__ void bwd_row_p(uint32_t st_addr, int c0, const float* lse2, float c,
+                                          int ilo, int ihi, float (&pv)[32]) {
+  uint32_t rs[32];
   tmem_ld32(st_addr + c0, rs);
-  tmem_ld32(dpt_addr + c0, rd);
   tmem_wait_ld();
   const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 l2 = *reinterpret_cast<const float2*>(lse2 + c0 + i);
+    const float2 x = ffma2(make_float2(u2f(rs[i]), u2f(rs[i + 1])), c2, make_float2(-l2.x, -l2.y));
+    pv[i] = (c0 + i < ilo || c0 + i > ihi) ? 0.f : ex2(x.x);
+    pv[i + 1] = (c0 + i + 1 < ilo || c0 + i + 1 > ihi) ? 0.f : ex2(x.y);
+  }
+}
+
+// dS^T = P^T * (dP^T - Delta) for the same columns: loads dP^T from TMEM and
+// writes P^T and dS^T as bf16 pairs into the 32 S^T columns read before (P^T
+// at columns c0 .. c0 + 15, dS^T at c0 + 16 .. c0 + 31: the A operands of
+// dV += P^T dO and dK += dS^T Q), and dS^T also as a bf16 shared-memory row
+// (4 swizzled 16-byte chunks: the B operand of dQ^T = K^T dS^T).  The dP^T
+// columns are left free for dQ^T.
+__device__ __forceinline__ void bwd_row_ds(uint32_t st_addr, uint32_t dpt_addr, int c0,
+                                           const float* dlt, const float (&pv)[32], uint8_t* drow,
+                                           int swz) {
+  uint32_t rd[32];
+  tmem_ld32(dpt_addr + c0, rd);
+  tmem_wait_ld();
   uint32_t pk[16], dk[16];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -292,16 +308,10 @@ __device__ __forceinline__ void bwd_row_half(uint32_t st_addr, uint32_t dpt_addr
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int i = 8 * u + 2 * e;  // column within this half
-      const float2 l2 = *reinterpret_cast<const float2*>(lse2 + c0 + i);
       const float2 dd = *reinterpret_cast<const float2*>(dlt + c0 + i);
-      const float2 x = ffma2(make_float2(u2f(rs[i]), u2f(rs[i + 1])), c2,
-                             make_float2(-l2.x, -l2.y));
-      float2 pv = make_float2(ex2(x.x), ex2(x.y));
-      if (c0 + i < ilo || c0 + i > ihi) pv.x = 0.f;
-      if (c0 + i + 1 < ilo || c0 + i + 1 > ihi) pv.y = 0.f;
       const float2 g = fsub2(make_float2(u2f(rd[i]), u2f(rd[i + 1])), dd);
-      pk[4 * u + e] = pack_bf16x2(pv.x, pv.y);
-      dw[e] = pack_bf16x2(pv.x * g.x, pv.y * g.y);
+      pk[4 * u + e] = pack_bf16x2(pv[i], pv[i + 1]);
+      dw[e] = pack_bf16x2(pv[i] * g.x, pv[i + 1] * g.y);
       dk[4 * u + e] = dw[e];
     }
     const int chunk = (c0 >> 3) + u;  // 16-byte chunk index within the 128-byte row
@@ -357,6 +367,7 @@ __global__ void __launch_bounds__(512, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(C::B_SP + s), 1);
+      mbar_init(BAR(C::B_SPD + s), 1);
       mbar_init(BAR(C::B_DQF + s), 1);
       mbar_init(BAR(C::B_DQE + s), 4);
     }
@@ -403,12 +414,10 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int buf = it & 1, stage = it % NQS, pb = it % NPB;
+      // S^T complete, and the row statistics (loaded with the slice's Q chunks)
       if (!W.wait_warp(BAR(C::B_SP + buf), (it >> 1) & 1, 60)) { ok = false; break; }
-      if (!W.wait_warp(BAR(C::B_QF + stage), (it / NQS) & 1, 61)) { ok = false; break; }
+      if (!W.wait_warp(BAR(C::B_WF), it & 1, 61)) { ok = false; break; }
       if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 0);
-      // the MMAs that read this P/dS buffer NPB iterations ago must be done
-      if (!W.wait_warp(BAR(C::B_PE + pb), ((it / NPB) & 1) ^ 1, 62)) { ok = false; break; }
-      if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 1);
       tc_fence_after();
       const float* lse2 = reinterpret_cast<const float*>(smem + C::S_STAT + stage * 512);
       const float* dlt = lse2 + 64;
@@ -419,7 +428,15 @@ __global__ void __launch_bounds__(512, 1)
       uint8_t* drow = smem + C::S_DS + pb * C::PTILE + j * 128;
       const uint32_t st_addr = tmem + lane_base + C::T_ST + 64 * buf;
       const uint32_t dpt_addr = tmem + lane_base + C::T_DPT + 64 * buf;
-      bwd_row_half(st_addr, dpt_addr, 32 * par, lse2, dlt, p.c, ilo, ihi, drow, j & 7);
+      float pv[32];
+      bwd_row_p(st_addr, 32 * par, lse2, p.c, ilo, ihi, pv);
+      // dP^T complete, and the MMAs that read this dS^T buffer NPB iterations
+      // ago done
+      if (!W.wait_warp(BAR(C::B_SPD + buf), (it >> 1) & 1, 64)) { ok = false; break; }
+      if (!W.wait_warp(BAR(C::B_PE + pb), ((it / NPB) & 1) ^ 1, 62)) { ok = false; break; }
+      if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 1);
+      tc_fence_after();
+      bwd_row_ds(st_addr, dpt_addr, 32 * par, dlt, pv, drow, j & 7);
       if ((threadIdx.x & 127) == 0) ETA_TRACE_AT(tcta, 0, it, 2);
       tmem_wait_st();
       fence_proxy_async_smem();  // generic-proxy smem writes -> tensor core reads
@@ -521,7 +538,7 @@ __global__ void __launch_bounds__(512, 1)
       // Q / dO chunks 2 half, 2 half + 1 are this CTA's D slice ("own"), the
       // other two are read only by S^T and dP^T
       const int c_own = 2 * half, c_oth = 2 - 2 * half;
-      int it = 0, oth_issued = 0, do_issued = 0;
+      int it = 0, oth_issued = 0, q_issued = 0;
       for (; it < n; ++it) {
         const int h = head_of(it);
         const int ig0 = qtile_of(it) * C::BR;
@@ -533,24 +550,24 @@ __global__ void __launch_bounds__(512, 1)
           tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, BAR(C::B_OF), c * 64, ig0, h, b);
         }
         ++oth_issued;
-        if (!W.wait(BAR(C::B_QE), (it & 1) ^ 1, 84)) break;
+        if (!W.wait(BAR(C::B_WE), (it & 1) ^ 1, 84)) break;
         ETA_TRACE_AT(tcta, 3, it, 1);
-        mbar_expect_tx(BAR(C::B_QF), 2 * C::QCHUNK + 512);
-        for (int c = c_own; c < c_own + 2; ++c)
-          tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, BAR(C::B_QF), c * 64, ig0, h, b);
-        const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
-        bulk_load(sbase + C::S_STAT, p.lse2 + srow, 256, BAR(C::B_QF));
-        bulk_load(sbase + C::S_STAT + 256, p.delta + srow, 256, BAR(C::B_QF));
-        ++do_issued;
-        if (!W.wait(BAR(C::B_WE), (it & 1) ^ 1, 85)) break;
-        ETA_TRACE_AT(tcta, 3, it, 2);
-        mbar_expect_tx(BAR(C::B_WF), 2 * C::QCHUNK);
+        mbar_expect_tx(BAR(C::B_WF), 2 * C::QCHUNK + 512);
         for (int c = c_own; c < c_own + 2; ++c)
           tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, BAR(C::B_WF), c * 64, ig0, h, b);
+        const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
+        bulk_load(sbase + C::S_STAT, p.lse2 + srow, 256, BAR(C::B_WF));
+        bulk_load(sbase + C::S_STAT + 256, p.delta + srow, 256, BAR(C::B_WF));
+        ++q_issued;
+        if (!W.wait(BAR(C::B_QE), (it & 1) ^ 1, 85)) break;
+        ETA_TRACE_AT(tcta, 3, it, 2);
+        mbar_expect_tx(BAR(C::B_QF), 2 * C::QCHUNK);
+        for (int c = c_own; c < c_own + 2; ++c)
+          tma_load_4d(sbase + C::S_DO + c * C::QCHUNK, &tm_do, BAR(C::B_QF), c * 64, ig0, h, b);
       }
       W.drain(BAR(C::B_KV), 0, 81);
-      if (do_issued > 0) W.drain(BAR(C::B_QF), static_cast<uint32_t>(do_issued - 1) & 1u, 82);
-      if (it > 0) W.drain(BAR(C::B_WF), static_cast<uint32_t>(it - 1) & 1u, 86);
+      if (q_issued > 0) W.drain(BAR(C::B_WF), static_cast<uint32_t>(q_issued - 1) & 1u, 82);
+      if (it > 0) W.drain(BAR(C::B_QF), static_cast<uint32_t>(it - 1) & 1u, 86);
       if (oth_issued > 0) W.drain(BAR(C::B_OF), static_cast<uint32_t>(oth_issued - 1) & 1u, 83);
     }
     __syncwarp();
@@ -584,15 +601,17 @@ __global__ void __launch_bounds__(512, 1)
         issue_half(true, it, c_oth, true);
         mma_commit(BAR(C::B_OE));
       };
-      // this slice's chunks: dP^T as soon as dO has arrived, then S^T
+      // this slice's chunks: S^T as soon as Q has arrived (the softmax starts
+      // on P while dP^T runs), then dP^T
       auto issue_own = [&](int it) -> bool {
-        if (!W.wait(BAR(C::B_QF), it & 1, 97)) return false;
-        tc_fence_after();
-        issue_half(true, it, c_own, false);
-        if (!W.wait(BAR(C::B_WF), it & 1, 98)) return false;
+        if (!W.wait(BAR(C::B_WF), it & 1, 97)) return false;
         tc_fence_after();
         issue_half(false, it, c_own, false);
         mma_commit(BAR(C::B_SP + (it & 1)));
+        if (!W.wait(BAR(C::B_QF), it & 1, 98)) return false;
+        tc_fence_after();
+        issue_half(true, it, c_own, false);
+        mma_commit(BAR(C::B_SPD + (it & 1)));
         return true;
       };
       bool ok = W.wait(BAR(C::B_KV), 0, 90) && (n == 0 || W.wait(BAR(C::B_OF), 0, 91));
@@ -624,19 +643,19 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t acc0 = it > 0 ? 1u : 0u;
         // P^T / dS^T of query rows [16 ks, 16 ks + 16) sit at S^T column
         // 32 (ks / 2) + 8 (ks % 2) (+ 16 for dS^T)
-        // dV += P^T dO_i with P^T read from TMEM (K = 64 query rows, 4 steps of 16);
-        // then the slice's dO chunks and the statistics are free
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_ts<false>(tmem + C::T_DV, tst + 32 * (ks >> 1) + 8 * (ks & 1), sdesc_at(ddo, ks * 2048),
-                        id_kv, ks > 0 ? 1u : acc0);
-        mma_commit(BAR(C::B_QE));
-        // dK += dS^T Q_i with dS^T read from TMEM; then the slice's Q chunks are free
+        // dK += dS^T Q_i with dS^T read from TMEM (K = 64 query rows, 4 steps of
+        // 16); then the slice's Q chunks and the statistics are free
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_ts<false>(tmem + C::T_DK, tst + 32 * (ks >> 1) + 16 + 8 * (ks & 1),
                         sdesc_at(dq, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
         mma_commit(BAR(C::B_WE));
+        // dV += P^T dO_i with P^T read from TMEM; then the slice's dO chunks are free
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts<false>(tmem + C::T_DV, tst + 32 * (ks >> 1) + 8 * (ks & 1), sdesc_at(ddo, ks * 2048),
+                        id_kv, ks > 0 ? 1u : acc0);
+        mma_commit(BAR(C::B_QE));
         // dQ_i^T = K^T dS^T (K = 128 key rows, 8 steps of 16) into the consumed dP^T buffer
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
