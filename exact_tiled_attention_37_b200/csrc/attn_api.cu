@@ -637,6 +637,7 @@ attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.wait_limit_ns = g_wait_limit_ns.load();
   p.bmask = block_mask;
   p.nt = (N + 127) / 128;
+  p.debug_flags = g_debug_flags.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // per head dimension: Q/dO stages of the dK/dV kernel, K/V ring slots of
   // the dQ kernel, elementwise warpgroups (measured best on B200)

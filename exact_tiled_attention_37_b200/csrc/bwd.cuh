@@ -105,6 +105,7 @@ struct BwdParams {
   unsigned long long wait_limit_ns;
   const uint8_t* bmask; // block-sparse tile mask [B, Hq, nt, nt] or null (D <= 128 only)
   int nt;               // ceil(N / 128)
+  int debug_flags;      // bit 1: the dK/dV producer drops its second Q load (timeout test)
 };
 
 // ---------------------------------------------------------------- preprocess
@@ -554,7 +555,8 @@ __global__ void __launch_bounds__(512, 1)
         ETA_TRACE_AT(tcta, 3, it, 1);
         mbar_expect_tx(BAR(C::B_WF), 2 * C::QCHUNK + 512);
         for (int c = c_own; c < c_own + 2; ++c)
-          tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, BAR(C::B_WF), c * 64, ig0, h, b);
+          if (!((p.debug_flags & 2) && it == 1))
+            tma_load_4d(sbase + C::S_Q + c * C::QCHUNK, &tm_q, BAR(C::B_WF), c * 64, ig0, h, b);
         const long long srow = static_cast<long long>(b * p.Hq + h) * p.Npad + ig0;
         bulk_load(sbase + C::S_STAT, p.lse2 + srow, 256, BAR(C::B_WF));
         bulk_load(sbase + C::S_STAT + 256, p.delta + srow, 256, BAR(C::B_WF));

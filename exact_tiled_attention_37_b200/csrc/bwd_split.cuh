@@ -736,8 +736,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
                 const uint32_t full = BAR(C::B_QF + stage);
                 mbar_expect_tx(full, C::TILE + 1024);
                 for (int c = 0; c < C::NCHUNK; ++c)
-                  tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full,
-                              c * 64, ig0, h, I.b);
+                  if (!((p.debug_flags & 2) && g == 1))
+                    tma_load_4d(sbase + C::S_Q + stage * C::TILE + c * C::CHUNK, &tm_q, full,
+                                c * 64, ig0, h, I.b);
                 const long long srow = static_cast<long long>(I.b * p.Hq + h) * p.Npad + ig0;
                 bulk_load(sbase + C::S_STAT + stage * 1024, p.lse2 + srow, 512, full);
                 bulk_load(sbase + C::S_STAT + stage * 1024 + 512, p.delta + srow, 512, full);

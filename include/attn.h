@@ -275,6 +275,7 @@ ATTN_API attn_status_t attn_device_status(void* stream, int* where);
  * Test hooks.  attn_debug_set_wait_limit_ns sets the time limit of every
  * in-kernel wait (default 2 s; 0 restores the default).
  * attn_debug_set_flags: bit 0 makes the next forward launches drop one tile
+ * load, bit 1 makes the next backward launches' dK/dV kernel drop one Q tile
  * load, so that their waits run out and report ATTN_ERR_DEVICE_TIMEOUT
  * through attn_device_status (0 = normal operation).
  */

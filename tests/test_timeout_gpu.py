@@ -9,7 +9,8 @@ import pytest
 import torch
 
 import oracle
-from exact_tiled_attention_37_b200 import attn_fwd, device_status, set_debug_flags, set_wait_limit_ns
+from exact_tiled_attention_37_b200 import (attn_bwd, attn_fwd, device_status, set_debug_flags,
+                                           set_wait_limit_ns)
 from exact_tiled_attention_37_b200.inputs import make_random
 
 from ._util import TOL_REL, rel_err, to_np
@@ -36,3 +37,28 @@ def test_dropped_load_times_out_and_recovers(D):
     assert device_status()[0] == 0
     o_ref, _ = oracle.attention_fwd(to_np(q), to_np(k), to_np(v), False, 1 / math.sqrt(D))
     assert rel_err(to_np(o), o_ref) <= TOL_REL
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_dropped_bwd_load_times_out_and_recovers(D):
+    """The dK/dV kernel's producer drops its second Q tile load: the MMA
+    warp's wait for it runs out, every role leaves its loop, the kernel
+    drains what it started and returns; the next backward is correct."""
+    q, k, v, do = (t.to("cuda") for t in make_random(1, 2, 2, 384, D, "bf16", seed=6))
+    o, lse = attn_fwd(q, k, v, causal=False)
+    assert device_status()[0] == 0
+    set_wait_limit_ns(50_000_000)  # 50 ms
+    set_debug_flags(2)
+    try:
+        attn_bwd(q, k, v, o, lse, do, causal=False)
+        code, where = device_status()
+    finally:
+        set_debug_flags(0)
+        set_wait_limit_ns(0)
+    assert code == 6, (code, where)
+    assert where != 0
+    dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=False)
+    assert device_status()[0] == 0
+    ref = oracle.attention_bwd(*(to_np(t) for t in (q, k, v, do)), False, 1 / math.sqrt(D))
+    for got, r in zip((dq, dk, dv), ref):
+        assert rel_err(to_np(got), r) <= TOL_REL
