@@ -1,5 +1,6 @@
 """Runs one forward (+ backward) of a named workload through the C ABI, for
-profilers: ``python -m exact_tiled_attention_37_b200.profile_case --workload 2``.
+profilers: ``python -m exact_tiled_attention_37_b200.profile_case --workload 2``
+(``--batch B`` keeps only the first B sequences, for smaller captures).
 ``--decode`` instead runs a paged decode: 8 sequences of 32768 cached keys,
 Hq=32, Hkv=8, D=128, one new token, the 2048 pages in a seeded random order.
 
@@ -40,19 +41,25 @@ def main(argv=None) -> int:
     ap.add_argument("--repeat", type=int, default=1)
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--decode", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run only the first BATCH sequences of the workload (smaller captures)")
     args = ap.parse_args(argv)
     if args.decode:
         return decode_case(args.repeat)
     w = workload(args.workload)
     causal = w.causal[-1]
-    q, k, v, *rest = (t.to("cuda") for t in make_inputs(w, with_do=w.backward))
+    ins = make_inputs(w, with_do=w.backward)
+    if args.batch > 0:
+        ins = tuple(t[: args.batch] for t in ins)
+    q, k, v, *rest = (t.to("cuda") for t in ins)
     for _ in range(args.repeat):
         o, lse = attn_fwd(q, k, v, causal=causal)
         if w.backward and not args.fwd_only:
             attn_bwd(q, k, v, o, lse, rest[0], causal=causal)
     torch.cuda.synchronize()
     code, where = device_status()
-    print(f"{w.name}: device status {code} (wait site {where})")
+    name = w.name + (f" (first {args.batch} sequences)" if args.batch > 0 else "")
+    print(f"{name}: device status {code} (wait site {where})")
     return 0 if code == 0 else 1
 
 
