@@ -118,6 +118,33 @@ attn_status_t make_map(CUtensorMap* m, const attn_tensor_t& t, int B, int H, int
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// 5-D TMA map over [B, H, N, D] seen as (128-byte chunk of a row, row, chunk,
+// head, batch): one box of box_rows rows x box_chunks chunks is a whole tile
+// in the chunked shared-memory layout [chunk][row][128 bytes].
+attn_status_t make_tile_map(CUtensorMap* m, const attn_tensor_t& t, int B, int H, int N, int D,
+                            int es, int box_rows, int box_chunks) {
+  auto enc = encode_fn();
+  if (!enc) return ATTN_ERR_CUDA;
+  int64_t sn = N > 1 ? t.sn : D;
+  int64_t sh = H > 1 ? t.sh : sn * N;
+  int64_t sb = B > 1 ? t.sb : sh * H;
+  const int epc = 128 / es;  // elements per chunk
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(epc), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(D / epc), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(sn * es), 128u,
+                           static_cast<cuuint64_t>(sh * es), static_cast<cuuint64_t>(sb * es)};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(epc), static_cast<cuuint32_t>(box_rows),
+                       static_cast<cuuint32_t>(box_chunks), 1u, 1u};
+  cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUtensorMapDataType dt = es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = enc(m, dt, 5, t.ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 template <typename Kernel>
 attn_status_t set_smem(Kernel k, int bytes) {
   // cudaFuncSetAttribute is cheap and idempotent; the result is per device.
@@ -146,9 +173,10 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
   using C = eta::SingleCfg<T, D, BC, NS>;
   CUtensorMap tq, tk, tv;
   attn_status_t s;
-  if ((s = make_map(&tq, q, B, Hq, N, D, sizeof(T), 128)) != ATTN_OK) return s;
-  if ((s = make_map(&tk, k, B, Hkv, N, D, sizeof(T), BC)) != ATTN_OK) return s;
-  if ((s = make_map(&tv, v, B, Hkv, N, D, sizeof(T), BC)) != ATTN_OK) return s;
+  // whole-tile boxes: one TMA instruction per Q tile and per K or V tile
+  if ((s = make_tile_map(&tq, q, B, Hq, N, D, sizeof(T), 128, C::NCHUNK)) != ATTN_OK) return s;
+  if ((s = make_tile_map(&tk, k, B, Hkv, N, D, sizeof(T), BC, C::NCHUNK)) != ATTN_OK) return s;
+  if ((s = make_tile_map(&tv, v, B, Hkv, N, D, sizeof(T), BC, C::NCHUNK)) != ATTN_OK) return s;
   auto kern = p.bmask ? eta::fwd_single_kernel<T, D, BC, NS, true>
                       : eta::fwd_single_kernel<T, D, BC, NS, false>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;

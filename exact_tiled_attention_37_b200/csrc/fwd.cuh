@@ -416,8 +416,7 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
     fence_proxy_async_smem();
     // the Q tile's load starts before TMEM allocation and the block-wide sync
     mbar_expect_tx(BAR(C::BAR_Q), C::QTILE);
-    for (int c = 0; c < C::NCHUNK; ++c)
-      tma_load_4d(sbase + C::SMEM_Q + c * C::QCHUNK, &tm_q, BAR(C::BAR_Q), c * C::EPC, q0, h, b);
+    tma_load_5d(sbase + C::SMEM_Q, &tm_q, BAR(C::BAR_Q), 0, q0, 0, h, b);
   }
   if (warp == 5) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::TMEM_COLS);
@@ -493,9 +492,8 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
           if (!W.wait(BAR(C::BAR_KVE + slot), ph ^ 1u, 30)) break;
           if ((p.debug_flags & 1) && kv == 1 && u == 0) continue;
           mbar_expect_tx(BAR(C::BAR_KVF + slot), C::KTILE);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sbase + C::SMEM_KV + slot * C::KTILE + c * C::KCHUNK, kv ? &tm_v : &tm_k,
-                        BAR(C::BAR_KVF + slot), c * C::EPC, BC * j, hk, b);
+          tma_load_5d(sbase + C::SMEM_KV + slot * C::KTILE, kv ? &tm_v : &tm_k,
+                      BAR(C::BAR_KVF + slot), 0, BC * j, 0, hk, b);
         }
       }
       const int issued = it;

@@ -143,6 +143,20 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// 5-D tiled load (no multicast): with a map whose dimensions are (128-byte
+// chunk of a row, row, chunk, head, batch) one instruction moves a whole tile
+// in the chunked layout [chunk][row][128 bytes].  Fewer, larger boxes load
+// faster: on B200, 32 KB tiles from L2 arrive at about 69 B per cycle per SM
+// as one box each, 43 B per cycle as four 8 KB boxes.
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
 // 1-D bulk copy global -> shared (no multicast); both addresses 16-byte
 // aligned, size a multiple of 16 bytes.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
