@@ -146,8 +146,8 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, 
 // 5-D tiled load (no multicast): with a map whose dimensions are (128-byte
 // chunk of a row, row, chunk, head, batch) one instruction moves a whole tile
 // in the chunked layout [chunk][row][128 bytes].  Fewer, larger boxes load
-// faster: on B200, 32 KB tiles from L2 arrive at about 69 B per cycle per SM
-// as one box each, 43 B per cycle as four 8 KB boxes.
+// faster: on B200 one CTA's 32 KB tiles from L2 arrive at about 69 B per
+// cycle as one box each, 43 B per cycle as four 8 KB boxes.
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
                                             int c0, int c1, int c2, int c3, int c4) {
   asm volatile(
