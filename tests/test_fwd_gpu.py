@@ -75,6 +75,23 @@ def test_strided_views(D):
         assert abs_err(to_np(lse), lse_ref) <= TOL_LSE
 
 
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_padded_input_rows(D):
+    # inputs are the first D columns of wider rows (row stride 2 D): tile loads
+    # must read D columns per row and no further
+    B, H, N = 1, 2, 200
+    g = torch.Generator().manual_seed(11 + D)
+    wide = [torch.randn(B, H, N, 2 * D, generator=g).to(torch.bfloat16).to(DEV) for _ in range(3)]
+    q, k, v = (t[..., :D] for t in wide)
+    assert q.stride(2) == 2 * D
+    for causal in (False, True):
+        o, lse = attn_fwd(q, k, v, causal=causal)
+        o_ref, lse_ref = oracle.attention_fwd(*(to_np(t) for t in (q, k, v)), causal,
+                                              1 / math.sqrt(D))
+        assert rel_err(to_np(o), o_ref) <= TOL_REL
+        assert abs_err(to_np(lse), lse_ref) <= TOL_LSE
+
+
 def test_output_into_strided_buffer():
     B, H, N, D = 1, 2, 256, 128
     q, k, v = (t.to(DEV) for t in make_random(B, H, H, N, D, "bf16", seed=3, with_do=False))
