@@ -7,6 +7,14 @@ the method.  Inputs are seeded synthetic N(0,1) tensors resident in HBM.
 Throughput counts 4*B*H*N^2*D FLOPs for the forward (halved for causal) and
 2.5x that for the backward.
 
+After the timed steps the same process times, with the same clock sampler,
+every other workload of the method (both masks of the B=4 H=16 N=2048
+forward, the 32K-token grouped-query forward, the D=256 forward and
+backward) and the mask and precision variants (sliding windows, block-sparse
+tiles, e4m3 forward), each as the median of CUDA-event timings with L2
+flushed before every call; these go under "configs" and do not enter the
+headline value.
+
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 For N > 1 launch with torchrun: every rank runs an independent replica of the
 workload (the path needs no exchange between GPUs; weak scaling).
@@ -30,13 +38,16 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD_INDEX = 2  # MHA fwd+bwd B=2 H=16 N=4096 D=128 causal
+METRIC = "attention fwd+bwd TFLOPS (bf16, 1xB200) and % of dense tensor-core peak"
 
 # The dominant kernel of the step: the backward's dK/dV kernel.
 DOMINANT_KERNEL = "bwd_kv_kernel<128,2,2>"
-# DRAM traffic of one launch of it from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum), with the hash of the kernel sources it was taken on;
-# it is reported as null once the sources change (profiles/ holds the capture).
+# DRAM traffic of one launch of the dK/dV and dQ kernels from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the kernel
+# sources it was taken on; reported as null once the sources change (profiles/
+# holds the capture).
 DOMINANT_TRAFFIC = {"bytes": 227364864, "src_sha": "4b5594ff11e21fc4"}
+DQ_TRAFFIC = {"bytes": 229018368, "src_sha": "4b5594ff11e21fc4"}
 
 
 def parse_args():
@@ -46,6 +57,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration timings after the timed steps")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="rough budget of the oracle CPU-baseline sample")
     return ap.parse_args()
@@ -79,23 +92,38 @@ def load_peaks():
                 "source": "fallback"}
 
 
+def choose_peak(peaks, clocks, region_ms):
+    """The burst figure describes a kernel timed alone at full clock, the
+    sustained one a kernel inside seconds of back-to-back work under the power
+    cap: burst when the sampled SM clock stayed within 5 % of its maximum and
+    the timed region is short (< 1 s per step), else sustained."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    burst = mhz is not None and mx and mhz >= 0.95 * mx and region_ms < 1000.0
+    kind = "burst" if burst else "sustained"
+    return (peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"]), kind
+
+
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+    """Samples SM clocks and throttle reasons with nvidia-smi (every 50 ms) while
+    it is open; mark() labels time windows so that each timed region's samples
+    can be summarised separately."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.samples = []   # (time, sm_mhz, max_mhz, power_w, reasons)
+        self.windows = {}
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -105,7 +133,19 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            try:
+                pw = float(parts[2])
+            except ValueError:
+                pw = None
+            reasons = {n for n, v in zip(self.NAMES, parts[3:7]) if v.lower().startswith("active")}
+            self.samples.append((time.monotonic(), sm, mx, pw, reasons))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -116,23 +156,19 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=2)
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "samples": len(sm), "reasons": sorted(reasons)}
+    def mark(self, name, t0, t1):
+        self.windows[name] = (t0, t1)
+
+    def summary(self, name=None):
+        t0, t1 = self.windows.get(name, (float("-inf"), float("inf"))) if name else \
+            (float("-inf"), float("inf"))
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        sm = [s[1] for s in sel]
+        reasons = sorted(set().union(*[s[4] for s in sel])) if sel else []
+        pw = [s[3] for s in sel if s[3] is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": sel[-1][2] if sel else None, "samples": len(sm),
+                "power_w_median": statistics.median(pw) if pw else None, "reasons": reasons}
 
 
 def max_over_ranks(values, device):
@@ -152,14 +188,39 @@ def whole_job_tflops(flops_per_step_per_rank: float, world: int, ms_per_step: fl
     return world * flops_per_step_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
+def visible_pairs(N: int, wl: int = -1, wr: int = -1, tile_mask=None, tile: int = 128) -> int:
+    """Number of (query, key) pairs one head computes under a window (wl, wr)
+    (-1 = unbounded side) and an optional [T, T] tile mask: the FLOP count of
+    masked variants is 4 * D per visible pair (backward 2.5x)."""
+    import numpy as np
+    i = np.arange(N)
+    lo = np.zeros(N, dtype=np.int64) if wl < 0 else np.maximum(0, i - wl)
+    hi = np.full(N, N - 1, dtype=np.int64) if wr < 0 else np.minimum(N - 1, i + wr)
+    if tile_mask is None:
+        return int(np.sum(hi - lo + 1))
+    total = 0
+    T = tile_mask.shape[0]
+    for qt in range(T):
+        rows = i[qt * tile:(qt + 1) * tile]
+        for kt in range(T):
+            if not tile_mask[qt, kt]:
+                continue
+            k0, k1 = kt * tile, min(N, (kt + 1) * tile) - 1
+            a = np.maximum(lo[rows], k0)
+            b = np.minimum(hi[rows], k1)
+            total += int(np.sum(np.maximum(0, b - a + 1)))
+    return total
+
+
 # ---------------------------------------------------------------- CPU baseline (oracle)
 
 
-def cpu_baseline(w, budget_s: float):
+def cpu_baseline(w, budget_s: float, pairs: int | None = None):
     """The fp64 oracle, as it stands, on a bounded sample of the workload: the
     forward and backward of one (batch, head) pair at a time, repeated until
-    the time budget is spent.  Returns TFLOPS on the counted FLOPs."""
-    import numpy as np
+    the time budget is spent (or `pairs` pairs are done).  Returns TFLOPS on
+    the counted FLOPs of the pairs it ran."""
+    import numpy as np  # noqa: F401
     from threadpoolctl import threadpool_limits
 
     import oracle
@@ -177,13 +238,143 @@ def cpu_baseline(w, budget_s: float):
             oracle.attention_fwd(q[sl], k[sl], v[sl], causal, w.scale)
             oracle.attention_bwd(q[sl], k[sl], v[sl], do[sl], causal, w.scale)
             done += 1
-            if time.perf_counter() - t0 > budget_s:
+            if (pairs is not None and done >= pairs) or \
+                    (pairs is None and time.perf_counter() - t0 > budget_s):
                 break
     dt = time.perf_counter() - t0
     return {"value": done * per_head / dt / 1e12, "unit": "TFLOPS", "cores": cores,
-            "kind": "oracle",
+            "kind": "oracle", "seconds": dt, "pairs": done,
             "sample": f"fwd+bwd of {done} (batch, head) pair(s) of {w.name} (of {w.B * w.Hq}), "
-                      f"fp64 NumPy/OpenBLAS, {dt:.1f} s"}
+                      f"fp64 NumPy/OpenBLAS, {dt:.1f} s; TFLOPS = counted FLOPs of those pairs / time"}
+
+
+# ---------------------------------------------------------------- per-configuration timings
+
+
+def time_calls(fn, flush, stream, n, warm=2):
+    """Median device time (ms) of fn() over n calls, L2 flushed before each;
+    events on the launching stream."""
+    import torch
+    for _ in range(warm):
+        fn()
+    es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for a, b in es:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    stream.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in es)
+
+
+def run_configs(dev, flush, stream, peak_burst, clocks):
+    """Forward/backward timings of the other workloads and of the mask and
+    precision variants.  Returns a list of result dicts."""
+    import numpy as np
+    import torch
+
+    from exact_tiled_attention_37_b200 import (attn_bwd, attn_fwd, attn_fwd_fp8,
+                                               bwd_workspace_bytes, device_status)
+    from exact_tiled_attention_37_b200.inputs import make_inputs, make_random, workload
+
+    out = []
+
+    def entry(name, kind, ms, flops, extra=None):
+        tf = flops / (ms * 1e-3) / 1e12
+        e = {"config": name, "pass": kind, "ms": round(ms, 4), "tflops": round(tf, 1),
+             "frac_of_burst_peak": round(tf / peak_burst, 4)}
+        if extra:
+            e.update(extra)
+        out.append(e)
+
+    def reps(ms_guess):
+        return 30 if ms_guess < 1 else (15 if ms_guess < 10 else 7)
+
+    # the workloads of the method (bf16; the fp32 single-head one is latency-bound)
+    for idx, passes in ((1, ("fwd",)), (2, ("fwd", "bwd")), (3, ("fwd",)), (4, ("fwd", "bwd"))):
+        w = workload(idx)
+        ins = [t.to(dev) for t in make_inputs(w, with_do="bwd" in passes)]
+        q, k, v = ins[:3]
+        for causal in w.causal:
+            o = torch.empty_like(q)
+            lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
+            t0 = time.monotonic()
+            ms = time_calls(lambda: attn_fwd(q, k, v, causal=causal, out=o, lse=lse), flush, stream,
+                            reps(w.fwd_flops(causal) / 1e12))
+            entry(f"{w.name}{', causal' if causal else ''}", "fwd", ms, w.fwd_flops(causal))
+            if "bwd" in passes:
+                do = ins[3]
+                dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+                ws = torch.empty(bwd_workspace_bytes(w.B, w.Hq, w.N, w.D), device=dev,
+                                 dtype=torch.uint8)
+                ms = time_calls(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dq, dk=dk,
+                                                 dv=dv, workspace=ws), flush, stream,
+                                reps(2.5 * w.fwd_flops(causal) / 1e12))
+                entry(f"{w.name}{', causal' if causal else ''}", "bwd", ms, w.bwd_flops(causal))
+                del dq, dk, dv, ws
+            clocks.mark(f"cfg{idx}{causal}", t0, time.monotonic())
+        del ins, q, k, v
+        torch.cuda.empty_cache()
+
+    # sliding windows on the B=2 H=16 N=4096 D=128 shapes (FLOPs over visible pairs)
+    w = workload(2)
+    q, k, v, do = (t.to(dev) for t in make_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
+    ws = torch.empty(bwd_workspace_bytes(w.B, w.Hq, w.N, w.D), device=dev, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for win in ((1023, 0), (111, 0)):
+        f = 4.0 * w.D * w.B * w.Hq * visible_pairs(w.N, *win)
+        ms = time_calls(lambda: attn_fwd(q, k, v, window=win, out=o, lse=lse), flush, stream, 30)
+        entry(f"{w.name}, local window {win}", "fwd", ms, f, {"flops": "visible pairs"})
+        ms = time_calls(lambda: attn_bwd(q, k, v, o, lse, do, window=win, dq=dq, dk=dk, dv=dv,
+                                         workspace=ws), flush, stream, 30)
+        entry(f"{w.name}, local window {win}", "bwd", ms, 2.5 * f, {"flops": "visible pairs"})
+
+    # e4m3 forward on the same inputs (per-tensor scales = max|x| / 448)
+    f8 = []
+    for t in (q, k, v):
+        s = float(t.float().abs().max()) / 448.0
+        f8.append(((t.float() / s).to(torch.float8_e4m3fn), s))
+    ms = time_calls(lambda: attn_fwd_fp8(f8[0][0], f8[1][0], f8[2][0], f8[0][1], f8[1][1],
+                                         f8[2][1], causal=True, out=o, lse=lse),
+                    flush, stream, 30)
+    entry(f"{w.name}, e4m3 inputs", "fwd", ms, w.fwd_flops(True), {"dtype": "e4m3"})
+    del q, k, v, do, o, dq, dk, dv, ws, f8
+    torch.cuda.empty_cache()
+
+    # block-sparse tiles: B=2 H=16 N=8192 D=128, a band of +-2 tiles plus every 8th key tile
+    B, H, N, D = 2, 16, 8192, 128
+    T = N // 128
+    qt, kt = np.meshgrid(np.arange(T), np.arange(T), indexing="ij")
+    tm = (np.abs(qt - kt) <= 2) | (kt % 8 == 0)
+    q, k, v, do = (t.to(dev) for t in make_random(B, H, H, N, D, "bf16", seed=77))
+    bm = torch.from_numpy(np.broadcast_to(tm, (B, H, T, T)).astype(np.uint8).copy()).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    ws = torch.empty(bwd_workspace_bytes(B, H, N, D), device=dev, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for causal in (False, True):
+        pairs = visible_pairs(N, -1, 0 if causal else -1, tm)
+        f = 4.0 * D * B * H * pairs
+        frac_vis = pairs / (N * N)
+        ms = time_calls(lambda: attn_fwd(q, k, v, causal=causal, block_mask=bm, out=o, lse=lse),
+                        flush, stream, 30)
+        entry(f"block-sparse B=2 H=16 N=8192 D=128, band +-2 tiles + every 8th key tile"
+              f"{', causal' if causal else ''}", "fwd", ms, f,
+              {"flops": "visible pairs", "visible": round(frac_vis, 4)})
+        ms = time_calls(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, block_mask=bm, dq=dq,
+                                         dk=dk, dv=dv, workspace=ws), flush, stream, 30)
+        entry(f"block-sparse B=2 H=16 N=8192 D=128, band +-2 tiles + every 8th key tile"
+              f"{', causal' if causal else ''}", "bwd", ms, 2.5 * f,
+              {"flops": "visible pairs", "visible": round(frac_vis, 4)})
+    del q, k, v, do, o, dq, dk, dv, ws, bm
+    torch.cuda.empty_cache()
+    code, where = device_status(dev)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at wait site {where} during the config timings")
+    return out
 
 
 # ---------------------------------------------------------------- native arm
@@ -226,9 +417,9 @@ def run_native(args):
         torch.cuda.synchronize(dev)
 
     K, W = args.steps, args.warmup
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    # per step: step start/stop, dK/dV kernel start/stop, dQ kernel start/stop
+    ev = [tuple(mk() for _ in range(6)) for _ in range(K)]
     for e in ev:  # create the driver events before the timed region
         for x in e:
             x.record(stream)
@@ -240,39 +431,44 @@ def run_native(args):
     if code != 0:
         raise RuntimeError(f"device status {code} at wait site {where} during warm-up")
 
+    peaks = load_peaks()
     with ClockSampler(local) as clocks:
+        time.sleep(0.2)
         barrier()
+        t_main0 = time.monotonic()
         for i in range(K):
             flush.zero_()
-            s0, s1, m0, m1 = ev[i]
+            s0, s1, m0, m1, d0, d1 = ev[i]
             s0.record(stream)
             L.attn_debug_set_bwd_events(m0.cuda_event, m1.cuda_event)
+            L.attn_debug_set_bwd_q_events(d0.cuda_event, d1.cuda_event)
             step()
             s1.record(stream)
         barrier()
-        time.sleep(0.25)
-    code, where = device_status(dev)
-    if code != 0:
-        raise RuntimeError(f"device status {code} at wait site {where} during timing")
-    step_ms = [a.elapsed_time(b) for a, b, _, _ in ev]
-    main_ms = [c.elapsed_time(d) for _, _, c, d in ev]
+        t_main1 = time.monotonic()
+        clocks.mark("main", t_main0, t_main1)
+        code, where = device_status(dev)
+        if code != 0:
+            raise RuntimeError(f"device status {code} at wait site {where} during timing")
+
+        # forward and backward separately (same region shape, fewer steps)
+        t0 = time.monotonic()
+        fwd_ms = time_calls(lambda: attn_fwd(q, k, v, causal=causal, out=o, lse=lse), flush,
+                            stream, min(K, 50), warm=0)
+        bwd_ms = time_calls(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dq, dk=dk,
+                                             dv=dv, workspace=ws), flush, stream, min(K, 50),
+                            warm=0)
+        clocks.mark("split", t0, time.monotonic())
+        configs = None
+        if rank == 0 and not args.no_configs:
+            t0 = time.monotonic()
+            configs = run_configs(dev, flush, stream, peaks["bf16_tflops"], clocks)
+            clocks.mark("configs", t0, time.monotonic())
+        time.sleep(0.1)
+    step_ms = [a.elapsed_time(b) for a, b, *_ in ev]
+    kv_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    dq_ms = [e[4].elapsed_time(e[5]) for e in ev]
     total_ms = sum(step_ms)
-
-    # forward and backward separately (same region shape, fewer steps)
-    def timed(fn, n):
-        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n)]
-        for a, b in es:
-            flush.zero_()
-            a.record(stream)
-            fn()
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        return statistics.median(a.elapsed_time(b) for a, b in es)
-
-    fwd_ms = timed(lambda: attn_fwd(q, k, v, causal=causal, out=o, lse=lse), min(K, 50))
-    bwd_ms = timed(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dq, dk=dk, dv=dv,
-                                    workspace=ws), min(K, 50))
 
     # end to end through the public API with host buffers: every step uploads
     # its inputs (pinned Q, K, V, dO), runs forward + backward and downloads its
@@ -338,19 +534,31 @@ def run_native(args):
     value = whole_job_tflops(flops_step, world, ms_per_step)
     e2e_value = whole_job_tflops(flops_step, world, e2e_ms)
 
-    peaks = load_peaks()
-    dom_ms = statistics.mean(main_ms)
-    # algorithmic FLOPs of one dK/dV-kernel launch: four products (S^T, dP^T,
-    # dV, dK) over the visible tile pairs, each as costly as one of the
-    # forward's two products
+    clk_main = clocks.summary("main")
+    clk_all = clocks.summary()
+    # the main region can be shorter than the sampling interval allows many
+    # samples for; the whole timing window (main + fwd/bwd + configs, the same
+    # kernels back to back) gives the clock a sample count worth reading
+    clk_ref = clk_main if clk_main["samples"] >= 5 else clk_all
+    peak, peak_kind = choose_peak(peaks, clk_ref, ms_per_step)
+
+    # dominant kernel: the dK/dV kernel does four of the method's products
+    # (S^T, dP^T, dV, dK) over the visible tile pairs, each as costly as one of
+    # the forward's two products
+    dom_ms = statistics.mean(kv_ms)
     dom_flops = 4 * w.fwd_flops(causal) / 2
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    traffic = DOMINANT_TRAFFIC["bytes"] if DOMINANT_TRAFFIC["src_sha"] == kernel_source_sha() else None
-    peak = peaks["bf16_tflops_sustained"]
-    clk = clocks.summary()
+    sha = kernel_source_sha()
+    traffic = DOMINANT_TRAFFIC["bytes"] if DOMINANT_TRAFFIC["src_sha"] == sha else None
+    # dQ kernel: three products (S, dP, dQ) of which the method counts one (dQ)
+    dq_mean = statistics.mean(dq_ms)
+    dq_method = (w.fwd_flops(causal) / 2) / (dq_mean * 1e-3) / 1e12
+    dq_exec = 3 * (w.fwd_flops(causal) / 2) / (dq_mean * 1e-3) / 1e12
+    dq_alg_bytes = 4 * w.B * w.Hq * w.N * w.D * 2 + w.B * w.Hq * w.N * w.D * 2  # Q,K,V,dO in; dQ out
+    dq_traffic = DQ_TRAFFIC["bytes"] if DQ_TRAFFIC["src_sha"] == sha else None
 
     result = {
-        "metric": "attention fwd+bwd TFLOPS (bf16, 1xB200) and % of dense tensor-core peak",
+        "metric": METRIC,
         "value": round(value, 2),
         "unit": "TFLOPS",
         "n_gpus": world,
@@ -372,14 +580,36 @@ def run_native(args):
         "roofline": {"kernel": DOMINANT_KERNEL, "bound": "tensor",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peaks['source']} bf16 sustained",
-                     "launch_ms": round(dom_ms, 4)},
+                     "peak_source": f"{peaks['source']} bf16 {peak_kind}",
+                     "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "launch_ms": round(dom_ms, 4),
+                     "flops_per_launch": dom_flops,
+                     "algorithmic_bytes": 4 * w.B * w.Hq * w.N * w.D * 2 + 2 * w.B * w.Hkv * w.N * w.D * 2},
+        "kernels": {
+            "bwd_q_kernel<128,5,2>": {
+                "launch_ms": round(dq_mean, 4),
+                "method_tflops": round(dq_method, 1),
+                "method_frac_of_burst_peak": round(dq_method / peaks["bf16_tflops"], 4),
+                "executed_tflops": round(dq_exec, 1),
+                "note": "three products (S, dP recomputed; dQ) per tile pair, one counted",
+                "traffic": dq_traffic, "algorithmic_bytes": dq_alg_bytes,
+                "traffic_ratio": round(dq_traffic / dq_alg_bytes, 3) if dq_traffic else None},
+        },
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
-                "pipeline": "upload / compute / download on three streams, double-buffered"},
-        "clocks": clk,
-        "gpu_launches": 4 * K,
+                "kind": "pipelined throughput through the public API: per step H2D of Q, K, V, dO "
+                        "and D2H of the gradients dQ, dK, dV (O and lse stay on the device); "
+                        "upload / compute / download on three streams, double-buffered"},
+        "clocks": {**clk_ref, "window": "main timed region" if clk_ref is clk_main else
+                   "main + fwd/bwd + config timings (main region alone had "
+                   f"{clk_main['samples']} samples)",
+                   "main_region": clk_main,
+                   "ms_x_mhz": round(ms_per_step * clk_ref["sm_mhz"], 1) if clk_ref["sm_mhz"] else None},
+        "gpu_launches": 4 * K,  # forward; backward preprocess, dK/dV, dQ
     }
+    if configs is not None:
+        result["configs"] = configs
+        result["configs_clocks"] = clocks.summary("configs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if world > 1:
@@ -394,37 +624,50 @@ def run_native(args):
 
 def run_reference(args):
     """The oracle (plain fp64 CPU implementation) as the reference arm, on the
-    same workload and metric, each step a bounded sample of the workload."""
+    same workload and metric.  Each step runs a fixed sample of the workload --
+    the forward and backward of one of its (batch, head) pairs -- and is timed
+    as it runs, so steps x ms_per_step is the time actually spent; the value is
+    the sample's counted FLOPs over its time (a whole workload step would take
+    about B x H times as long)."""
     rank, world, _ = dist_info()
     if rank != 0:
         return
     from exact_tiled_attention_37_b200.inputs import workload
     w = workload(WORKLOAD_INDEX)
-    budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(w, budget)
-    vals = [cpu_baseline(w, budget) for _ in range(args.steps)]
-    v = statistics.median(x["value"] for x in vals)
+        cpu_baseline(w, 0.0, pairs=1)
+    t0 = time.perf_counter()
+    vals = [cpu_baseline(w, 0.0, pairs=1) for _ in range(args.steps)]
+    timed_s = time.perf_counter() - t0
+    secs = [x["seconds"] for x in vals]
     causal = w.causal[0]
-    flops_step = w.fwd_flops(causal) + w.bwd_flops(causal)
+    sample_flops = (w.fwd_flops(causal) + w.bwd_flops(causal)) / (w.B * w.Hq)
+    ms_step = statistics.median(secs) * 1e3
+    v = sample_flops / (ms_step * 1e-3) / 1e12
     result = {
         "impl": "reference",
-        "metric": "attention fwd+bwd TFLOPS (bf16, 1xB200) and % of dense tensor-core peak",
+        "metric": METRIC,
         "value": v,
         "unit": "TFLOPS",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": flops_step / (v * 1e12) * 1e3,
+        "ms_per_step": ms_step,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
-                   "causal": causal, "passes": "fwd+bwd"},
+                   "causal": causal, "passes": "fwd+bwd",
+                   "sample": f"each step: fwd+bwd of 1 of the {w.B * w.Hq} (batch, head) pairs; "
+                             "value = that sample's counted FLOPs / its time, extrapolated to "
+                             "the whole workload only through the TFLOPS unit"},
+        "timed_seconds": round(timed_s, 2),
         "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": vals[0]["cores"],
-                         "kind": "oracle", "sample": vals[0]["sample"]},
+                         "kind": "oracle",
+                         "sample": f"{args.steps} steps of 1 (batch, head) pair each of {w.name}, "
+                                   f"fp64 NumPy/OpenBLAS, {timed_s:.1f} s timed"},
         "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(result), flush=True)

@@ -88,6 +88,8 @@ def lib(path: str | None = None) -> ctypes.CDLL:
     L.attn_debug_exp2.argtypes = [vp, vp, i, i, vp]
     L.attn_debug_set_bwd_events.restype = None
     L.attn_debug_set_bwd_events.argtypes = [vp, vp]
+    L.attn_debug_set_bwd_q_events.restype = None
+    L.attn_debug_set_bwd_q_events.argtypes = [vp, vp]
     if path is None:
         _LIB = L
     return L

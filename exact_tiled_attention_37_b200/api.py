@@ -44,6 +44,16 @@ def _check(code: int, what: str):
         raise AttnError(code, what)
 
 
+def _check_device(device: torch.device, what: str):
+    """Waits for the current stream of `device` and raises AttnError when a
+    kernel's bounded wait gave up since the device status was last read.  The
+    status word is per device and shared by all streams (see attn.h), so a
+    failure of work on another stream of the same device is reported here too."""
+    code, where = device_status(device)
+    if code != 0:
+        raise AttnError(code, f"{what} (device wait site {where})")
+
+
 def _window(causal: bool, window) -> tuple[int, int]:
     """(window_left, window_right) of the C ABI: -1 = unbounded; causal caps the right side at 0."""
     wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
@@ -67,13 +77,17 @@ def _block_mask(block_mask, B, Hq, N, device) -> ctypes.c_void_p:
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              scale: float | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, window=None, block_mask=None):
+             lse: torch.Tensor | None = None, window=None, block_mask=None,
+             check: bool = False):
     """O, lse = attention(q, k, v): q [B,Hq,N,D], k/v [B,Hkv,N,D] on one CUDA device.
 
     window=(wl, wr): query i sees keys i - wl .. i + wr (-1 = unbounded side).
     block_mask: [B,Hq,T,T] uint8 (T = ceil(N/128)); 128x128 tile pairs whose
     entry is 0 are skipped (rows that see no key get O = 0, lse = -inf).
     Returns O (dtype of q) and lse [B,Hq,N] fp32 (natural log).
+    check=True waits for the call to finish and raises AttnError if a kernel's
+    bounded wait timed out (otherwise the outputs of such a call are undefined
+    and only device_status() reveals it).
     """
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
@@ -96,6 +110,8 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
                              ctypes.c_void_p(lse.data_ptr()), B, Hq, Hkv, N, D, _dtype_code(q),
                              wl, wr, bm, float(scale), _stream(q.device))
     _check(code, "attn_fwd")
+    if check:
+        _check_device(q.device, "attn_fwd")
     return out, lse
 
 
@@ -105,9 +121,9 @@ def bwd_workspace_bytes(B: int, Hq: int, N: int, D: int) -> int:
 
 def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, window=None,
-             block_mask=None):
+             block_mask=None, check: bool = False):
     """dQ, dK, dV of attention from the forward's O and lse and the gradient dO
-    (window and block_mask as in attn_fwd)."""
+    (window, block_mask and check as in attn_fwd)."""
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
     if scale is None:
@@ -136,6 +152,8 @@ def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
                              ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                              _stream(q.device))
     _check(code, "attn_bwd")
+    if check:
+        _check_device(q.device, "attn_bwd")
     return dq, dk, dv
 
 
@@ -171,7 +189,8 @@ def decode_workspace_bytes(B: int, Hq: int, Sq: int, D: int, max_pages: int) -> 
 
 
 def attn_decode(q, k_pool, v_pool, block_table, seqlens, causal: bool = False,
-                scale: float | None = None, out=None, lse=None, workspace=None):
+                scale: float | None = None, out=None, lse=None, workspace=None,
+                check: bool = False):
     """Decode against a paged cache: q [B,Hq,Sq,D] (newest tokens), k_pool/v_pool
     [P,128,Hkv,D], block_table int32 [B,max_pages], seqlens int32 [B].
 
@@ -209,12 +228,14 @@ def attn_decode(q, k_pool, v_pool, block_table, seqlens, causal: bool = False,
                                ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                                _stream(q.device))
     _check(code, "attn_decode")
+    if check:
+        _check_device(q.device, "attn_decode")
     return out, lse
 
 
 def attn_fwd_fp8(q, k, v, q_scale: float = 1.0, k_scale: float = 1.0, v_scale: float = 1.0,
                  causal: bool = False, scale: float | None = None, out=None, lse=None,
-                 window=None):
+                 window=None, check: bool = False):
     """Forward on e4m3 inputs (torch.float8_e4m3fn, D = 128) holding x / scale with
     per-tensor scales; returns O (bf16) and lse of attention on the dequantised inputs."""
     B, Hq, N, D = q.shape
@@ -236,4 +257,6 @@ def attn_fwd_fp8(q, k, v, q_scale: float = 1.0, k_scale: float = 1.0, v_scale: f
                                    float(q_scale), float(k_scale), float(v_scale), wl, wr,
                                    float(scale), _stream(q.device))
     _check(code, "attn_fwd_fp8")
+    if check:
+        _check_device(q.device, "attn_fwd_fp8")
     return out, lse

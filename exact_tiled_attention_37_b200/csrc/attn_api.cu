@@ -46,6 +46,8 @@ std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_debug_flags{0};
 std::atomic<void*> g_bwd_ev_start{nullptr};
 std::atomic<void*> g_bwd_ev_stop{nullptr};
+std::atomic<void*> g_bwd_q_ev_start{nullptr};
+std::atomic<void*> g_bwd_q_ev_stop{nullptr};
 
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {};
@@ -90,6 +92,25 @@ attn_status_t check_tensor(const attn_tensor_t& t, int B, int H, int N, int es) 
   if (t.sb < 0 || t.sh < 0 || t.sn < 0) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(t.ptr)) return ATTN_ERR_MISALIGNED;
   if ((t.sb * es) % 16 || (t.sh * es) % 16 || (t.sn * es) % 16) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+// An output tensor must not overlap itself: otherwise two CTAs write the same
+// elements and the result depends on their order.  Sufficient condition: with
+// the dimensions of extent > 1 sorted by stride (D has stride 1), every stride
+// reaches past the whole span of the dimensions inside it.
+attn_status_t check_output_layout(const attn_tensor_t& t, int B, int H, int N, int D) {
+  struct Dim { long long extent, stride; } d[4] = {{D, 1}, {N, t.sn}, {H, t.sh}, {B, t.sb}};
+  Dim v[4];
+  int n = 0;
+  for (const Dim& x : d)
+    if (x.extent > 1) v[n++] = x;
+  std::sort(v, v + n, [](const Dim& a, const Dim& b) { return a.stride < b.stride; });
+  long long span = 0;  // largest element offset reachable through the inner dimensions
+  for (int i = 0; i < n; ++i) {
+    if (v[i].stride <= span) return ATTN_ERR_INVALID_ARG;
+    span += (v[i].extent - 1) * v[i].stride;
+  }
   return ATTN_OK;
 }
 
@@ -223,6 +244,8 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
   dim3 grid(p.Hkv * C::DSPLIT, p.B, (p.N + C::BC - 1) / C::BC);
   cudaEvent_t ev0 = static_cast<cudaEvent_t>(g_bwd_ev_start.exchange(nullptr));
   cudaEvent_t ev1 = static_cast<cudaEvent_t>(g_bwd_ev_stop.exchange(nullptr));
+  g_bwd_q_ev_start.store(nullptr);  // this form has no separate dQ kernel
+  g_bwd_q_ev_stop.store(nullptr);
   const bool timed = ev0 && ev1;
   if (timed && cudaEventRecord(ev0, st) != cudaSuccess) return ATTN_ERR_CUDA;
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
@@ -273,8 +296,14 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   CUtensorMap tdq;
   const attn_tensor_t dq_t{p.dq, p.dqsb, p.dqsh, p.dqsn};
   if ((s = make_map(&tdq, dq_t, p.B, p.Hq, p.N, D, 2, 32)) != ATTN_OK) return s;
+  cudaEvent_t eq0 = static_cast<cudaEvent_t>(g_bwd_q_ev_start.exchange(nullptr));
+  cudaEvent_t eq1 = static_cast<cudaEvent_t>(g_bwd_q_ev_stop.exchange(nullptr));
+  const bool qtimed = eq0 && eq1;
+  if (qtimed && cudaEventRecord(eq0, st) != cudaSuccess) return ATTN_ERR_CUDA;
   kq<<<dim3(p.Hq, p.B, tiles), CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
-  return last_launch();
+  if ((s = last_launch()) != ATTN_OK) return s;
+  if (qtimed && cudaEventRecord(eq1, st) != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }
 
 // ---------------------------------------------------------------- decode
@@ -386,6 +415,11 @@ void attn_debug_set_bwd_events(void* start, void* stop) {
   g_bwd_ev_stop.store(stop);
 }
 
+void attn_debug_set_bwd_q_events(void* start, void* stop) {
+  g_bwd_q_ev_start.store(start);
+  g_bwd_q_ev_stop.store(stop);
+}
+
 #ifdef ETA_TRACE
 ATTN_API int attn_debug_read_ftrace(void* dst, size_t bytes) {
   if (bytes > sizeof(eta::g_eta_ftrace)) bytes = sizeof(eta::g_eta_ftrace);
@@ -453,6 +487,7 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   if ((s = check_tensor(k, B, Hkv, N, es)) != ATTN_OK) return s;
   if ((s = check_tensor(v, B, Hkv, N, es)) != ATTN_OK) return s;
   if ((s = check_tensor(o, B, Hq, N, es)) != ATTN_OK) return s;
+  if ((s = check_output_layout(o, B, Hq, N, D)) != ATTN_OK) return s;
   if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
 
   eta::FwdParams p;
@@ -509,6 +544,7 @@ attn_status_t attn_fwd_fp8(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, at
   if ((s = check_tensor(k, B, Hkv, N, 1)) != ATTN_OK) return s;
   if ((s = check_tensor(v, B, Hkv, N, 1)) != ATTN_OK) return s;
   if ((s = check_tensor(o, B, Hq, N, 2)) != ATTN_OK) return s;
+  if ((s = check_output_layout(o, B, Hq, N, D)) != ATTN_OK) return s;
   if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
   eta::FwdParams p;
   p.o = o.ptr;
@@ -559,6 +595,7 @@ attn_status_t attn_decode_paged(attn_tensor_t q, attn_tensor_t k_pool, attn_tens
   if ((Hq / Hkv) * Sq > 128 || B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
   if ((s = check_tensor(q, B, Hq, Sq, 2)) != ATTN_OK) return s;
   if ((s = check_tensor(o, B, Hq, Sq, 2)) != ATTN_OK) return s;
+  if ((s = check_output_layout(o, B, Hq, Sq, D)) != ATTN_OK) return s;
   if ((s = check_pool(k_pool, num_pages, Hkv)) != ATTN_OK) return s;
   if ((s = check_pool(v_pool, num_pages, Hkv)) != ATTN_OK) return s;
   if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
@@ -634,6 +671,9 @@ attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   const attn_tensor_t* ks[] = {&k, &v, &dk, &dv};
   for (auto* t : ks)
     if ((s = check_tensor(*t, B, Hkv, N, es)) != ATTN_OK) return s;
+  if ((s = check_output_layout(dq, B, Hq, N, D)) != ATTN_OK) return s;
+  if ((s = check_output_layout(dk, B, Hkv, N, D)) != ATTN_OK) return s;
+  if ((s = check_output_layout(dv, B, Hkv, N, D)) != ATTN_OK) return s;
   if (!aligned16(lse)) return ATTN_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
   if (workspace_bytes < eta::bwd_workspace_bytes(B, Hq, N, D)) return ATTN_ERR_WORKSPACE;

@@ -82,9 +82,11 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int L = p.seqlens[b];
-  // pages of this sequence (a length beyond its block-table row is cut there)
-  const int npages = min(p.max_pages, (L + 127) / 128);
+  // The sequence length, clamped to [0, 128 max_pages] (what its block-table
+  // row can hold): keys and query positions both follow the clamped length.
+  const int L = static_cast<int>(
+      min(static_cast<long long>(max(p.seqlens[b], 0)), 128ll * p.max_pages));
+  const int npages = (L + 127) / 128;  // pages of this sequence
   const int pg0 = split * p.pages_per_split;
   const int n = max(0, min(npages, pg0 + p.pages_per_split) - pg0);  // pages of this CTA
   const int M = p.group * p.Sq;  // real query rows

@@ -43,8 +43,10 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSoftExp8 = ETA_SOFT_EXP8;
 
 #ifdef ETA_TRACE
-// Debug builds only: clock64() timelines of two CTAs of the dQ kernel
-// ([cta][role: elementwise warpgroup 0, 1, MMA][key tile][event]).
+// Debug builds only: clock64() timelines of two CTAs of whichever kernel
+// records them ([cta][role][tile][event]); the macro is defined here so that
+// every kernel header can use it, and today the backward's dQ kernel does
+// (roles: elementwise warpgroups 0 and 1, MMA warp).
 __device__ unsigned long long g_eta_ftrace[2][3][256][4];
 #define ETA_FTRACE_AT(cta, role, it, ev)                                          \
   do {                                                                           \

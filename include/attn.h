@@ -29,14 +29,23 @@
  *   B, Hq, Hkv, N >= 1; Hq % Hkv == 0; D in {64, 128, 256};
  *   every pointer 16-byte aligned and every stride a multiple of 16 bytes
  *   (the tensor-memory-accelerator rule);
- *   ATTN_FP32 (fp32 storage, tf32 tensor-core products) only for the forward
- *   with D = 64; the backward supports bf16 with D in {64, 128, 256}.
+ *   ATTN_FP32 (fp32 storage, products and accumulation in fp32 on the CUDA
+ *   cores, not the tensor cores) only for the forward with D = 64; the
+ *   backward supports bf16 with D in {64, 128, 256};
+ *   an output tensor must not overlap itself (with its dimensions sorted by
+ *   stride, each stride must exceed the span of the dimensions inside it),
+ *   else ATTN_ERR_INVALID_ARG.
  *
  * Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
  * default stream).  The return value reports host-side validation and launch
  * errors only.  A kernel whose internal wait times out (it never hangs: each
  * wait is bounded) records ATTN_ERR_DEVICE_TIMEOUT in a device status word
- * that attn_device_status() reads.
+ * that attn_device_status() reads.  There is one status word per device,
+ * shared by every stream and host thread that calls the library on it: the
+ * first failure since the last read is kept, and attn_device_status() on any
+ * stream returns (and clears) it.  A caller that runs work on several streams
+ * should synchronise all of them before reading it, so that the failure is
+ * attributed to the right batch of calls.
  */
 #ifndef EXACT_TILED_ATTENTION_ATTN_H_
 #define EXACT_TILED_ATTENTION_ATTN_H_
@@ -65,7 +74,7 @@ typedef struct attn_tensor {
 
 typedef enum attn_dtype {
   ATTN_BF16 = 0, /* bf16 storage, fp32 accumulation */
-  ATTN_FP32 = 1  /* fp32 storage, tf32 products, fp32 accumulation */
+  ATTN_FP32 = 1  /* fp32 storage, fp32 products and accumulation (CUDA cores) */
 } attn_dtype_t;
 
 typedef enum attn_status {
@@ -243,7 +252,11 @@ ATTN_API attn_status_t attn_fwd_fp8(attn_tensor_t q, attn_tensor_t k, attn_tenso
  * stride (elements; unit stride on D; 16-byte multiples).  Key t of sequence
  * b is row t % 128 of page block_table[b * max_pages + t / 128] (int32 device
  * array [B][max_pages]); seqlens is an int32 device array [B] with
- * 0 <= seqlens[b] <= 128 * max_pages.  causal != 0: token i sees keys at
+ * 0 <= seqlens[b] <= 128 * max_pages (a length outside that range is clamped
+ * into it: the sequence is taken to hold min(max(seqlens[b], 0),
+ * 128 * max_pages) tokens, for its keys and its query positions alike;
+ * there is no error, since the lengths are device data the host does not
+ * read).  causal != 0: token i sees keys at
  * positions <= its own; otherwise all seqlens[b] keys.  Writes o [B, Hq, Sq,
  * D] (bf16) and lse [B, Hq, Sq] (fp32, natural log, contiguous); a token that
  * sees no key gets o = 0, lse = -inf.
@@ -289,6 +302,13 @@ ATTN_API void attn_debug_set_flags(int flags);
  * this times that kernel alone inside a longer stream of work.
  */
 ATTN_API void attn_debug_set_bwd_events(void* start, void* stop);
+
+/*
+ * The same for the backward's row-parallel dQ kernel (head dimensions 64 and
+ * 128; the D = 256 backward has no such kernel and leaves the events
+ * unrecorded).
+ */
+ATTN_API void attn_debug_set_bwd_q_events(void* start, void* stop);
 
 /*
  * Test hook for the exponential the softmax kernels use: y[i] = 2^x[i] for

@@ -27,7 +27,7 @@ What it computes (the definition, written out, nothing more):
   this oracle does not use the shortcut ``rowsum(dO * O)`` for the row term,
   it sums ``P * dP`` directly.
 
-Readings where the pages are silent (each listed in the design doc): top-left
+Readings where the pages are silent (the plainest ones the rest supports): top-left
 causal alignment with equal query and key lengths; contiguous GQA groups
 (query head h reads key/value head ``h // G``); lse in natural log.
 

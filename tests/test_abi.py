@@ -141,3 +141,22 @@ def test_python_api_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         attn_fwd(q, q, q)
+
+
+def test_overlapping_outputs_are_rejected(L):
+    """An output whose rows (or heads, or batches) overlap would be written by
+    several CTAs in an undefined order: refused before anything is launched."""
+    B, Hq, N, D = 2, 2, 256, 128
+    lse = ctypes.c_void_p(0x20000)
+    q = _t(0x10000, Hq * N * D, N * D, D)
+    for bad in (_t(0x10000, Hq * N * D, N * D, D // 2),       # rows overlap
+                _t(0x10000, Hq * N * D, (N - 1) * D, D),      # heads overlap
+                _t(0x10000, N * D, N * D, D),                 # batches overlap heads
+                _t(0x10000, Hq * N * D, N * D, 0)):           # every row on one
+        assert L.attn_fwd(q, q, q, bad, lse, B, Hq, Hq, N, D, 0, 1, 0.1, None) == 1
+        ws = L.attn_bwd_workspace_bytes(B, Hq, N, D)
+        for slot in range(3):
+            outs = [q, q, q]
+            outs[slot] = bad
+            assert L.attn_bwd(q, q, q, q, lse, q, *outs, B, Hq, Hq, N, D, 0, 1, 0.1,
+                              ctypes.c_void_p(0x40000), ws, None) == 1

@@ -110,3 +110,25 @@ def test_long_context_batch():
                                            seqlens.numpy(), True, 1 / math.sqrt(D), page=PAGE)
         assert rel_err(to_np(o[:, h:h + 1]), o_h) <= TOL_REL
         assert float(np.max(np.abs(to_np(lse[:, h:h + 1]) - l_h))) <= TOL_LSE
+
+
+def test_lengths_outside_the_table_are_clamped():
+    """A length beyond what the block-table row holds (128 * max_pages) is taken
+    as that maximum, for keys and query positions alike, and a negative length
+    as 0 (no key: O = 0, lse = -inf): the result equals the call with the
+    clamped lengths."""
+    lens = [3 * PAGE, 2 * PAGE - 5]
+    q, kp, vp, table, seqlens = make_case(len(lens), 8, 2, 2, 128, lens, seed=123)
+    cap = table.shape[1] * PAGE
+    args = [t.to(DEV) for t in (q, kp, vp, table)]
+    for causal in (False, True):
+        clamped = torch.tensor([cap, 0], dtype=torch.int32)
+        wild = torch.tensor([cap + 1000, -7], dtype=torch.int32)
+        o_c, l_c = attn_decode(*args, clamped.to(DEV), causal=causal)
+        o_w, l_w = attn_decode(*args, wild.to(DEV), causal=causal)
+        torch.cuda.synchronize()
+        assert device_status()[0] == 0
+        assert torch.equal(o_c, o_w)
+        assert torch.equal(l_c, l_w)
+        assert torch.all(o_w[1] == 0) and torch.all(torch.isneginf(l_w[1]))
+        run_and_check(q, kp, vp, table, clamped, causal)

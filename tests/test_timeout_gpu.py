@@ -62,3 +62,26 @@ def test_dropped_bwd_load_times_out_and_recovers(D):
     ref = oracle.attention_bwd(*(to_np(t) for t in (q, k, v, do)), False, 1 / math.sqrt(D))
     for got, r in zip((dq, dk, dv), ref):
         assert rel_err(to_np(got), r) <= TOL_REL
+
+
+@pytest.mark.parametrize("which", ["fwd", "bwd"])
+def test_check_option_raises_on_timeout(which):
+    """check=True turns a device-side timeout into an AttnError at the call
+    (the same dropped loads as above); a normal call with check=True returns."""
+    from exact_tiled_attention_37_b200 import AttnError
+    q, k, v, do = (t.to("cuda") for t in make_random(1, 2, 2, 384, 128, "bf16", seed=8))
+    o, lse = attn_fwd(q, k, v, causal=True, check=True)
+    set_wait_limit_ns(50_000_000)  # 50 ms
+    set_debug_flags(1 if which == "fwd" else 2)
+    try:
+        with pytest.raises(AttnError) as ei:
+            if which == "fwd":
+                attn_fwd(q, k, v, causal=True, check=True)
+            else:
+                attn_bwd(q, k, v, o, lse, do, causal=True, check=True)
+    finally:
+        set_debug_flags(0)
+        set_wait_limit_ns(0)
+    assert ei.value.code == 6
+    assert device_status()[0] == 0  # the failed call's status was read and cleared
+    attn_bwd(q, k, v, o, lse, do, causal=True, check=True)
