@@ -84,6 +84,8 @@ def lib(path: str | None = None) -> ctypes.CDLL:
     L.attn_debug_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     L.attn_debug_set_flags.restype = None
     L.attn_debug_set_flags.argtypes = [i]
+    L.attn_debug_set_fwd_variant.restype = None
+    L.attn_debug_set_fwd_variant.argtypes = [i]
     L.attn_debug_exp2.restype = i
     L.attn_debug_exp2.argtypes = [vp, vp, i, i, vp]
     L.attn_debug_set_bwd_events.restype = None

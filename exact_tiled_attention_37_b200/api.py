@@ -174,6 +174,12 @@ def set_debug_flags(flags: int):
     _lib.lib().attn_debug_set_flags(int(flags))
 
 
+def set_fwd_variant(variant: int):
+    """Forward kernel for bf16 D = 128 without a block mask: 0 default, 1 one
+    CTA per query tile, 2 CTA pairs with 2-CTA tensor-core products."""
+    _lib.lib().attn_debug_set_fwd_variant(int(variant))
+
+
 def _pool_desc(t: torch.Tensor, name: str) -> AttnTensor:
     """[P, 128, Hkv, D] page pool -> (ptr, page stride, head stride, row stride)."""
     if not t.is_cuda:

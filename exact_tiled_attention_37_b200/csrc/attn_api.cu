@@ -17,6 +17,7 @@
 #include "bwd.cuh"
 #include "bwd_split.cuh"
 #include "fwd.cuh"
+#include "fwd_pair.cuh"
 #include "decode.cuh"
 #include "fwd_fp32.cuh"
 
@@ -44,6 +45,9 @@ __global__ void debug_exp2_kernel(const float* __restrict__ x, float* __restrict
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_debug_flags{0};
+// Forward kernel for bf16, D = 128 without a block mask: 0 = the default, 1 =
+// the single-CTA kernel, 2 = the CTA-pair kernel (selectable for comparisons).
+std::atomic<int> g_fwd_variant{0};
 std::atomic<void*> g_bwd_ev_start{nullptr};
 std::atomic<void*> g_bwd_ev_stop{nullptr};
 std::atomic<void*> g_bwd_q_ev_start{nullptr};
@@ -206,6 +210,44 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
   const attn_tensor_t o_t{p.o, p.osb, p.osh, p.osn};
   if ((s = make_map(&to, o_t, B, Hq, N, D, 2, 32)) != ATTN_OK) return s;
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, to, p);
+  return last_launch();
+}
+
+// CTA pairs (tcgen05 .cta_group::2): two query heads of one GQA group when
+// the group size is even, else two adjacent query tiles of one head; a
+// cluster of two CTAs per pair.
+template <int D, int BC, int NS>
+attn_status_t launch_pair(const attn_tensor_t& q, const attn_tensor_t& k, const attn_tensor_t& v,
+                          const eta::FwdParams& p, int B, int Hq, int Hkv, int N,
+                          cudaStream_t st) {
+  using C = eta::PairCfg<D, BC, NS>;
+  CUtensorMap tq, tk, tv, to;
+  attn_status_t s;
+  if ((s = make_tile_map(&tq, q, B, Hq, N, D, 2, 128, C::NCHUNK)) != ATTN_OK) return s;
+  // this CTA's half of a K tile: BC/2 rows, every chunk; of a V tile: every
+  // row, half of the chunks
+  if ((s = make_tile_map(&tk, k, B, Hkv, N, D, 2, C::KROWS, C::NCHUNK)) != ATTN_OK) return s;
+  if ((s = make_tile_map(&tv, v, B, Hkv, N, D, 2, BC, C::VCH)) != ATTN_OK) return s;
+  const attn_tensor_t o_t{p.o, p.osb, p.osh, p.osn};
+  if ((s = make_map(&to, o_t, B, Hq, N, D, 2, 32)) != ATTN_OK) return s;
+  auto kern = eta::fwd_pair_kernel<D, BC, NS>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
+  const int tiles = (N + 127) / 128;
+  const int heads_paired = (Hq / Hkv) % 2 == 0 ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = heads_paired ? dim3(Hq, B, tiles) : dim3(2 * Hq, B, (tiles + 1) / 2);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, p, heads_paired) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   return last_launch();
 }
 
@@ -410,6 +452,10 @@ void attn_debug_set_wait_limit_ns(unsigned long long ns) {
 
 void attn_debug_set_flags(int flags) { g_debug_flags.store(flags); }
 
+void attn_debug_set_fwd_variant(int variant) {
+  g_fwd_variant.store(variant >= 0 && variant <= 2 ? variant : 0);
+}
+
 void attn_debug_set_bwd_events(void* start, void* stop) {
   g_bwd_ev_start.store(start);
   g_bwd_ev_stop.store(stop);
@@ -524,7 +570,10 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   // CTA's loads and epilogue overlap the other's products).
   switch (D) {
     case 64: return launch_single<__nv_bfloat16, 64, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
-    case 128: return launch_single<__nv_bfloat16, 128, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
+    case 128:
+      if (!block_mask && g_fwd_variant.load() == 2)
+        return launch_pair<128, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
+      return launch_single<__nv_bfloat16, 128, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
     default: return launch_single<__nv_bfloat16, 256, 64, 4>(q, k, v, p, B, Hq, Hkv, N, st);
   }
 }

@@ -296,6 +296,18 @@ ATTN_API void attn_debug_set_wait_limit_ns(unsigned long long ns);
 ATTN_API void attn_debug_set_flags(int flags);
 
 /*
+ * Choice of forward kernel for bf16 inputs with D = 128 and no block mask
+ * (other forwards have one kernel each): 0 = the library's default, 1 = one
+ * CTA per 128-row query tile, 2 = pairs of CTAs issuing 2-CTA tensor-core
+ * products (tcgen05 .cta_group::2; FlashAttention entity page, finding
+ * "FlashAttention-4: Algorithm and Kernel Pipelining for Blackwell GPUs":
+ * 2-CTA MMA).  Both give the same results up to rounding order; the switch
+ * exists so that the two can be compared.  Applies to calls made after it,
+ * from any thread; other values select the default.
+ */
+ATTN_API void attn_debug_set_fwd_variant(int variant);
+
+/*
  * Timing hook.  When both are non-NULL (cudaEvent_t handles owned by the
  * caller), the next attn_bwd call records `start` on its stream right before
  * launching its dK/dV kernel and `stop` right after it, then forgets them;
