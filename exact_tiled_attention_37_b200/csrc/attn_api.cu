@@ -205,7 +205,8 @@ attn_status_t launch_single(const attn_tensor_t& q, const attn_tensor_t& k, cons
   auto kern = p.bmask ? eta::fwd_single_kernel<T, D, BC, NS, true>
                       : eta::fwd_single_kernel<T, D, BC, NS, false>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != ATTN_OK) return s;
-  dim3 grid(Hq, B, (N + 127) / 128);
+  const unsigned tiles = static_cast<unsigned>((N + 127) / 128);
+  const dim3 grid = p.head_major ? dim3(tiles, Hq, B) : dim3(Hq, B, tiles);
   CUtensorMap to;  // O as [B, Hq, N, D] bf16 ({64, 32} boxes) for TMA-store epilogues
   const attn_tensor_t o_t{p.o, p.osb, p.osh, p.osn};
   if ((s = make_map(&to, o_t, B, Hq, N, D, 2, 32)) != ATTN_OK) return s;
@@ -342,7 +343,8 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   cudaEvent_t eq1 = static_cast<cudaEvent_t>(g_bwd_q_ev_stop.exchange(nullptr));
   const bool qtimed = eq0 && eq1;
   if (qtimed && cudaEventRecord(eq0, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  kq<<<dim3(p.Hq, p.B, tiles), CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
+  const dim3 qgrid = p.head_major ? dim3(tiles, p.Hq, p.B) : dim3(p.Hq, p.B, tiles);
+  kq<<<qgrid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
   if ((s = last_launch()) != ATTN_OK) return s;
   if (qtimed && cudaEventRecord(eq1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
@@ -418,6 +420,18 @@ attn_status_t launch_decode(const attn_tensor_t& kp, const attn_tensor_t& vp, in
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Sq;
   eta::decode_combine_kernel<D><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);
   return last_launch();
+}
+
+// Grid order of the kernels with one CTA per query tile (forward, dQ): a
+// head's query tiles together when every tile does about the same work (no
+// block mask, and no key range that grows with the query index as under the
+// causal mask), else the longest tiles of every head first.  Measured on B200:
+// the 4x16x2048 non-causal forward 0.1505 -> 0.1413 ms head-major, the
+// 2x16x4096 causal one 0.136 -> 0.165 ms (the late start of each head's
+// longest tile leaves a tail).
+int grid_head_major(int wl, int wr, const uint8_t* block_mask) {
+  if (block_mask) return 0;
+  return (wl < 0 && wr >= 0) ? 0 : 1;
 }
 
 attn_status_t check_sizes(int B, int Hq, int Hkv, int N) {
@@ -555,6 +569,7 @@ attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.o_mul = 1.f;
   p.bmask = block_mask;
   p.nt = (N + 127) / 128;
+  p.head_major = grid_head_major(p.wl, p.wr, block_mask);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!bf16) {
@@ -617,6 +632,7 @@ attn_status_t attn_fwd_fp8(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, at
   p.o_mul = v_scale / eta::kP8Scale;
   p.bmask = nullptr;
   p.nt = (N + 127) / 128;
+  p.head_major = grid_head_major(p.wl, p.wr, nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return launch_single<__nv_fp8_e4m3, 128, 64, 8>(q, k, v, p, B, Hq, Hkv, N, st);
 }
@@ -755,6 +771,7 @@ attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.bmask = block_mask;
   p.nt = (N + 127) / 128;
   p.debug_flags = g_debug_flags.load();
+  p.head_major = grid_head_major(p.wl, p.wr, block_mask);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // per head dimension: Q/dO stages of the dK/dV kernel, K/V ring slots of
   // the dQ kernel, elementwise warpgroups (measured best on B200)

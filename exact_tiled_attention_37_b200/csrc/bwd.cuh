@@ -106,6 +106,7 @@ struct BwdParams {
   const uint8_t* bmask; // block-sparse tile mask [B, Hq, nt, nt] or null (D <= 128 only)
   int nt;               // ceil(N / 128)
   int debug_flags;      // bit 1: the dK/dV producer drops its second Q load (timeout test)
+  int head_major;       // grid order of the dQ kernel (as FwdParams::head_major)
 };
 
 // ---------------------------------------------------------------- preprocess
