@@ -586,7 +586,7 @@ def run_native(args):
                      "flops_per_launch": dom_flops,
                      "algorithmic_bytes": 4 * w.B * w.Hq * w.N * w.D * 2 + 2 * w.B * w.Hkv * w.N * w.D * 2},
         "kernels": {
-            "bwd_q_kernel<128,5,2>": {
+            "bwd_q_kernel<128,3,2,2>": {
                 "launch_ms": round(dq_mean, 4),
                 "method_tflops": round(dq_method, 1),
                 "method_frac_of_burst_peak": round(dq_method / peaks["bf16_tflops"], 4),

@@ -301,12 +301,12 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
 
 // Head dimensions 64 and 128: preprocess, then the column-parallel dK/dV
 // kernel and the row-parallel dQ kernel (no scratch, no atomics).
-template <int D, int NQS, int NS, int NWG>
+template <int D, int NQS, int NK, int NV, int NWG>
 attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
                                const attn_tensor_t& v, const attn_tensor_t& dout,
                                eta::BwdParams& p, cudaStream_t st) {
   using CKV = eta::BwdKVCfg<D, NQS, NWG>;
-  using CQ = eta::BwdQCfg<D, NS, NWG>;
+  using CQ = eta::BwdQCfg<D, NK, NV, NWG>;
   CUtensorMap tq, tk, tv, tdo;
   attn_status_t s;
   if ((s = make_map(&tq, q, p.B, p.Hq, p.N, D, 2, 128)) != ATTN_OK) return s;
@@ -317,7 +317,7 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows / eta::kPrepRows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
   auto kkv = eta::bwd_kv_kernel<D, NQS, NWG>;
-  auto kq = eta::bwd_q_kernel<D, NS, NWG>;
+  auto kq = eta::bwd_q_kernel<D, NK, NV, NWG>;
   if ((s = set_smem(kkv, CKV::SMEM_BYTES)) != ATTN_OK) return s;
   if ((s = set_smem(kq, CQ::SMEM_BYTES)) != ATTN_OK) return s;
   const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128);
@@ -773,10 +773,10 @@ attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.debug_flags = g_debug_flags.load();
   p.head_major = grid_head_major(p.wl, p.wr, block_mask);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // per head dimension: Q/dO stages of the dK/dV kernel, K/V ring slots of
-  // the dQ kernel, elementwise warpgroups (measured best on B200)
-  if (D == 64) return launch_bwd_split<64, 4, 8, 4>(q, k, v, dout, p, st);
-  if (D == 128) return launch_bwd_split<128, 2, 5, 2>(q, k, v, dout, p, st);
+  // per head dimension: Q/dO stages of the dK/dV kernel, K and V ring slots
+  // of the dQ kernel, elementwise warpgroups (measured best on B200)
+  if (D == 64) return launch_bwd_split<64, 4, 5, 3, 4>(q, k, v, dout, p, st);
+  if (D == 128) return launch_bwd_split<128, 2, 3, 2, 2>(q, k, v, dout, p, st);
   return launch_bwd<256, 1, 1>(q, k, v, dout, p, st);
 }
 

@@ -71,7 +71,12 @@ __device__ __forceinline__ void tmem_store_packed(uint32_t taddr, const uint32_t
 }
 
 // ============================================================ dQ kernel
-template <int D, int NS_, int NWG_>
+// K_j is read by S(j) and, last, by dQ(j); V_j only by dP(j), which comes
+// early.  So K and V have rings of their own: V_{j+1} reuses the slot of
+// V_{j-1} (free since dP(j-1)) instead of waiting, in one shared ring, for a
+// K tile that dQ still reads (clock64 timelines of the 4096-token causal
+// backward: the MMA warp waited ~1.5k cycles per key tile for V_{j+1} there).
+template <int D, int NK_, int NV_, int NWG_>
 struct BwdQCfg {
   static constexpr int BM = 128, BN = 128;
   static constexpr int NWG = NWG_, CW = 128 / NWG;
@@ -80,18 +85,20 @@ struct BwdQCfg {
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * ROWB;
   static constexpr int KSTEPS = ROWB / 32;      // S, dP over D
-  static constexpr int NS = NS_;                // K/V ring slots (K_j, V_j alternate)
+  static constexpr int NK = NK_, NV = NV_;      // K ring and V ring slots
   // TMEM: S[2] (128 each; dS bf16 written back) | dP | dQ
   static constexpr int T_S = 0, T_DP = 256, T_DQ = 384, TMEM_COLS = 512;
-  static constexpr int SMEM_Q = 0, SMEM_DO = TILE, SMEM_KV = 2 * TILE;
-  static constexpr int SMEM_BAR = SMEM_KV + NS * TILE;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], dp_full, ds_full[2], dq_done, done,
-  // dp_consumed.  ds_full alternates by key tile: a warp may arrive for tile
-  // u + 1 (it needs only dP(u) loaded by every warp, not dS(u) written)
-  // before the last warp arrives for tile u.
-  static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NS, B_S = 1 + 2 * NS, B_DP = 3 + 2 * NS,
-                       B_DS = 4 + 2 * NS, B_DQ = 6 + 2 * NS, B_DONE = 7 + 2 * NS,
-                       B_DPC = 8 + 2 * NS, NBAR = 9 + 2 * NS;
+  static constexpr int SMEM_Q = 0, SMEM_DO = TILE, SMEM_K = 2 * TILE;
+  static constexpr int SMEM_V = SMEM_K + NK * TILE;
+  static constexpr int SMEM_BAR = SMEM_V + NV * TILE;
+  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
+  // dp_full, ds_full[2], dq_done, done, dp_consumed.  ds_full alternates by
+  // key tile: a warp may arrive for tile u + 1 (it needs only dP(u) loaded by
+  // every warp, not dS(u) written) before the last warp arrives for tile u.
+  static constexpr int B_Q = 0, B_KF = 1, B_KE = 1 + NK, B_VF = 1 + 2 * NK,
+                       B_VE = 1 + 2 * NK + NV, B_S = 1 + 2 * NK + 2 * NV,
+                       B_DP = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 5, B_DONE = B_S + 6,
+                       B_DPC = B_S + 7, NBAR = B_S + 8;
   static constexpr int SMEM_MISC = SMEM_BAR + 8 * NBAR;
   static constexpr int SMEM_BITS = SMEM_MISC + 16;  // block-sparse: computed key tiles
   static constexpr int SMEM_BYTES = SMEM_BITS + 4 * kMaskWords + 1024;
@@ -101,13 +108,13 @@ struct BwdQCfg {
   static_assert(D % (16 * NWG) == 0, "dQ columns per warpgroup");
 };
 
-template <int D, int NS, int NWG>
+template <int D, int NK, int NV, int NWG>
 __global__ void __launch_bounds__(128 * NWG + 64, 1)
     bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_dq,
                  const BwdParams p) {
-  using C = BwdQCfg<D, NS, NWG>;
+  using C = BwdQCfg<D, NK, NV, NWG>;
   constexpr int CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -153,9 +160,13 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_Q), 1);
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(BAR(C::B_KVF + s), 1);
-      mbar_init(BAR(C::B_KVE + s), 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(BAR(C::B_KF + s), 1);
+      mbar_init(BAR(C::B_KE + s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(BAR(C::B_VF + s), 1);
+      mbar_init(BAR(C::B_VE + s), 1);
     }
     mbar_init(BAR(C::B_S + 0), 1);
     mbar_init(BAR(C::B_S + 1), 1);
@@ -218,6 +229,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       }
       if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 1);
       if (!W.wait_warp(BAR(C::B_DP), u & 1, 101)) { ok = false; break; }
+      // dP(u) is complete, so V_u's slot is free: released from here rather
+      // than by a commit of its own
+      if (threadIdx.x == 0) mbar_arrive(BAR(C::B_VE + u % NV));
       if (r == 0) ETA_FTRACE_AT(tcta, par & 1, u, 2);
       tc_fence_after();
       float dp[CW];
@@ -279,23 +293,30 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         tma_load_4d_hint(sbase + C::SMEM_DO + c * C::CHUNK, &tm_do, BAR(C::B_Q), c * 64, q0, h, b,
                          pol_once);
       }
-      int it = 0;
+      int issued_k = 0, issued_v = 0;  // tiles whose K (V) load was issued
       for (int u = 0, j = next_key(jlo); u < n && !W.aborted(); ++u, j = next_key(j + 1)) {
-        for (int kv = 0; kv < 2; ++kv, ++it) {
-          const int slot = it % C::NS;
-          if (!W.wait(BAR(C::B_KVE + slot), (static_cast<uint32_t>(it / C::NS) & 1u) ^ 1u, 110)) break;
-          mbar_expect_tx(BAR(C::B_KVF + slot), C::TILE);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d_hint(sbase + C::SMEM_KV + slot * C::TILE + c * C::CHUNK,
-                             kv ? &tm_v : &tm_k, BAR(C::B_KVF + slot), c * 64, C::BN * j, hk, b,
-                             pol_kv);
-        }
+        const int ks = u % NK, vs = u % NV;
+        if (!W.wait(BAR(C::B_KE + ks), (static_cast<uint32_t>(u / NK) & 1u) ^ 1u, 110)) break;
+        mbar_expect_tx(BAR(C::B_KF + ks), C::TILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d_hint(sbase + C::SMEM_K + ks * C::TILE + c * C::CHUNK, &tm_k,
+                           BAR(C::B_KF + ks), c * 64, C::BN * j, hk, b, pol_kv);
+        issued_k = u + 1;
+        if (!W.wait(BAR(C::B_VE + vs), (static_cast<uint32_t>(u / NV) & 1u) ^ 1u, 113)) break;
+        mbar_expect_tx(BAR(C::B_VF + vs), C::TILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d_hint(sbase + C::SMEM_V + vs * C::TILE + c * C::CHUNK, &tm_v,
+                           BAR(C::B_VF + vs), c * 64, C::BN * j, hk, b, pol_kv);
+        issued_v = u + 1;
       }
-      const int issued = it;
       W.drain(BAR(C::B_Q), 0, 111);
-      for (int s = 0; s < C::NS && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / C::NS) * C::NS;
-        W.drain(BAR(C::B_KVF + s), static_cast<uint32_t>(last / C::NS) & 1u, 112);
+      for (int s = 0; s < NK && s < issued_k; ++s) {
+        const int last = s + ((issued_k - 1 - s) / NK) * NK;
+        W.drain(BAR(C::B_KF + s), static_cast<uint32_t>(last / NK) & 1u, 112);
+      }
+      for (int s = 0; s < NV && s < issued_v; ++s) {
+        const int last = s + ((issued_v - 1 - s) / NV) * NV;
+        W.drain(BAR(C::B_VF + s), static_cast<uint32_t>(last / NV) & 1u, 114);
       }
     }
     __syncwarp();
@@ -305,15 +326,15 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     constexpr uint32_t id_q = idesc_make(128, D, 1u, false, true);     // dQ += dS K
     const SDesc dq_ = sdesc_base(sbase + C::SMEM_Q, 16, 1024);
     const SDesc ddo = sdesc_base(sbase + C::SMEM_DO, 16, 1024);
-    auto kslot = [&](int u) { return (2 * u) % C::NS; };
-    auto kph = [&](int u) { return static_cast<uint32_t>((2 * u) / C::NS) & 1u; };
-    auto vslot = [&](int u) { return (2 * u + 1) % C::NS; };
-    auto vph = [&](int u) { return static_cast<uint32_t>((2 * u + 1) / C::NS) & 1u; };
+    auto kslot = [&](int u) { return u % NK; };
+    auto kph = [&](int u) { return static_cast<uint32_t>(u / NK) & 1u; };
+    auto vslot = [&](int u) { return u % NV; };
+    auto vph = [&](int u) { return static_cast<uint32_t>(u / NV) & 1u; };
     // S(u) = Q K^T into S[u % 2]
     auto issue_s = [&](int u) -> bool {
-      if (!W.wait_warp(BAR(C::B_KVF + kslot(u)), kph(u), 120)) return false;
+      if (!W.wait_warp(BAR(C::B_KF + kslot(u)), kph(u), 120)) return false;
       tc_fence_after();
-      const SDesc kb = sdesc_base(sbase + C::SMEM_KV + kslot(u) * C::TILE, 16, 1024);
+      const SDesc kb = sdesc_base(sbase + C::SMEM_K + kslot(u) * C::TILE, 16, 1024);
       const uint32_t d = tmem + C::T_S + 128 * (u & 1);
 #pragma unroll
       for (int ks = 0; ks < C::KSTEPS; ++ks) {
@@ -325,16 +346,15 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     };
     // dP(u) = dO V^T
     auto issue_dp = [&](int u) -> bool {
-      if (!W.wait_warp(BAR(C::B_KVF + vslot(u)), vph(u), 121)) return false;
+      if (!W.wait_warp(BAR(C::B_VF + vslot(u)), vph(u), 121)) return false;
       tc_fence_after();
-      const SDesc vb = sdesc_base(sbase + C::SMEM_KV + vslot(u) * C::TILE, 16, 1024);
+      const SDesc vb = sdesc_base(sbase + C::SMEM_V + vslot(u) * C::TILE, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < C::KSTEPS; ++ks) {
         const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
         mma_ss_w(tmem + C::T_DP, sdesc_at(ddo, off), sdesc_at(vb, off), id_s, ks > 0);
       }
-      mma_commit_w(BAR(C::B_DP));
-      mma_commit_w(BAR(C::B_KVE + vslot(u)));  // V_u is not read again
+      mma_commit_w(BAR(C::B_DP));  // also frees V_u's slot (elementwise thread 0 arrives)
       return true;
     };
     bool ok = W.wait_warp(BAR(C::B_Q), 0, 122);
@@ -352,13 +372,13 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
       ETA_FTRACE_AT(tcta, 2, u, 0);
       tc_fence_after();
       // dQ += dS K_u: A = dS from TMEM, B = K_u as an MN-major operand (N = D, K = 128 keys)
-      const SDesc kb = sdesc_base(sbase + C::SMEM_KV + kslot(u) * C::TILE, C::CHUNK, 1024);
+      const SDesc kb = sdesc_base(sbase + C::SMEM_K + kslot(u) * C::TILE, C::CHUNK, 1024);
       const uint32_t a = tmem + C::T_S + 128 * (u & 1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         mma_ts_w(tmem + C::T_DQ, a + packed_col<CW>(ks), sdesc_at(kb, ks * 2048), id_q,
                  (u > 0 || ks > 0) ? 1u : 0u);
-      mma_commit_w(BAR(C::B_KVE + kslot(u)));  // K_u is not read again
+      mma_commit_w(BAR(C::B_KE + kslot(u)));  // K_u is not read again
       ETA_FTRACE_AT(tcta, 2, u, 1);
       // S(u + 2) into S[u % 2] after dQ(u) has read dS(u) (issue order)
       if (u + 2 < n && !issue_s(u + 2)) { ok = false; break; }
@@ -416,13 +436,14 @@ struct BwdKVCfg {
   static constexpr int S_STAT = S_P + 128 * 256;               // [NQS] lse2[128], delta[128]
   static constexpr int S_BAR = S_STAT + NQS * 1024;
   // kv (K, V loaded), q_full[NQS] (Q_i and its row statistics), q_empty[NQS],
-  // do_full[NQS], do_empty[NQS], s, s_consumed, dp, p, p_empty, ds,
-  // kv_done (dK, dV complete), done, kv_empty (K, V no longer read)
+  // do_full[NQS], do_empty[NQS] (dV done: dO_i and the P^T tile free), s,
+  // s_consumed, dp, p, ds, kv_done (dK, dV complete), done, kv_empty (K, V no
+  // longer read)
   static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NQS, B_OF = 1 + 2 * NQS,
                        B_OE = 1 + 3 * NQS, B_S = 1 + 4 * NQS, B_SC = 2 + 4 * NQS,
-                       B_DP = 3 + 4 * NQS, B_P = 4 + 4 * NQS, B_PE = 5 + 4 * NQS,
-                       B_DS = 6 + 4 * NQS, B_KVD = 7 + 4 * NQS, B_DONE = 8 + 4 * NQS,
-                       B_KVE = 9 + 4 * NQS, NBAR = 10 + 4 * NQS;
+                       B_DP = 3 + 4 * NQS, B_P = 4 + 4 * NQS, B_DS = 5 + 4 * NQS,
+                       B_KVD = 6 + 4 * NQS, B_DONE = 7 + 4 * NQS, B_KVE = 8 + 4 * NQS,
+                       NBAR = 9 + 4 * NQS;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int S_META = S_MISC + 16;   // [NQS] entry index of each stage
   static constexpr int LAYOUT = S_META + 16;
@@ -521,7 +542,6 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     mbar_init(BAR(C::B_SC), 4 * NWG);
     mbar_init(BAR(C::B_DP), 1);
     mbar_init(BAR(C::B_P), 4 * NWG);
-    mbar_init(BAR(C::B_PE), 1);
     mbar_init(BAR(C::B_DS), 4 * NWG);
     mbar_init(BAR(C::B_KVD), 1);
     mbar_init(BAR(C::B_DONE), 1);
@@ -605,8 +625,13 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
           }
         }
         // the dV MMA of the previous tile must be done reading P^T (and the
-        // epilogue's TMA stores with the staging rows)
-        if (!W.wait_warp(BAR(C::B_PE), (g & 1) ^ 1, 133)) { ok = false; break; }
+        // epilogue's TMA stores with the staging rows): dV(g-1) completing is
+        // what frees entry g-1's dO stage, whose next release needs P^T of a
+        // later entry, so its parity cannot alias
+        if (g > 0 && !W.wait_warp(BAR(C::B_OE + (g - 1) % NQS), ((g - 1) / NQS) & 1, 133)) {
+          ok = false;
+          break;
+        }
         if (kTmaEpi && store_pending) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
@@ -841,8 +866,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         for (int ks = 0; ks < 8; ++ks)
           mma_ss_w(tmem + C::T_DV, sdesc_at(dP, (ks >> 2) * C::CHUNK + (ks & 3) * 32),
                    sdesc_at(ddo, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-        mma_commit_w(BAR(C::B_PE));
-        mma_commit_w(BAR(C::B_OE + stage));  // dO_i is not read again
+        mma_commit_w(BAR(C::B_OE + stage));  // dO_i and P^T are not read again
         ETA_TRACE_AT(tcta, 3, g, 2);
         // dK += dS^T Q_i with dS^T read from TMEM
         if (!W.wait_warp(BAR(C::B_DS), g & 1, 153)) { ok = false; break; }

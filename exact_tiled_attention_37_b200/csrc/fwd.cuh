@@ -455,6 +455,10 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       const int buf = u & 1;
       const uint32_t s_addr = tmem + lane_base + C::S_COL + BC * buf;
       if (!W.wait_warp(BAR(C::BAR_S + buf), (u >> 1) & 1, 10)) { ok = false; break; }
+      // S(u) is complete, so K_u's slot is free: released from here rather
+      // than by a commit of its own (a commit costs the tensor pipe about as
+      // much as a short product)
+      if (threadIdx.x == 0) mbar_arrive(BAR(C::BAR_KVE + (2 * u) % NS));
       tc_fence_after();
       float s[BC];
       tmem_load_row<BC>(s_addr, s);
@@ -574,15 +578,13 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       if (ok) {
         tc_fence_after();
         issue_s(0, kslot(0));
-        mma_commit(BAR(C::BAR_S + 0));
-        mma_commit(BAR(C::BAR_KVE + kslot(0)));
+        mma_commit(BAR(C::BAR_S + 0));  // also frees K_0's slot (softmax warp 0 arrives)
       }
       for (int j = 0; ok && j < n; ++j) {
         if (j + 1 < n) {
           if (!W.wait(BAR(C::BAR_KVF + kslot(j + 1)), kph(j + 1), 42)) { ok = false; break; }
           issue_s((j + 1) & 1, kslot(j + 1));
           mma_commit(BAR(C::BAR_S + ((j + 1) & 1)));
-          mma_commit(BAR(C::BAR_KVE + kslot(j + 1)));
         }
         if (!W.wait(BAR(C::BAR_P + (j & 1)), (j >> 1) & 1, 43)) { ok = false; break; }
         if (!W.wait(BAR(C::BAR_KVF + vslot(j)), vph(j), 44)) { ok = false; break; }
