@@ -16,10 +16,17 @@
 #include "attn.h"
 #include "bwd.cuh"
 #include "bwd_split.cuh"
+#include "bwd_kv3.cuh"
 #include "fwd.cuh"
 #include "fwd_pair.cuh"
 #include "decode.cuh"
 #include "fwd_fp32.cuh"
+
+// Head dimension 128 backward: 1 = the dK/dV kernel with three Q stages
+// (bwd_kv3.cuh), 0 = the two-stage one (bwd_split.cuh), kept for comparison.
+#ifndef ETA_KV3
+#define ETA_KV3 1
+#endif
 
 // Device status word: [0] code, [1] wait site, [2..3] block of the first failure.
 __device__ int g_attn_status[4];
@@ -305,7 +312,10 @@ template <int D, int NQS, int NK, int NV, int NWG>
 attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
                                const attn_tensor_t& v, const attn_tensor_t& dout,
                                eta::BwdParams& p, cudaStream_t st) {
+  // D = 128: the dK/dV kernel with three Q stages (P^T in tensor memory)
+  constexpr bool kKV3 = D == 128 && ETA_KV3;
   using CKV = eta::BwdKVCfg<D, NQS, NWG>;
+  using CKV3 = eta::BwdKV3Cfg<128, 3, 2, 2>;
   using CQ = eta::BwdQCfg<D, NK, NV, NWG>;
   CUtensorMap tq, tk, tv, tdo;
   attn_status_t s;
@@ -316,9 +326,11 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
   eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows / eta::kPrepRows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
-  auto kkv = eta::bwd_kv_kernel<D, NQS, NWG>;
+  auto kkv = kKV3 ? eta::bwd_kv3_kernel<128, 3, 2, 2> : eta::bwd_kv_kernel<D, NQS, NWG>;
+  const int kv_smem = kKV3 ? CKV3::SMEM_BYTES : CKV::SMEM_BYTES;
+  const int kv_threads = kKV3 ? CKV3::THREADS : CKV::THREADS;
   auto kq = eta::bwd_q_kernel<D, NK, NV, NWG>;
-  if ((s = set_smem(kkv, CKV::SMEM_BYTES)) != ATTN_OK) return s;
+  if ((s = set_smem(kkv, kv_smem)) != ATTN_OK) return s;
   if ((s = set_smem(kq, CQ::SMEM_BYTES)) != ATTN_OK) return s;
   const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128);
   cudaEvent_t ev0 = static_cast<cudaEvent_t>(g_bwd_ev_start.exchange(nullptr));
@@ -333,7 +345,7 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   const attn_tensor_t dk_t{p.dk, p.dksb, p.dksh, p.dksn}, dv_t{p.dv, p.dvsb, p.dvsh, p.dvsn};
   if ((s = make_map(&tdk, dk_t, p.B, p.Hkv, p.N, D, 2, 32)) != ATTN_OK) return s;
   if ((s = make_map(&tdv, dv_t, p.B, p.Hkv, p.N, D, 2, 32)) != ATTN_OK) return s;
-  kkv<<<kv_ctas, CKV::THREADS, CKV::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+  kkv<<<kv_ctas, kv_threads, kv_smem, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   if ((s = last_launch()) != ATTN_OK) return s;
   if (timed && cudaEventRecord(ev1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   CUtensorMap tdq;
