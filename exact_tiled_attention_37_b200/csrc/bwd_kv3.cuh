@@ -358,17 +358,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
             const int h = head_of(I, e);
             const int ig0 = qtile_of(I, e) * C::BR;
             const long long srow = static_cast<long long>(I.b * p.Hq + h) * p.Npad + ig0;
-            if (!pok) {
-            } else if (!W.wait(BAR(C::B_OE + os), ((g / NO) & 1) ^ 1, 243)) {
-              pok = false;
-            } else {
-              const uint32_t ofull = BAR(C::B_OF + os);
-              mbar_expect_tx(ofull, C::TILE + 512);
-              for (int c = 0; c < C::NCHUNK; ++c)
-                tma_load_4d_hint(sbase + C::S_DO + os * C::TILE + c * C::CHUNK, &tm_do, ofull,
-                                 c * 64, ig0, h, I.b, l2_policy_evict_last());
-              bulk_load(sbase + C::S_OST + os * 512, p.delta + srow, 512, ofull);
-              issued_do = g + 1;
+            // Q_i first: with three stages its slot is free long before dO_i's
+            // (which waits for dV two tiles back), and S^T(i) needs it first
+            if (pok) {
               bool qfree = W.wait(BAR(C::B_QE + qs), ((g / NQ) & 1) ^ 1, 240);
               if (qfree && ((epi_pending >> qs) & 1u)) {
                 // the stage held an item's last entry: its epilogue's stores
@@ -391,6 +383,19 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
                 bulk_load(sbase + C::S_QST + qs * 512, p.lse2 + srow, 512, full);
                 issued_q = g + 1;
                 if (++done_in_item == nI) epi_pending |= 1u << qs;
+              }
+            }
+            if (pok) {
+              if (!W.wait(BAR(C::B_OE + os), ((g / NO) & 1) ^ 1, 243)) {
+                pok = false;
+              } else {
+                const uint32_t ofull = BAR(C::B_OF + os);
+                mbar_expect_tx(ofull, C::TILE + 512);
+                for (int c = 0; c < C::NCHUNK; ++c)
+                  tma_load_4d_hint(sbase + C::S_DO + os * C::TILE + c * C::CHUNK, &tm_do, ofull,
+                                   c * 64, ig0, h, I.b, l2_policy_evict_last());
+                bulk_load(sbase + C::S_OST + os * 512, p.delta + srow, 512, ofull);
+                issued_do = g + 1;
               }
             }
           }
