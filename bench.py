@@ -41,13 +41,13 @@ WORKLOAD_INDEX = 2  # MHA fwd+bwd B=2 H=16 N=4096 D=128 causal
 METRIC = "attention fwd+bwd TFLOPS (bf16, 1xB200) and % of dense tensor-core peak"
 
 # The dominant kernel of the step: the backward's dK/dV kernel.
-DOMINANT_KERNEL = "bwd_kv_kernel<128,2,2>"
+DOMINANT_KERNEL = "bwd_kv3_kernel<128,3,2,2>"
 # DRAM traffic of one launch of the dK/dV and dQ kernels from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the kernel
 # sources it was taken on; reported as null once the sources change (profiles/
 # holds the capture).
-DOMINANT_TRAFFIC = {"bytes": 197060864, "src_sha": "0eaf90af9f20464b"}
-DQ_TRAFFIC = {"bytes": 196587264, "src_sha": "0eaf90af9f20464b"}
+DOMINANT_TRAFFIC = {"bytes": 190515200, "src_sha": "0932d17c2cb4982f"}
+DQ_TRAFFIC = {"bytes": 197497856, "src_sha": "0932d17c2cb4982f"}
 
 
 def parse_args():
@@ -73,7 +73,7 @@ def dist_info():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "bwd.cuh", "bwd_split.cuh"):
+    for f in ("ptx.cuh", "bwd.cuh", "bwd_split.cuh", "bwd_kv3.cuh"):
         with open(os.path.join(ROOT, "exact_tiled_attention_37_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
