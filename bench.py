@@ -418,9 +418,14 @@ def run_native(args):
 
     K, W = args.steps, args.warmup
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    # per step: step start/stop, dK/dV kernel start/stop, dQ kernel start/stop
-    ev = [tuple(mk() for _ in range(6)) for _ in range(K)]
-    for e in ev:  # create the driver events before the timed region
+    # per step: start/stop
+    ev = [(mk(), mk()) for _ in range(K)]
+    # per-kernel diagnostics (a separate pass: an event recorded between the
+    # dK/dV and dQ kernels would keep the dQ kernel from starting on the SMs
+    # the dK/dV kernel leaves): dK/dV start/stop, dQ start/stop
+    n_diag = max(10, min(K, 50))
+    ev_k = [tuple(mk() for _ in range(4)) for _ in range(n_diag)]
+    for e in ev + ev_k:  # create the driver events before the timed region
         for x in e:
             x.record(stream)
     for _ in range(W):
@@ -433,15 +438,15 @@ def run_native(args):
 
     peaks = load_peaks()
     with ClockSampler(local) as clocks:
-        time.sleep(0.2)
+        # let nvidia-smi finish starting up (its first queries run while it
+        # initialises its monitoring library) before the timed region
+        time.sleep(1.5)
         barrier()
         t_main0 = time.monotonic()
         for i in range(K):
             flush.zero_()
-            s0, s1, m0, m1, d0, d1 = ev[i]
+            s0, s1 = ev[i]
             s0.record(stream)
-            L.attn_debug_set_bwd_events(m0.cuda_event, m1.cuda_event)
-            L.attn_debug_set_bwd_q_events(d0.cuda_event, d1.cuda_event)
             step()
             s1.record(stream)
         barrier()
@@ -450,14 +455,23 @@ def run_native(args):
         code, where = device_status(dev)
         if code != 0:
             raise RuntimeError(f"device status {code} at wait site {where} during timing")
+        # per-kernel times of the dominant backward kernels (same step, hooks on)
+        t0 = time.monotonic()
+        for m0, m1, d0, d1 in ev_k:
+            flush.zero_()
+            L.attn_debug_set_bwd_events(m0.cuda_event, m1.cuda_event)
+            L.attn_debug_set_bwd_q_events(d0.cuda_event, d1.cuda_event)
+            step()
+        torch.cuda.synchronize(dev)
+        clocks.mark("kernels", t0, time.monotonic())
 
         # forward and backward separately (same region shape, fewer steps)
         t0 = time.monotonic()
         fwd_ms = time_calls(lambda: attn_fwd(q, k, v, causal=causal, out=o, lse=lse), flush,
-                            stream, min(K, 50), warm=0)
+                            stream, max(10, min(K, 50)), warm=3)
         bwd_ms = time_calls(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dq, dk=dk,
-                                             dv=dv, workspace=ws), flush, stream, min(K, 50),
-                            warm=0)
+                                             dv=dv, workspace=ws), flush, stream,
+                            max(10, min(K, 50)), warm=3)
         clocks.mark("split", t0, time.monotonic())
         configs = None
         if rank == 0 and not args.no_configs:
@@ -465,9 +479,9 @@ def run_native(args):
             configs = run_configs(dev, flush, stream, peaks["bf16_tflops"], clocks)
             clocks.mark("configs", t0, time.monotonic())
         time.sleep(0.1)
-    step_ms = [a.elapsed_time(b) for a, b, *_ in ev]
-    kv_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    dq_ms = [e[4].elapsed_time(e[5]) for e in ev]
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    kv_ms = [e[0].elapsed_time(e[1]) for e in ev_k]
+    dq_ms = [e[2].elapsed_time(e[3]) for e in ev_k]
     total_ms = sum(step_ms)
 
     # end to end through the public API with host buffers: every step uploads

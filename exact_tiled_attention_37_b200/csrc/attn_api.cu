@@ -356,7 +356,20 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   const bool qtimed = eq0 && eq1;
   if (qtimed && cudaEventRecord(eq0, st) != cudaSuccess) return ATTN_ERR_CUDA;
   const dim3 qgrid = p.head_major ? dim3(tiles, p.Hq, p.B) : dim3(p.Hq, p.B, tiles);
-  kq<<<qgrid, CQ::THREADS, CQ::SMEM_BYTES, st>>>(tq, tk, tv, tdo, tdq, p);
+  // programmatic dependent launch: the dQ kernel's CTAs take the SMs the
+  // persistent dK/dV CTAs leave as they finish (it reads nothing they write);
+  // an event recorded in between (the timing hook) serialises the two
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = qgrid;
+  cfg.blockDim = dim3(CQ::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = CQ::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kq, tq, tk, tv, tdo, tdq, p) != cudaSuccess) return ATTN_ERR_CUDA;
   if ((s = last_launch()) != ATTN_OK) return s;
   if (qtimed && cudaEventRecord(eq1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;

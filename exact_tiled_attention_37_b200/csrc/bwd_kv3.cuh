@@ -96,6 +96,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
 
+  // the dQ kernel that follows reads nothing this kernel writes: let it start
+  // on the SMs this kernel's CTAs leave as they finish
+  grid_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Persistent CTAs over work items (key/value head, batch, key tile), key
   // tile slowest, dealt out in snake order (as bwd_kv_kernel).

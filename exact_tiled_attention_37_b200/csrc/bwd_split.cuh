@@ -396,6 +396,11 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  // Launched as a programmatic dependent of the dK/dV kernel (it reads only
+  // the inputs and the preprocess's statistics, complete before that kernel
+  // started): waiting here, after all the work, makes this grid's completion
+  // imply the dK/dV kernel's, so later work in the stream is ordered after both.
+  grid_dependency_wait();
 }
 
 // Round r of a persistent CTA's static schedule: items sorted by decreasing
@@ -479,6 +484,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
 
+  grid_launch_dependents();  // the dQ kernel that follows does not read our output
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Persistent CTAs: work items (key/value head, batch, key tile) ordered key
   // tile slowest (causal key tile 0, the most work, first) and dealt out in
