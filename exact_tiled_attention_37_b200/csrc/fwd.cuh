@@ -495,11 +495,14 @@ __global__ void __launch_bounds__(256, D <= 128 ? 2 : 1)
       store_empty_row<__nv_bfloat16, D>(p, b, h, qrow);  // O is bf16 for either input
     } else if (ok && W.wait_warp(BAR(C::BAR_O), 0, 20)) {
       tc_fence_after();
-      // O / l through TMA stores ({64, 32} boxes), staged in this warp's rows
-      // of Q's first chunk (every MMA reading Q is complete)
+      // O / l through TMA stores ({64, 32} boxes) staged in this warp's rows of
+      // Q (every MMA reading Q is complete).  bf16: box k in Q's chunk k (one
+      // chunk per 64 columns), so the boxes go out back to back; e4m3 (Q is
+      // one chunk): every box in chunk 0, each waiting for the previous one
+      static_assert(C::FP8 || C::NCHUNK == D / 64, "one Q chunk per output box");
       uint8_t* stage = smem + C::SMEM_Q + warp * 32 * 128;
       tmem_rows_tma_store<D>(o_addr, stage, &tm_o, 0, q0 + warp * 32, h, b,
-                             l > 0.f ? p.o_mul / l : 0.f);
+                             l > 0.f ? p.o_mul / l : 0.f, C::FP8 ? 0u : C::QCHUNK);
       if (qrow < p.N)
         p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] =
             l > 0.f ? m * p.scale + logf(l) : -INFINITY;

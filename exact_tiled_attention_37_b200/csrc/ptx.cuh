@@ -557,21 +557,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // columns (one {64, 32} box) at a time, written into the warp's 4 KB staging
 // region in the box's 128-byte-swizzled layout (row i at 128 i, 16-byte unit
 // u at unit u ^ (i & 7)); lane 0 stores each box at (col0 + c, row0, h, b).
-// The last box may still be reading the staging region on return.
+// stage_stride = 0: every box reuses the one region (waiting until the
+// previous box has been read); otherwise box k stages at stage + k
+// stage_stride, with no wait in between.  The last boxes may still be reading
+// their staging regions on return.
 template <int NC>
 __device__ __forceinline__ void tmem_rows_tma_store(uint32_t taddr, uint8_t* stage,
                                                     const CUtensorMap* m, int col0, int row0,
-                                                    int h, int b, float mul) {
+                                                    int h, int b, float mul,
+                                                    uint32_t stage_stride = 0) {
   static_assert(NC % 64 == 0, "64-column boxes");
   const int lane = threadIdx.x & 31;
-  uint8_t* srow = stage + lane * 128;
 #pragma unroll 1
   for (int c = 0; c < NC; c += 64) {
+    uint8_t* box_stage = stage + (c / 64) * stage_stride;
+    uint8_t* srow = box_stage + lane * 128;
     uint32_t r0[32], r1[32];
     tmem_ld32(taddr + c, r0);
     tmem_ld32(taddr + c + 32, r1);
     tmem_wait_ld();
-    if (c > 0) {
+    if (c > 0 && stage_stride == 0) {
       if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging region
       __syncwarp();
     }
@@ -587,7 +592,7 @@ __device__ __forceinline__ void tmem_rows_tma_store(uint32_t taddr, uint8_t* sta
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_4d(m, smem_u32(stage), col0 + c, row0, h, b);
+      tma_store_4d(m, smem_u32(box_stage), col0 + c, row0, h, b);
       bulk_commit();
     }
   }
