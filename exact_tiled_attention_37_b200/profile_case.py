@@ -14,7 +14,7 @@ import sys
 
 import torch
 
-from . import attn_bwd, attn_decode, attn_fwd, device_status
+from . import attn_bwd, attn_decode, attn_fwd, device_status, set_fwd_variant
 from .inputs import make_inputs, workload
 
 
@@ -41,11 +41,16 @@ def main(argv=None) -> int:
     ap.add_argument("--repeat", type=int, default=1)
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--decode", action="store_true")
+    ap.add_argument("--fwd-variant", type=int, default=0,
+                    help="forward kernel for bf16 D=128: 0 default, 1 one CTA per query tile, "
+                         "2 CTA pairs with 2-CTA products")
     ap.add_argument("--batch", type=int, default=0,
                     help="run only the first BATCH sequences of the workload (smaller captures)")
     args = ap.parse_args(argv)
     if args.decode:
         return decode_case(args.repeat)
+    if args.fwd_variant:
+        set_fwd_variant(args.fwd_variant)
     w = workload(args.workload)
     causal = w.causal[-1]
     ins = make_inputs(w, with_do=w.backward)

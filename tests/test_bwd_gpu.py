@@ -122,3 +122,27 @@ def test_deterministic(D, window):
         again = attn_bwd(q, k, v, o, lse, do, causal=causal, window=window)
         for a, b in zip(first, again):
             assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_work_after_the_backward_is_ordered_after_both_kernels(D):
+    """The dQ kernel may start on SMs the dK/dV kernel leaves (programmatic
+    dependent launch) and could finish first; it waits for the dK/dV grid
+    before it ends, so that work queued next on the stream -- here, zeroing the
+    inputs in place -- cannot run while the dK/dV kernel still reads them.
+    dK and dV must equal those of a call followed by a full synchronisation."""
+    B, H, N = 2, 8, 2048  # enough work per key tile that dQ CTAs start early
+    q, k, v, do = (t.to(DEV) for t in make_random(B, H, H, N, D, "bf16", seed=31))
+    o, lse = attn_fwd(q, k, v, causal=True)
+    ref = attn_bwd(q, k, v, o, lse, do, causal=True)
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in ref]
+    for _ in range(3):
+        qq, kk, vv, dd = (t.clone() for t in (q, k, v, do))
+        dq, dk, dv = attn_bwd(qq, kk, vv, o, lse, dd, causal=True)
+        for t in (qq, kk, vv, dd):  # same stream, right after the call
+            t.zero_()
+        torch.cuda.synchronize()
+        assert device_status()[0] == 0
+        assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+        assert torch.equal(dq, ref[0])
