@@ -75,6 +75,8 @@ def lib(path: str | None = None) -> ctypes.CDLL:
                                     ctypes.c_size_t, vp]
     L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    L.attn_bwd_workspace_bytes_ds.restype = ctypes.c_size_t
+    L.attn_bwd_workspace_bytes_ds.argtypes = [i, i, i, i, i, i]
     L.attn_bwd.restype = i
     L.attn_bwd.argtypes = [T, T, T, T, vp, T, T, T, T, i, i, i, i, i, i, i, f, vp,
                            ctypes.c_size_t, vp]

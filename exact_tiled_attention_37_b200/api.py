@@ -116,14 +116,26 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
 
 
 def bwd_workspace_bytes(B: int, Hq: int, N: int, D: int) -> int:
+    """Smallest workspace attn_bwd accepts (dQ recomputed at D <= 128)."""
     return int(_lib.lib().attn_bwd_workspace_bytes(B, Hq, N, D))
+
+
+def bwd_workspace_bytes_ds(B: int, Hq: int, N: int, D: int, causal: bool = False,
+                           window=None) -> int:
+    """Workspace with which attn_bwd stores dS tiles and sums dQ from them
+    (D = 128; equal to bwd_workspace_bytes where that form does not apply)."""
+    wl, wr = _window(causal, window)
+    return int(_lib.lib().attn_bwd_workspace_bytes_ds(B, Hq, N, D, wl, wr))
 
 
 def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, window=None,
-             block_mask=None, check: bool = False):
+             block_mask=None, check: bool = False, store_ds: bool = True):
     """dQ, dK, dV of attention from the forward's O and lse and the gradient dO
-    (window, block_mask and check as in attn_fwd)."""
+    (window, block_mask and check as in attn_fwd).  Without a workspace one is
+    allocated: with store_ds, large enough for the stored-dS form (see
+    bwd_workspace_bytes_ds), else the smallest one.  A given workspace selects
+    the form by its size."""
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
     if scale is None:
@@ -135,14 +147,15 @@ def attn_bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     if dv is None:
         dv = torch.empty_like(v, memory_format=torch.contiguous_format)
     L = _lib.lib()
+    wl, wr = _window(causal, window)
     need = int(L.attn_bwd_workspace_bytes(B, Hq, N, D))
     if workspace is None:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+        want = int(L.attn_bwd_workspace_bytes_ds(B, Hq, N, D, wl, wr)) if store_ds else need
+        workspace = torch.empty(want, device=q.device, dtype=torch.uint8)
     if workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace too small: {need} bytes needed")
     if not lse.is_contiguous() or lse.dtype != torch.float32:
         raise ValueError("lse must be contiguous fp32")
-    wl, wr = _window(causal, window)
     bm = _block_mask(block_mask, B, Hq, N, q.device)
     code = L.attn_bwd_masked(_desc(q, "q"), _desc(k, "k"), _desc(v, "v"), _desc(o, "o"),
                              ctypes.c_void_p(lse.data_ptr()), _desc(do, "do"), _desc(dq, "dq"),

@@ -17,6 +17,7 @@
 #include "bwd.cuh"
 #include "bwd_split.cuh"
 #include "bwd_kv3.cuh"
+#include "bwd_dqs.cuh"
 #include "fwd.cuh"
 #include "fwd_pair.cuh"
 #include "decode.cuh"
@@ -307,16 +308,20 @@ attn_status_t launch_bwd(const attn_tensor_t& q, const attn_tensor_t& k, const a
 }
 
 // Head dimensions 64 and 128: preprocess, then the column-parallel dK/dV
-// kernel and the row-parallel dQ kernel (no scratch, no atomics).
-template <int D, int NQS, int NK, int NV, int NWG>
+// kernel and the row-parallel dQ kernel (no scratch, no atomics).  With DS
+// (D = 128, p.ds set) the dK/dV kernel also stores every visible dS^T tile and
+// the dQ kernel sums dS K_j from them (bwd_dqs.cuh) instead of recomputing.
+template <int D, int NQS, int NK, int NV, int NWG, bool DS = false>
 attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
                                const attn_tensor_t& v, const attn_tensor_t& dout,
                                eta::BwdParams& p, cudaStream_t st) {
   // D = 128: the dK/dV kernel with three Q stages (P^T in tensor memory)
   constexpr bool kKV3 = D == 128 && ETA_KV3;
+  static_assert(!DS || kKV3, "stored dS tiles come from the three-stage dK/dV kernel");
   using CKV = eta::BwdKVCfg<D, NQS, NWG>;
   using CKV3 = eta::BwdKV3Cfg<128, 3, 2, 2>;
   using CQ = eta::BwdQCfg<D, NK, NV, NWG>;
+  using CQS = eta::BwdDqsCfg<3>;
   CUtensorMap tq, tk, tv, tdo;
   attn_status_t s;
   if ((s = make_map(&tq, q, p.B, p.Hq, p.N, D, 2, 128)) != ATTN_OK) return s;
@@ -326,12 +331,17 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
   eta::bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows / eta::kPrepRows * (D / 8) + 255) / 256), 256, 0, st>>>(p);
   if ((s = last_launch()) != ATTN_OK) return s;
-  auto kkv = kKV3 ? eta::bwd_kv3_kernel<128, 3, 2, 2> : eta::bwd_kv_kernel<D, NQS, NWG>;
+  auto kkv = kKV3 ? eta::bwd_kv3_kernel<128, 3, 2, 2, DS> : eta::bwd_kv_kernel<D, NQS, NWG>;
   const int kv_smem = kKV3 ? CKV3::SMEM_BYTES : CKV::SMEM_BYTES;
   const int kv_threads = kKV3 ? CKV3::THREADS : CKV::THREADS;
   auto kq = eta::bwd_q_kernel<D, NK, NV, NWG>;
+  auto kqs = eta::bwd_dqs_kernel<3>;
   if ((s = set_smem(kkv, kv_smem)) != ATTN_OK) return s;
-  if ((s = set_smem(kq, CQ::SMEM_BYTES)) != ATTN_OK) return s;
+  if (DS) {
+    if ((s = set_smem(kqs, CQS::SMEM_BYTES)) != ATTN_OK) return s;
+  } else {
+    if ((s = set_smem(kq, CQ::SMEM_BYTES)) != ATTN_OK) return s;
+  }
   const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128);
   cudaEvent_t ev0 = static_cast<cudaEvent_t>(g_bwd_ev_start.exchange(nullptr));
   cudaEvent_t ev1 = static_cast<cudaEvent_t>(g_bwd_ev_stop.exchange(nullptr));
@@ -357,19 +367,26 @@ attn_status_t launch_bwd_split(const attn_tensor_t& q, const attn_tensor_t& k,
   if (qtimed && cudaEventRecord(eq0, st) != cudaSuccess) return ATTN_ERR_CUDA;
   const dim3 qgrid = p.head_major ? dim3(tiles, p.Hq, p.B) : dim3(p.Hq, p.B, tiles);
   // programmatic dependent launch: the dQ kernel's CTAs take the SMs the
-  // persistent dK/dV CTAs leave as they finish (it reads nothing they write);
-  // an event recorded in between (the timing hook) serialises the two
+  // persistent dK/dV CTAs leave as they finish (the seven-product one reads
+  // nothing they write; the stored-dS one waits for their completion before
+  // its first read of the tiles); an event recorded in between (the timing
+  // hook) serialises the two
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = qgrid;
-  cfg.blockDim = dim3(CQ::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = CQ::SMEM_BYTES;
+  // the stored-dS dQ kernel is persistent: one CTA per SM (at most one per query tile)
+  const long long q_items = static_cast<long long>(p.Hq) * p.B * tiles;
+  cfg.gridDim = DS ? dim3(static_cast<unsigned>(std::min<long long>(q_items, sm_count())), 1, 1)
+                   : qgrid;
+  cfg.blockDim = dim3(DS ? CQS::THREADS : CQ::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = DS ? CQS::SMEM_BYTES : CQ::SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kq, tq, tk, tv, tdo, tdq, p) != cudaSuccess) return ATTN_ERR_CUDA;
+  const cudaError_t le = DS ? cudaLaunchKernelEx(&cfg, kqs, tk, tdq, p)
+                            : cudaLaunchKernelEx(&cfg, kq, tq, tk, tv, tdo, tdq, p);
+  if (le != cudaSuccess) return ATTN_ERR_CUDA;
   if ((s = last_launch()) != ATTN_OK) return s;
   if (qtimed && cudaEventRecord(eq1, st) != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
@@ -721,6 +738,15 @@ size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D) {
   return eta::bwd_workspace_bytes(B, Hq, N, D);
 }
 
+size_t attn_bwd_workspace_bytes_ds(int B, int Hq, int N, int D, int window_left,
+                                   int window_right) {
+  if (B < 1 || Hq < 1 || N < 1 || D < 1 || window_left < -1 || window_right < -1) return 0;
+  const int wl = window_left >= N ? -1 : window_left, wr = window_right >= N ? -1 : window_right;
+  const size_t ds = eta::ds_bytes(B, Hq, N, D, wl, wr);
+  if (ds == 0) return eta::bwd_workspace_bytes(B, Hq, N, D);
+  return eta::ds_offset(B, Hq, N, D) + ds;
+}
+
 attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
                        const float* lse, attn_tensor_t dout, attn_tensor_t dq, attn_tensor_t dk,
                        attn_tensor_t dv, int B, int Hq, int Hkv, int N, int D,
@@ -797,10 +823,21 @@ attn_status_t attn_bwd_masked(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v,
   p.nt = (N + 127) / 128;
   p.debug_flags = g_debug_flags.load();
   p.head_major = grid_head_major(p.wl, p.wr, block_mask);
+  // stored dS tiles when the workspace holds them (head dimension 128)
+  p.ds = nullptr;
+  p.ds_head = 0;
+  p.ds_tri = 0;
+  p.ds_w = 0;
+  const size_t ds_need = ETA_KV3 ? eta::ds_bytes(B, Hq, N, D, p.wl, p.wr) : 0;
+  if (ds_need > 0 && workspace_bytes >= eta::ds_offset(B, Hq, N, D) + ds_need) {
+    p.ds = reinterpret_cast<uint8_t*>(ws + eta::ds_offset(B, Hq, N, D));
+    eta::ds_layout(N, p.wl, p.wr, &p.ds_tri, &p.ds_w, &p.ds_head);
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // per head dimension: Q/dO stages of the dK/dV kernel, K and V ring slots
   // of the dQ kernel, elementwise warpgroups (measured best on B200)
   if (D == 64) return launch_bwd_split<64, 4, 5, 3, 4>(q, k, v, dout, p, st);
+  if (D == 128 && p.ds) return launch_bwd_split<128, 2, 3, 2, 2, true>(q, k, v, dout, p, st);
   if (D == 128) return launch_bwd_split<128, 2, 3, 2, 2>(q, k, v, dout, p, st);
   return launch_bwd<256, 1, 1>(q, k, v, dout, p, st);
 }

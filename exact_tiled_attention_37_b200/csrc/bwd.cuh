@@ -107,6 +107,13 @@ struct BwdParams {
   int nt;               // ceil(N / 128)
   int debug_flags;      // bit 1: the dK/dV producer drops its second Q load (timeout test)
   int head_major;       // grid order of the dQ kernel (as FwdParams::head_major)
+  // Stored dS^T tiles (head dimension 128, when the workspace holds them):
+  // the dK/dV kernel writes each visible tile's dS^T (bf16, 32 KB) and the
+  // dQ kernel sums dS K_j from them instead of recomputing S and dP.
+  uint8_t* ds;          // null: the dQ kernel recomputes (seven products)
+  long long ds_head;    // tiles per (batch, query head)
+  int ds_tri;           // 1: causal triangle, slot i (i + 1) / 2 + j
+  int ds_w;             // 0: band of ds_w slots per query tile, slot i ds_w + j - j_lo(i)
 };
 
 // ---------------------------------------------------------------- preprocess

@@ -22,9 +22,13 @@
 //
 // Row statistics travel with the tile that needs them: lse2 with Q_i (for
 // P^T), Delta with dO_i (for dS^T).
+//
+// With DS, each elementwise thread also writes its row of every tile's dS^T
+// (64 bf16 values per warpgroup) to the stored-dS scratch, in the layout the
+// dQ kernel of bwd_dqs.cuh copies straight into shared memory.
 #pragma once
 
-#include "bwd_split.cuh"
+#include "bwd_dqs.cuh"
 
 namespace eta {
 
@@ -54,7 +58,8 @@ struct BwdKV3Cfg {
   static constexpr int S_OST = S_QST + NQ * 512;               // [NO] delta[128]
   static constexpr int S_BAR = S_OST + NO * 512;
   // kv (K, V loaded), q_full[NQ] (Q_i, lse2), q_empty[NQ] (dK done),
-  // do_full[NO] (dO_i, Delta), do_empty[NO] (dV done), epi[NQ] (the
+  // do_full[NO] (dO_i, Delta), do_empty[NO] (dK done: Delta is read until
+  // dS^T is complete), epi[NQ] (the
   // epilogue's stores staged in the Q stage have read it), s, s_consumed,
   // dp, p, ds, kv_done (dK, dV complete), done, kv_empty (K, V no longer read)
   static constexpr int B_KV = 0, B_QF = 1, B_QE = 1 + NQ, B_OF = 1 + 2 * NQ,
@@ -74,7 +79,7 @@ struct BwdKV3Cfg {
   static_assert(CW == 64, "P^T and dS^T halves of 32 packed columns");
 };
 
-template <int D, int NQ, int NO, int NWG>
+template <int D, int NQ, int NO, int NWG, bool DS>
 __global__ void __launch_bounds__(128 * NWG + 64, 1)
     bwd_kv3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -82,6 +87,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
                    const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using C = BwdKV3Cfg<D, NQ, NO, NWG>;
   constexpr int CW = C::CW;
+  static_assert(!DS || (D == 128 && CW == 64), "stored dS^T rows of 64 queries per warpgroup");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -96,8 +102,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::S_MISC + 4);
 
-  // the dQ kernel that follows reads nothing this kernel writes: let it start
-  // on the SMs this kernel's CTAs leave as they finish
+  // let the dQ kernel that follows start on the SMs this kernel's CTAs leave
+  // as they finish (with DS it waits for this grid's completion before it
+  // reads the stored tiles)
   grid_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Persistent CTAs over work items (key/value head, batch, key tile), key
@@ -207,7 +214,9 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::B_SC));  // S^T may be overwritten
         const float* lse2 = reinterpret_cast<const float*>(smem + C::S_QST + qs * 512) + CW * par;
-        const int ig0 = qtile_of(I, meta[qs]) * C::BR + CW * par;
+        // (read now: the producer rewrites the slot once dK of this entry is done)
+        const int ecur = meta[qs];
+        const int ig0 = qtile_of(I, ecur) * C::BR + CW * par;
         // window: query ig0 + i sees key jg iff jg - wr <= ig0 + i <= jg + wl
         const int ilo = p.wr < 0 ? -(1 << 30) : jg - p.wr - ig0;
         const int ihi = p.wl < 0 ? (1 << 30) : jg + p.wl - ig0;
@@ -264,6 +273,20 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::B_P));
         if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 1);
+        // stored dS^T (see below): this key's values of the upper 32 queries
+        // now, the lower 32 once they are computed (two bursts of stores)
+        auto ds_row = [&]() -> uint8_t* {
+          return p.ds + ds_slot(p, I.b, head_of(I, ecur), qtile_of(I, ecur), I.kt) * kDsTileBytes +
+                 par * (kDsTileBytes / 2) + j * 16;
+        };
+        if constexpr (DS) {
+          uint8_t* trow = ds_row();
+          const uint64_t pol = l2_policy_evict_first();
+#pragma unroll
+          for (int m = 4; m < 8; ++m)
+            st_global_v4_hint(trow + m * 2048,
+                              make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]), pol);
+        }
         // the lower half
         {
           uint32_t rl[32];
@@ -282,6 +305,19 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::B_DS));
+        if constexpr (DS) {
+          // this key's dS^T values into the stored tile: queries 8 m .. 8 m + 7
+          // of this warpgroup's 64 form query group 8 par + m (2 KB apart),
+          // row j (16 bytes); a warp's 32 keys write 512 contiguous bytes.
+          // The tiles are read back only after this kernel: L2 evict first,
+          // so that they do not push out the Q, dO tiles other CTAs reuse
+          uint8_t* trow = ds_row();
+          const uint64_t pol = l2_policy_evict_first();
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            st_global_v4_hint(trow + m * 2048,
+                              make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]), pol);
+        }
         if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 3);
       }
       if (!ok) break;
@@ -362,7 +398,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
             const int ig0 = qtile_of(I, e) * C::BR;
             const long long srow = static_cast<long long>(I.b * p.Hq + h) * p.Npad + ig0;
             // Q_i first: with three stages its slot is free long before dO_i's
-            // (which waits for dV two tiles back), and S^T(i) needs it first
+            // (which waits for dK two tiles back), and S^T(i) needs it first
             if (pok) {
               bool qfree = W.wait(BAR(C::B_QE + qs), ((g / NQ) & 1) ^ 1, 240);
               if (qfree && ((epi_pending >> qs) & 1u)) {
@@ -486,7 +522,6 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         for (int ks = 0; ks < 8; ++ks)
           mma_ts_w(tmem + C::T_DV, tmem + C::T_DPT + packed_col_hi<CW>(ks),
                    sdesc_at(ddo, ks * 2048), id_kv, ks > 0 ? 1u : acc0);
-        mma_commit_w(BAR(C::B_OE + os));  // dO_i is not read again
         ETA_TRACE_AT(tcta, 3, g, 2);
         // dK += dS^T Q_i with dS^T from TMEM (lower halves)
         if (!W.wait_warp(BAR(C::B_DS), g & 1, 253)) { ok = false; break; }
@@ -497,6 +532,11 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         for (int ks = 0; ks < 8; ++ks)
           mma_ts_w(tmem + C::T_DK, tmem + C::T_DPT + packed_col<CW>(ks), sdesc_at(dq, ks * 2048),
                    id_kv, ks > 0 ? 1u : acc0);
+        // dO_i is last read by dV(i), but its stage also holds Delta_i, which
+        // the elementwise warps read for the second half of dS^T after they
+        // have released P^T (and with it dV(i)): the stage is free only once
+        // their dS^T is in, i.e. after dK(i)
+        mma_commit_w(BAR(C::B_OE + os));
         mma_commit_w(BAR(C::B_QE + qs));  // Q_i (and lse2) are not read again
         if (it + 1 < n) {
           if (!issue_dp(g + 1)) { ok = false; break; }

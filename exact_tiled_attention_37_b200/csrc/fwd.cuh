@@ -268,7 +268,7 @@ __device__ __forceinline__ void store_empty_row(const FwdParams& p, int b, int h
 
 // Keys [lo, hi) that query rows [qs, qe) may see under the window (wl, wr)
 // (-1 = unbounded; the causal mask is (-1, 0)), clipped to [0, N).
-__device__ __forceinline__ int2 window_keys(int qs, int qe, int N, int wl, int wr) {
+__host__ __device__ __forceinline__ int2 window_keys(int qs, int qe, int N, int wl, int wr) {
   const int lo = wl < 0 ? 0 : max(0, qs - wl);
   const int hi = wr < 0 ? N : min(N, qe + wr);
   return make_int2(lo, hi);
@@ -292,7 +292,7 @@ __device__ __forceinline__ void apply_mask(float (&s)[BC], int2 cw) {
 
 // Key-tile range [j_lo, j_hi) of a 128-row query tile starting at qs (empty
 // when the tile lies past N).
-__device__ __forceinline__ int2 key_tiles(int qs, int N, int wl, int wr, int BN) {
+__host__ __device__ __forceinline__ int2 key_tiles(int qs, int N, int wl, int wr, int BN) {
   if (qs >= N) return make_int2(0, 0);
   const int2 kr = window_keys(qs, min(N, qs + 128), N, wl, wr);
   return make_int2(kr.x / BN, (kr.y + BN - 1) / BN);

@@ -213,6 +213,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
 }
+// 16-byte global store with an L2 eviction policy.
+__device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
+}
+
+// bulk_load with an L2 eviction policy.
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
+}
 
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -295,6 +311,17 @@ __device__ __forceinline__ SDesc sdesc_base(uint32_t saddr, uint32_t lbo, uint32
   SDesc d;
   d.lo = ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
   d.hi = ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+  return d;
+}
+// The same for an operand without swizzling (layout type 0): core matrices
+// of 8 rows x 16 bytes, each 128 contiguous bytes; for an MN-major operand
+// lbo is the byte distance between core matrices adjacent along K and sbo
+// the distance between those adjacent along M (or N) (checked on B200
+// against the oracle; the opposite assignment gives wrong products).
+__device__ __forceinline__ SDesc sdesc_base_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  SDesc d;
+  d.lo = ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+  d.hi = ((sbo >> 4) & 0x3FFFu) | (1u << 14);
   return d;
 }
 __device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t byte_off) {

@@ -148,6 +148,23 @@ ATTN_API attn_status_t attn_fwd_masked(attn_tensor_t q, attn_tensor_t k, attn_te
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D);
 
 /*
+ * Bytes of workspace with which attn_bwd (window_left = -1, window_right = 0
+ * for causal, -1 otherwise), attn_bwd_window and attn_bwd_masked with this
+ * window store dS: head dimension 128 only.  The dK/dV kernel then also
+ * writes each visible 128 x 128 tile's dS (bf16, 32 KB per tile: N^2 / 2
+ * bytes per (batch, query head) for the causal mask, up to 2 N^2 for other
+ * windows) into the workspace, and dQ is summed from those tiles (one
+ * product per tile pair) instead of being recomputed with S and dP (three
+ * products per tile pair).  Both forms sum in a fixed order (no atomics) and
+ * are bitwise reproducible.  Equals attn_bwd_workspace_bytes where the
+ * stored form does not apply (D != 128, or more than 4 GiB of tiles); 0 for
+ * invalid sizes or windows.  A smaller workspace (at least
+ * attn_bwd_workspace_bytes) selects the recomputing form.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes_ds(int B, int Hq, int N, int D, int window_left,
+                                            int window_right);
+
+/*
  * Backward.  Reads q, k, v, the forward's o and lse, and the upstream
  * gradient dout [B,Hq,N,D]; writes dq [B,Hq,N,D], dk and dv [B,Hkv,N,D]
  * (bf16).  workspace: device memory of at least attn_bwd_workspace_bytes()
@@ -158,8 +175,11 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int N, int D);
  * (FlashAttention (Metal Port) README, Documentation section): a
  * column-parallel kernel computes dK and dV, a row-parallel kernel computes
  * dQ, every gradient element is summed in one fixed order and the results
- * are bitwise reproducible.  D = 256 uses the five-product form with dQ
- * partial sums added into the fp32 workspace.
+ * are bitwise reproducible.  At D = 128 a workspace of
+ * attn_bwd_workspace_bytes_ds() bytes replaces the row-parallel recomputation
+ * by stored dS tiles (five products per tile pair, still in a fixed order).
+ * D = 256 uses the five-product form with dQ partial sums added into the
+ * fp32 workspace.
  */
 ATTN_API attn_status_t attn_bwd(attn_tensor_t q, attn_tensor_t k, attn_tensor_t v, attn_tensor_t o,
                        const float* lse, attn_tensor_t dout, attn_tensor_t dq, attn_tensor_t dk,

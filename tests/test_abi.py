@@ -57,6 +57,28 @@ def test_workspace_size(L):
     assert L.attn_bwd_workspace_bytes(0, H, N, 128) == 0
 
 
+def test_stored_ds_workspace_size(L):
+    """Stored dS tiles: 32 KB per visible 128 x 128 tile after the row
+    statistics (rounded up to 64 KB); D = 128 only, at most 4 GiB of tiles."""
+    f = L.attn_bwd_workspace_bytes_ds
+    B, H, N = 2, 16, 4096
+    nt = N // 128
+    base = L.attn_bwd_workspace_bytes(B, H, N, 128)
+    off = -(-base // 65536) * 65536
+    assert f(B, H, N, 128, -1, 0) == off + B * H * (nt * (nt + 1) // 2) * 32768   # causal
+    assert f(B, H, N, 128, -1, -1) == off + B * H * nt * nt * 32768               # no mask
+    # a window of 1023 keys to the left: each query tile sees at most 9 key tiles
+    assert f(B, H, N, 128, 1023, 0) == off + B * H * nt * 9 * 32768
+    # sides >= N are unbounded
+    assert f(B, H, N, 128, N, 0) == f(B, H, N, 128, -1, 0)
+    # other head dimensions, or more than 4 GiB of tiles: the smallest workspace
+    assert f(B, H, N, 64, -1, 0) == L.attn_bwd_workspace_bytes(B, H, N, 64)
+    assert f(B, H, N, 256, -1, 0) == L.attn_bwd_workspace_bytes(B, H, N, 256)
+    assert f(1, 32, 32768, 128, -1, 0) == L.attn_bwd_workspace_bytes(1, 32, 32768, 128)
+    assert f(0, H, N, 128, -1, 0) == 0
+    assert f(B, H, N, 128, -2, 0) == 0
+
+
 def _t(ptr, sb, sh, sn):
     return _lib.AttnTensor(ctypes.c_void_p(ptr), sb, sh, sn)
 

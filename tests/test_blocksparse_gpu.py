@@ -38,19 +38,20 @@ def check_lse(got, ref):
         assert float(np.max(np.abs(g[fin] - r[fin]))) <= TOL_LSE
 
 
-def run(q, k, v, do, causal, window, mask, D):
+def run(q, k, v, do, causal, window, mask, D, store_ds=True):
     qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
     bm = torch.from_numpy(mask).to(DEV)
     o, lse = attn_fwd(qd, kd, vd, causal=causal, window=window, block_mask=bm)
-    dq, dk, dv = attn_bwd(qd, kd, vd, o, lse, dod, causal=causal, window=window, block_mask=bm)
+    dq, dk, dv = attn_bwd(qd, kd, vd, o, lse, dod, causal=causal, window=window, block_mask=bm,
+                          store_ds=store_ds)
     torch.cuda.synchronize()
     code, where = device_status()
     assert code == 0, f"device status {code} at wait site {where}"
     return o, lse, dq, dk, dv
 
 
-def check_all(q, k, v, do, causal, window, mask, D):
-    o, lse, dq, dk, dv = run(q, k, v, do, causal, window, mask, D)
+def check_all(q, k, v, do, causal, window, mask, D, store_ds=True):
+    o, lse, dq, dk, dv = run(q, k, v, do, causal, window, mask, D, store_ds)
     args = [t.float().numpy() for t in (q, k, v)]
     scale = 1 / math.sqrt(D)
     o_ref, l_ref = oracle.attention_fwd(*args, causal, scale, window=window, block_mask=mask)
@@ -64,13 +65,13 @@ def check_all(q, k, v, do, causal, window, mask, D):
         assert e <= TOL_REL
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D,store_ds", [(64, True), (128, True), (128, False)])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N,density", [(700, 0.5), (1000, 0.3), (1024, 0.8)])
-def test_random_masks(D, causal, N, density):
+def test_random_masks(D, causal, N, density, store_ds):
     q, k, v, do = make_random(1, 4, 2, N, D, "bf16", seed=N + D + causal)
     mask = make_mask(1, 4, N, density, seed=N * 3 + D, empty_row=1)
-    check_all(q, k, v, do, causal, None, mask, D)
+    check_all(q, k, v, do, causal, None, mask, D, store_ds)
 
 
 @pytest.mark.parametrize("D", [64, 128])

@@ -18,20 +18,20 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def run(q, k, v, do, causal, scale=None):
+def run(q, k, v, do, causal, scale=None, store_ds=True):
     q, k, v, do = (t.to(DEV) for t in (q, k, v, do))
     o, lse = attn_fwd(q, k, v, causal=causal, scale=scale)
-    dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=causal, scale=scale)
+    dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=causal, scale=scale, store_ds=store_ds)
     torch.cuda.synchronize()
     code, where = device_status()
     assert code == 0, f"device status {code} at wait site {where}"
     return dq, dk, dv
 
 
-def check(q, k, v, do, causal, heads=None, scale=None):
+def check(q, k, v, do, causal, heads=None, scale=None, store_ds=True):
     D = q.shape[-1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    dq, dk, dv = run(q, k, v, do, causal, scale)
+    dq, dk, dv = run(q, k, v, do, causal, scale, store_ds)
     ref = oracle.attention_bwd(q.float().numpy(), k.float().numpy(), v.float().numpy(),
                                do.float().numpy(), causal, scale, heads=heads)
     errs = []
@@ -62,6 +62,63 @@ def test_small_shapes(D, causal, N):
 def test_grouped_query_heads(D, causal, hq, hkv):
     q, k, v, do = make_random(2, hq, hkv, 333, D, "bf16", seed=hq * 11 + hkv + D)
     check(q, k, v, do, causal)
+
+
+# Head dimension 128 takes the stored-dS form above (the default workspace
+# holds the tiles); the same cases with the smallest workspace run the
+# seven-product form, whose dQ kernel recomputes S and dP.
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 100, 128, 300, 640])
+def test_small_shapes_recomputed_dq(causal, N):
+    q, k, v, do = make_random(1, 2, 2, N, 128, "bf16", seed=N * 3 + 128 + causal)
+    check(q, k, v, do, causal, store_ds=False)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hq,hkv", [(4, 1), (6, 3)])
+def test_grouped_query_heads_recomputed_dq(causal, hq, hkv):
+    q, k, v, do = make_random(2, hq, hkv, 333, 128, "bf16", seed=hq * 11 + hkv + 128)
+    check(q, k, v, do, causal, store_ds=False)
+
+
+@pytest.mark.parametrize("causal,window", [(True, None), (False, None), (False, (200, 200)),
+                                           (False, (-1, 50))])
+def test_stored_and_recomputed_dq_agree(causal, window):
+    """Both forms compute dK and dV in the same kernel with the same
+    arithmetic (bit for bit), and dQ from the same dS values."""
+    q, k, v, do = (t.to(DEV) for t in make_random(2, 4, 2, 555, 128, "bf16", seed=77))
+    o, lse = attn_fwd(q, k, v, causal=causal, window=window)
+    a = [t.clone() for t in attn_bwd(q, k, v, o, lse, do, causal=causal, window=window)]
+    b = attn_bwd(q, k, v, o, lse, do, causal=causal, window=window, store_ds=False)
+    torch.cuda.synchronize()
+    assert device_status()[0] == 0
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert rel_err(to_np(a[0]), to_np(b[0])) <= 1e-2
+
+
+def test_workspace_size_selects_the_form():
+    """Any workspace of at least the smallest size is accepted; the stored form
+    runs only when the workspace holds the tiles."""
+    from exact_tiled_attention_37_b200 import bwd_workspace_bytes, bwd_workspace_bytes_ds
+    B, H, N, D = 1, 2, 700, 128
+    small = bwd_workspace_bytes(B, H, N, D)
+    big = bwd_workspace_bytes_ds(B, H, N, D, causal=True)
+    assert big > small
+    q, k, v, do = (t.to(DEV) for t in make_random(B, H, H, N, D, "bf16", seed=5))
+    o, lse = attn_fwd(q, k, v, causal=True)
+    outs = []
+    for n in (small, big - 1, big):
+        ws = torch.empty(n, device=DEV, dtype=torch.uint8)
+        outs.append([t.clone() for t in attn_bwd(q, k, v, o, lse, do, causal=True, workspace=ws)])
+    torch.cuda.synchronize()
+    assert device_status()[0] == 0
+    # one byte short of the stored form: the seven-product form, as with the smallest
+    for x, y in zip(outs[0], outs[1]):
+        assert torch.equal(x, y)
+    ref = oracle.attention_bwd(*(t.float().cpu().numpy() for t in (q, k, v, do)), True,
+                               1 / math.sqrt(D))
+    for got, r in zip(outs[2], ref):
+        assert rel_err(to_np(got), r) <= TOL_REL
 
 
 def test_strided_views():
@@ -106,26 +163,26 @@ def test_workload_head_dim_256():
     check(q, k, v, do, False, heads=[(3, 5)])
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D,store_ds", [(64, True), (128, True), (128, False)])
 @pytest.mark.parametrize("window", [None, (64, 300), (200, 200)])
-def test_deterministic(D, window):
+def test_deterministic(D, window, store_ds):
     """For D <= 128 every gradient element is summed in one fixed order (no
     atomics): repeated runs agree bit for bit (which also exposes barrier
     phases that a fast warp could complete for a slow one)."""
     causal = window is None
     q, k, v, do = (t.to(DEV) for t in make_random(2, 4, 2, 777, D, "bf16", seed=31 + D))
     o, lse = attn_fwd(q, k, v, causal=causal, window=window)
-    first = attn_bwd(q, k, v, o, lse, do, causal=causal, window=window)
+    first = attn_bwd(q, k, v, o, lse, do, causal=causal, window=window, store_ds=store_ds)
     first = [t.clone() for t in first]
     assert all(torch.isfinite(t).all() for t in first)
     for _ in range(4):
-        again = attn_bwd(q, k, v, o, lse, do, causal=causal, window=window)
+        again = attn_bwd(q, k, v, o, lse, do, causal=causal, window=window, store_ds=store_ds)
         for a, b in zip(first, again):
             assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("D", [64, 128])
-def test_work_after_the_backward_is_ordered_after_both_kernels(D):
+@pytest.mark.parametrize("D,store_ds", [(64, True), (128, True), (128, False)])
+def test_work_after_the_backward_is_ordered_after_both_kernels(D, store_ds):
     """The dQ kernel may start on SMs the dK/dV kernel leaves (programmatic
     dependent launch) and could finish first; it waits for the dK/dV grid
     before it ends, so that work queued next on the stream -- here, zeroing the
@@ -134,12 +191,12 @@ def test_work_after_the_backward_is_ordered_after_both_kernels(D):
     B, H, N = 2, 8, 2048  # enough work per key tile that dQ CTAs start early
     q, k, v, do = (t.to(DEV) for t in make_random(B, H, H, N, D, "bf16", seed=31))
     o, lse = attn_fwd(q, k, v, causal=True)
-    ref = attn_bwd(q, k, v, o, lse, do, causal=True)
+    ref = attn_bwd(q, k, v, o, lse, do, causal=True, store_ds=store_ds)
     torch.cuda.synchronize()
     ref = [t.clone() for t in ref]
     for _ in range(3):
         qq, kk, vv, dd = (t.clone() for t in (q, k, v, do))
-        dq, dk, dv = attn_bwd(qq, kk, vv, o, lse, dd, causal=True)
+        dq, dk, dv = attn_bwd(qq, kk, vv, o, lse, dd, causal=True, store_ds=store_ds)
         for t in (qq, kk, vv, dd):  # same stream, right after the call
             t.zero_()
         torch.cuda.synchronize()

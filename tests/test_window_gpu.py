@@ -44,14 +44,14 @@ def test_forward_window_fp32(window):
     assert abs_err(to_np(lse), l_ref) <= 1e-4
 
 
-@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("D,store_ds", [(64, True), (128, True), (128, False), (256, True)])
 @pytest.mark.parametrize("window", [(111, 0), (0, 0), (200, 200), (64, 300), (-1, 50)])
-def test_backward_window(D, window):
+def test_backward_window(D, window, store_ds):
     N = 700
     q, k, v, do = make_random(1, 4, 2, N, D, "bf16", seed=D + window[1])
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     o, lse = attn_fwd(qd, kd, vd, window=window)
-    dq, dk, dv = attn_bwd(qd, kd, vd, o, lse, dod, window=window)
+    dq, dk, dv = attn_bwd(qd, kd, vd, o, lse, dod, window=window, store_ds=store_ds)
     assert device_status()[0] == 0
     ref = oracle.attention_bwd(*(t.float().numpy() for t in (q, k, v, do)), False,
                                1 / math.sqrt(D), window=window)
