@@ -40,14 +40,16 @@ sys.path.insert(0, ROOT)
 WORKLOAD_INDEX = 2  # MHA fwd+bwd B=2 H=16 N=4096 D=128 causal
 METRIC = "attention fwd+bwd TFLOPS (bf16, 1xB200) and % of dense tensor-core peak"
 
-# The dominant kernel of the step: the backward's dK/dV kernel.
-DOMINANT_KERNEL = "bwd_kv3_kernel<128,3,2,2>"
+# The dominant kernel of the step: the backward's dK/dV kernel (which also
+# stores the dS tiles the dQ kernel sums from).
+DOMINANT_KERNEL = "bwd_kv3_kernel<128,3,2,2,true>"
+DQ_KERNEL = "bwd_dqs_kernel<3>"
 # DRAM traffic of one launch of the dK/dV and dQ kernels from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the kernel
 # sources it was taken on; reported as null once the sources change (profiles/
 # holds the capture).
-DOMINANT_TRAFFIC = {"bytes": 193995776, "src_sha": "ec89907ddf11d949"}
-DQ_TRAFFIC = {"bytes": 199356160, "src_sha": "ec89907ddf11d949"}
+DOMINANT_TRAFFIC = {"bytes": 826909696, "src_sha": "8e1480aed1ffc738"}
+DQ_TRAFFIC = {"bytes": 590113792, "src_sha": "8e1480aed1ffc738"}
 
 
 def parse_args():
@@ -73,7 +75,7 @@ def dist_info():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "bwd.cuh", "bwd_split.cuh", "bwd_kv3.cuh"):
+    for f in ("ptx.cuh", "bwd.cuh", "bwd_split.cuh", "bwd_kv3.cuh", "bwd_dqs.cuh"):
         with open(os.path.join(ROOT, "exact_tiled_attention_37_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -275,7 +277,7 @@ def run_configs(dev, flush, stream, peak_burst, clocks):
     import torch
 
     from exact_tiled_attention_37_b200 import (attn_bwd, attn_fwd, attn_fwd_fp8,
-                                               bwd_workspace_bytes, device_status)
+                                               bwd_workspace_bytes_ds, device_status)
     from exact_tiled_attention_37_b200.inputs import make_inputs, make_random, workload
 
     out = []
@@ -306,8 +308,8 @@ def run_configs(dev, flush, stream, peak_burst, clocks):
             if "bwd" in passes:
                 do = ins[3]
                 dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-                ws = torch.empty(bwd_workspace_bytes(w.B, w.Hq, w.N, w.D), device=dev,
-                                 dtype=torch.uint8)
+                ws = torch.empty(bwd_workspace_bytes_ds(w.B, w.Hq, w.N, w.D, causal=causal),
+                                 device=dev, dtype=torch.uint8)
                 ms = time_calls(lambda: attn_bwd(q, k, v, o, lse, do, causal=causal, dq=dq, dk=dk,
                                                  dv=dv, workspace=ws), flush, stream,
                                 reps(2.5 * w.fwd_flops(causal) / 1e12))
@@ -322,9 +324,10 @@ def run_configs(dev, flush, stream, peak_burst, clocks):
     q, k, v, do = (t.to(dev) for t in make_inputs(w))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
-    ws = torch.empty(bwd_workspace_bytes(w.B, w.Hq, w.N, w.D), device=dev, dtype=torch.uint8)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for win in ((1023, 0), (111, 0)):
+        ws = torch.empty(bwd_workspace_bytes_ds(w.B, w.Hq, w.N, w.D, window=win), device=dev,
+                         dtype=torch.uint8)
         f = 4.0 * w.D * w.B * w.Hq * visible_pairs(w.N, *win)
         ms = time_calls(lambda: attn_fwd(q, k, v, window=win, out=o, lse=lse), flush, stream, 30)
         entry(f"{w.name}, local window {win}", "fwd", ms, f, {"flops": "visible pairs"})
@@ -353,7 +356,8 @@ def run_configs(dev, flush, stream, peak_burst, clocks):
     bm = torch.from_numpy(np.broadcast_to(tm, (B, H, T, T)).astype(np.uint8).copy()).to(dev)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
-    ws = torch.empty(bwd_workspace_bytes(B, H, N, D), device=dev, dtype=torch.uint8)
+    # (the stored-dS workspace of the unmasked problem covers every mask)
+    ws = torch.empty(bwd_workspace_bytes_ds(B, H, N, D), device=dev, dtype=torch.uint8)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for causal in (False, True):
         pairs = visible_pairs(N, -1, 0 if causal else -1, tm)
@@ -384,7 +388,7 @@ def run_native(args):
     import torch
     import torch.distributed as dist
 
-    from exact_tiled_attention_37_b200 import _lib, attn_bwd, attn_fwd, bwd_workspace_bytes, \
+    from exact_tiled_attention_37_b200 import _lib, attn_bwd, attn_fwd, bwd_workspace_bytes_ds, \
         device_status
     from exact_tiled_attention_37_b200.inputs import make_inputs, workload
 
@@ -402,7 +406,9 @@ def run_native(args):
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(bwd_workspace_bytes(w.B, w.Hq, w.N, w.D), device=dev, dtype=torch.uint8)
+    # the workspace that selects the stored-dS backward (dS tiles of the mask)
+    ws = torch.empty(bwd_workspace_bytes_ds(w.B, w.Hq, w.N, w.D, causal=causal), device=dev,
+                     dtype=torch.uint8)
     flush = torch.empty(256 * 1024 * 1024, device=dev, dtype=torch.uint8)  # > 126 MB L2
     L = _lib.lib()
     stream = torch.cuda.current_stream(dev)
@@ -564,11 +570,16 @@ def run_native(args):
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     sha = kernel_source_sha()
     traffic = DOMINANT_TRAFFIC["bytes"] if DOMINANT_TRAFFIC["src_sha"] == sha else None
-    # dQ kernel: three products (S, dP, dQ) of which the method counts one (dQ)
+    # stored dS tiles (bf16 128 x 128) of the visible tile pairs: written by
+    # the dK/dV kernel, read by the dQ kernel
+    nt = (w.N + 127) // 128
+    ds_bytes = w.B * w.Hq * (nt * (nt + 1) // 2 if causal else nt * nt) * 128 * 128 * 2
+    # dQ kernel: one product per tile pair (dQ += dS K_j), bound by reading
+    # the dS tiles: dS and K in, dQ out
     dq_mean = statistics.mean(dq_ms)
     dq_method = (w.fwd_flops(causal) / 2) / (dq_mean * 1e-3) / 1e12
-    dq_exec = 3 * (w.fwd_flops(causal) / 2) / (dq_mean * 1e-3) / 1e12
-    dq_alg_bytes = 4 * w.B * w.Hq * w.N * w.D * 2 + w.B * w.Hq * w.N * w.D * 2  # Q,K,V,dO in; dQ out
+    dq_alg_bytes = ds_bytes + w.B * w.Hkv * w.N * w.D * 2 + w.B * w.Hq * w.N * w.D * 2
+    dq_gbs = dq_alg_bytes / (dq_mean * 1e-3) / 1e9
     dq_traffic = DQ_TRAFFIC["bytes"] if DQ_TRAFFIC["src_sha"] == sha else None
 
     result = {
@@ -598,14 +609,17 @@ def run_native(args):
                      "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "launch_ms": round(dom_ms, 4),
                      "flops_per_launch": dom_flops,
-                     "algorithmic_bytes": 4 * w.B * w.Hq * w.N * w.D * 2 + 2 * w.B * w.Hkv * w.N * w.D * 2},
+                     # Q, K, V, dO in; dK, dV and the dS tiles out
+                     "algorithmic_bytes": (4 * w.B * w.Hq * w.N * w.D * 2 +
+                                           2 * w.B * w.Hkv * w.N * w.D * 2 + ds_bytes)},
         "kernels": {
-            "bwd_q_kernel<128,3,2,2>": {
+            DQ_KERNEL: {
+                "bound": "hbm",
                 "launch_ms": round(dq_mean, 4),
+                "achieved_gbs": round(dq_gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                "frac": round(dq_gbs / peaks["hbm_gbs"], 4),
                 "method_tflops": round(dq_method, 1),
-                "method_frac_of_burst_peak": round(dq_method / peaks["bf16_tflops"], 4),
-                "executed_tflops": round(dq_exec, 1),
-                "note": "three products (S, dP recomputed; dQ) per tile pair, one counted",
+                "note": "one product per tile pair (dQ += dS K_j) from the stored dS tiles",
                 "traffic": dq_traffic, "algorithmic_bytes": dq_alg_bytes,
                 "traffic_ratio": round(dq_traffic / dq_alg_bytes, 3) if dq_traffic else None},
         },

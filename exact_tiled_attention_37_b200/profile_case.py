@@ -46,6 +46,9 @@ def main(argv=None) -> int:
                          "2 CTA pairs with 2-CTA products")
     ap.add_argument("--batch", type=int, default=0,
                     help="run only the first BATCH sequences of the workload (smaller captures)")
+    ap.add_argument("--recompute-dq", action="store_true",
+                    help="backward with the smallest workspace: the seven-product form, whose "
+                         "dQ kernel recomputes S and dP (default: stored dS tiles at D = 128)")
     args = ap.parse_args(argv)
     if args.decode:
         return decode_case(args.repeat)
@@ -60,7 +63,7 @@ def main(argv=None) -> int:
     for _ in range(args.repeat):
         o, lse = attn_fwd(q, k, v, causal=causal)
         if w.backward and not args.fwd_only:
-            attn_bwd(q, k, v, o, lse, rest[0], causal=causal)
+            attn_bwd(q, k, v, o, lse, rest[0], causal=causal, store_ds=not args.recompute_dq)
     torch.cuda.synchronize()
     code, where = device_status()
     name = w.name + (f" (first {args.batch} sequences)" if args.batch > 0 else "")
