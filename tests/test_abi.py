@@ -79,6 +79,45 @@ def test_stored_ds_workspace_size(L):
     assert f(B, H, N, 128, -2, 0) == 0
 
 
+def _visible_key_tiles(N, wl, wr, i):
+    """Key tiles (128 rows) holding a key that some query of query tile i may
+    see under the window (wl, wr), counted one query and key at a time."""
+    qs = range(128 * i, min(N, 128 * i + 128))
+    tiles = set()
+    for q in qs:
+        lo = 0 if wl < 0 else max(0, q - wl)
+        hi = N - 1 if wr < 0 else min(N - 1, q + wr)
+        tiles.update(range(lo // 128, hi // 128 + 1))
+    return tiles
+
+
+@pytest.mark.parametrize("N", [1, 127, 128, 129, 300, 640, 1000])
+@pytest.mark.parametrize("window", [(-1, 0), (-1, -1), (0, 0), (111, 0), (200, 200), (64, 300),
+                                    (-1, 50), (1023, 0)])
+def test_stored_ds_slots_cover_every_visible_tile(L, N, window):
+    """The stored-dS workspace holds, per (batch, head), one slot per query
+    tile and key tile it must (causal: the triangle; other windows: a band as
+    wide as the widest query tile's run of visible key tiles), checked against
+    tiles counted by brute force."""
+    wl, wr = window
+    wl_n = -1 if wl >= N else wl
+    wr_n = -1 if wr >= N else wr
+    B, H, D = 1, 2, 128
+    nt = -(-N // 128)
+    rows = [_visible_key_tiles(N, wl_n, wr_n, i) for i in range(nt)]
+    for r in rows:  # each query tile sees one contiguous run of key tiles
+        assert not r or max(r) - min(r) + 1 == len(r)
+    if wl_n < 0 and wr_n == 0:
+        slots = nt * (nt + 1) // 2
+        assert [len(r) for r in rows] == [i + 1 for i in range(nt)]
+    else:
+        slots = nt * max(len(r) for r in rows)
+    got = L.attn_bwd_workspace_bytes_ds(B, H, N, D, wl, wr)
+    base = L.attn_bwd_workspace_bytes(B, H, N, D)
+    off = -(-base // 65536) * 65536
+    assert got == off + B * H * slots * 32768
+
+
 def _t(ptr, sb, sh, sn):
     return _lib.AttnTensor(ctypes.c_void_p(ptr), sb, sh, sn)
 
