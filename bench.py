@@ -48,8 +48,8 @@ DQ_KERNEL = "bwd_dqs_kernel<3>"
 # (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the kernel
 # sources it was taken on; reported as null once the sources change (profiles/
 # holds the capture).
-DOMINANT_TRAFFIC = {"bytes": 826909696, "src_sha": "8e1480aed1ffc738"}
-DQ_TRAFFIC = {"bytes": 590113792, "src_sha": "8e1480aed1ffc738"}
+DOMINANT_TRAFFIC = {"bytes": 843696640, "src_sha": "71708753997cd66f"}
+DQ_TRAFFIC = {"bytes": 589824512, "src_sha": "71708753997cd66f"}
 
 
 def parse_args():

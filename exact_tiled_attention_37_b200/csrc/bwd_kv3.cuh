@@ -69,7 +69,8 @@ struct BwdKV3Cfg {
                        NBAR = B_S + 8;
   static constexpr int S_MISC = S_BAR + 8 * NBAR;
   static constexpr int S_META = S_MISC + 16;  // [NQ] entry index of each Q stage
-  static constexpr int LAYOUT = S_META + 16;
+  static constexpr int S_SLOT = S_META + 16;  // [NQ] its stored-dS tile slot (DS)
+  static constexpr int LAYOUT = S_SLOT + 16;
   static constexpr int SMEM_BYTES = LAYOUT + 1024 <= 232448 ? LAYOUT + 1024 : 232448;
   static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;
   static constexpr int THREADS = 128 * NWG + 64;
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
     return c;
   };
   volatile int* meta = reinterpret_cast<volatile int*>(smem + C::S_META);
+  volatile int* slot_of = reinterpret_cast<volatile int*>(smem + C::S_SLOT);
 #ifdef ETA_TRACE
   const int tcta = blockIdx.x == 0 ? 0 : (blockIdx.x == 1 ? 1 : -1);
 #else
@@ -274,18 +276,21 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         if (lane == 0) mbar_arrive(BAR(C::B_P));
         if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 1);
         // stored dS^T (see below): this key's values of the upper 32 queries
-        // now, the lower 32 once they are computed (two bursts of stores)
+        // now, the lower 32 once they are computed (two bursts of stores).
+        // The entry's tile slot comes from the load warp (read before this
+        // thread's dS^T hand-off, after which the stage may be reloaded)
+        int dslot = 0;
         auto ds_row = [&]() -> uint8_t* {
-          return p.ds + ds_slot(p, I.b, head_of(I, ecur), qtile_of(I, ecur), I.kt) * kDsTileBytes +
-                 par * (kDsTileBytes / 2) + j * 16;
+          return p.ds + static_cast<long long>(dslot) * kDsTileBytes + par * (kDsTileBytes / 2) +
+                 j * 16;
         };
         if constexpr (DS) {
+          dslot = slot_of[qs];
           uint8_t* trow = ds_row();
-          const uint64_t pol = l2_policy_evict_first();
 #pragma unroll
           for (int m = 4; m < 8; ++m)
-            st_global_v4_hint(trow + m * 2048,
-                              make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]), pol);
+            *reinterpret_cast<uint4*>(trow + m * 2048) =
+                make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]);
         }
         // the lower half
         {
@@ -308,15 +313,12 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
         if constexpr (DS) {
           // this key's dS^T values into the stored tile: queries 8 m .. 8 m + 7
           // of this warpgroup's 64 form query group 8 par + m (2 KB apart),
-          // row j (16 bytes); a warp's 32 keys write 512 contiguous bytes.
-          // The tiles are read back only after this kernel: L2 evict first,
-          // so that they do not push out the Q, dO tiles other CTAs reuse
+          // row j (16 bytes); a warp's 32 keys write 512 contiguous bytes
           uint8_t* trow = ds_row();
-          const uint64_t pol = l2_policy_evict_first();
 #pragma unroll
           for (int m = 0; m < 4; ++m)
-            st_global_v4_hint(trow + m * 2048,
-                              make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]), pol);
+            *reinterpret_cast<uint4*>(trow + m * 2048) =
+                make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]);
         }
         if (j == 0) ETA_TRACE_AT(tcta, par & 1, g, 3);
       }
@@ -413,6 +415,7 @@ __global__ void __launch_bounds__(128 * NWG + 64, 1)
               } else {
                 ETA_TRACE_AT(tcta, 3, g, 0);
                 meta[qs] = e;
+                if constexpr (DS) slot_of[qs] = static_cast<int>(ds_slot(p, I.b, h, qtile_of(I, e), I.kt));
                 const uint32_t full = BAR(C::B_QF + qs);
                 mbar_expect_tx(full, C::TILE + 512);
                 for (int c = 0; c < C::NCHUNK; ++c)
